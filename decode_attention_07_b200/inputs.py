@@ -1,0 +1,80 @@
+"""Seeded synthetic inputs for decode attention, shared by the CUDA path's
+tests and benchmark and by the CPU oracle's tests.
+
+This module holds no arithmetic of the attention method: it only draws
+normal variates, scales them by the workload's standard deviation, rounds
+them to bf16 (round-to-nearest-even, torch's conversion) and marks padding.
+
+Recipe (for workload w and seed s):
+  1. seqlens: all equal to w.Lmax, or, for a ragged workload, drawn with
+     ``torch.randint(1, w.Lmax + 1, (w.B,))`` from a CPU generator seeded s.
+  2. q, K, V: fp32 ``randn`` from a generator on ``device`` seeded s, in the
+     order q, then K one sequence at a time (b = 0..B-1), then V the same
+     way; each is multiplied by its sigma and rounded to bf16. Drawing one
+     sequence at a time bounds the fp32 temporary to one sequence's cache.
+  3. Padding: with w.nan_pad, K and V positions t >= seqlens[b] are set to
+     NaN, so any read of them would poison the output.
+The same seed gives the same bytes on the same device type; a CPU draw and a
+CUDA draw of one seed differ (different generators), so each comparison
+draws once and hands the same bytes to both sides.
+"""
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from .configs import Workload
+
+
+@dataclass
+class DecodeInputs:
+    workload: Workload
+    seed: int
+    q: torch.Tensor          # [B, Hq, D] bf16
+    k: torch.Tensor          # [B, Hkv, Lmax, D] bf16
+    v: torch.Tensor          # [B, Hkv, Lmax, D] bf16
+    seqlens: torch.Tensor    # [B] int32, same device as q
+    seqlens_host: np.ndarray  # [B] int32 copy on the host
+    scale: float
+
+    def kv_bytes(self) -> int:
+        """Bytes of K and V that lie inside the sequences (t < seqlen)."""
+        w = self.workload
+        return int(self.seqlens_host.astype(np.int64).sum()) * w.Hkv * w.D * 2 * 2
+
+
+def draw_seqlens(w: Workload, seed: int) -> np.ndarray:
+    if not w.ragged:
+        return np.full((w.B,), w.Lmax, dtype=np.int32)
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    return torch.randint(1, w.Lmax + 1, (w.B,), generator=g, dtype=torch.int32).numpy()
+
+
+def make_inputs(w: Workload, seed: int = 0, device="cpu", seqlens=None) -> DecodeInputs:
+    """Draw one workload's tensors. ``seqlens`` (host ints) overrides the
+    drawn lengths, for edge cases."""
+    device = torch.device(device)
+    if seqlens is None:
+        lens = draw_seqlens(w, seed)
+    else:
+        lens = np.asarray(seqlens, dtype=np.int32).reshape(w.B)
+    g = torch.Generator(device=device).manual_seed(int(seed))
+    q = (torch.randn((w.B, w.Hq, w.D), generator=g, device=device) * w.sigma_q).to(torch.bfloat16)
+    k = torch.empty((w.B, w.Hkv, w.Lmax, w.D), dtype=torch.bfloat16, device=device)
+    v = torch.empty_like(k)
+    for dst, sigma in ((k, w.sigma_k), (v, w.sigma_v)):
+        for b in range(w.B):
+            dst[b] = (torch.randn((w.Hkv, w.Lmax, w.D), generator=g, device=device) * sigma).to(torch.bfloat16)
+    if w.nan_pad:
+        for b in range(w.B):
+            L = int(lens[b])
+            if L < w.Lmax:
+                k[b, :, max(L, 0):, :] = float("nan")
+                v[b, :, max(L, 0):, :] = float("nan")
+    seqlens_t = torch.from_numpy(lens.copy()).to(device)
+    return DecodeInputs(w, int(seed), q, k, v, seqlens_t, lens.copy(), w.scale)
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    """The bf16 tensor's bit patterns as a host numpy uint16 array."""
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
