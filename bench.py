@@ -1,0 +1,381 @@
+"""Benchmark: decode attention (split-KV, Flash-Decoding style) on B200.
+
+One step = one fd_decode call (split kernel + combine kernel) over one batch
+of the workload, inputs resident in HBM. Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl fd|reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank decodes its own
+independent batch of the same shape (seed + rank); nothing is exchanged on the
+data path, so scaling is weak and value = sum over ranks of KV bytes / the
+slowest rank's device time.
+
+The reference arm (--impl reference) is the CPU oracle (fp64, host cores) on
+a bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import decode_attention_07_b200 as fd  # noqa: E402
+from decode_attention_07_b200.configs import HEADLINE, WORKLOADS  # noqa: E402
+from decode_attention_07_b200.inputs import bf16_bits, make_inputs  # noqa: E402
+
+METRIC = "decode-attention µs/call and KV-read GB/s as % of B200 HBM peak, 1 GPU"
+NOMINAL_HBM_GBS = 8000.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed work runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[5:9]):
+                if flag.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ byte counts --
+
+def byte_counts(w, lens, S):
+    """Algorithmic bytes of one call: K/V inside the sequences, q, and the
+    outputs / workspace segments each stage writes and reads."""
+    lens = np.clip(lens.astype(np.int64), 0, w.Lmax)
+    kv = int(lens.sum()) * w.Hkv * w.D * 2 * 2
+    q = w.B * w.Hq * w.D * 2
+    seg = fd.fd_segments(w.B, w.Hkv, w.Lmax, lens.astype(np.int32), S)
+    used = seg["row"] >= 0
+    row_bytes = w.g * (w.D + 1) * 4
+    n_whole = int(seg["whole"][used].sum())
+    n_part = int(used.sum()) - n_whole
+    multi_rows = len(set(seg["row"][used & (seg["whole"] == 0)].tolist()))
+    empty_rows = int((lens == 0).sum()) * w.Hkv
+    split_bytes = kv + q + (n_whole + n_part) * row_bytes + w.B * 4
+    combine_bytes = n_part * row_bytes + (multi_rows + empty_rows) * row_bytes + w.B * 4
+    return dict(kv=kv, q=q, split=split_bytes, combine=combine_bytes, total=split_bytes + combine_bytes,
+                segments=n_part, whole_rows=n_whole, multi_rows=multi_rows)
+
+
+# ------------------------------------------------------------- the CPU arm --
+
+def oracle_sample(x, budget_s=12.0, nthreads=0):
+    """Time the CPU oracle on a bounded sample of the workload: whole
+    (sequence, kv-head) rows, all of their query heads, until about
+    `budget_s` seconds of work. Returns (kv_bytes_processed, seconds,
+    threads, description)."""
+    import oracle
+    w = x.workload
+    order = np.argsort(-x.seqlens_host, kind="stable")     # longest sequences first: full-length rows
+    done_bytes, spent, rows, threads = 0, 0.0, 0, 0
+    host = {}
+    for b in order:
+        L = int(min(max(x.seqlens_host[b], 0), w.Lmax))
+        if L == 0:
+            continue
+        for j in range(w.Hkv):
+            key = (int(b), j)
+            if key not in host:
+                host[key] = (bf16_bits(x.q[b:b + 1, j * w.g:(j + 1) * w.g]), bf16_bits(x.k[b:b + 1, j:j + 1, :L]),
+                             bf16_bits(x.v[b:b + 1, j:j + 1, :L]))
+            qh, kh, vh = host[key]
+            orc = oracle.default()
+            t0 = time.perf_counter()
+            orc.attention(qh, kh, vh, np.array([L], np.int32), x.scale, nthreads)
+            spent += time.perf_counter() - t0
+            threads = max(threads, orc.threads_used)
+            done_bytes += L * w.D * 2 * 2
+            rows += 1
+            if spent >= budget_s:
+                break
+        if spent >= budget_s:
+            break
+    desc = f"{rows} (sequence, kv-head) rows x {w.g} query heads of {w.name} seed {x.seed}, longest sequences first"
+    return done_bytes, spent, threads, desc
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    x = make_inputs(w, args.seed, device="cuda" if torch.cuda.is_available() else "cpu")
+    per_step = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(x, budget_s=per_step)
+    total_b, total_s, threads, desc = 0, 0.0, 0, ""
+    for _ in range(args.steps):
+        b, s, t, desc = oracle_sample(x, budget_s=per_step)
+        total_b += b
+        total_s += s
+        threads = max(threads, t)
+    gbs = total_b / total_s / 1e9
+    kv_full = int(np.clip(x.seqlens_host, 0, w.Lmax).astype(np.int64).sum()) * w.Hkv * w.D * 4
+    line = {
+        "metric": METRIC, "impl": "reference", "value": gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": kv_full / (gbs * 1e9) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w, None, "n/a (host memory)"),
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w, S, l2):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "Lmax": w.Lmax,
+            "ragged": w.ragged, "num_splits": S, "l2": l2, "description": w.description}
+
+
+# ------------------------------------------------------------- the GPU arm --
+
+def run_fd(args, w, rank, world):
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.Lmax)
+    xs = [make_inputs(w, args.seed + rank, device=dev)]
+    kv_per_copy = xs[0].kv_bytes()
+    if kv_per_copy >= L2_BYTES:
+        # rotate input copies so every call streams bytes that are not in L2
+        n_copies = 2
+        l2_note = f"inputs larger than L2: {n_copies} input copies of {kv_per_copy / 1e6:.0f} MB rotated"
+    else:
+        n_copies = 1
+        l2_note = "L2 flushed before every timed call (256 MiB write outside the timed events)"
+    for c in range(1, n_copies):
+        xs.append(make_inputs(w, args.seed + rank + 1000 * c, device=dev))
+    nbytes = fd.fd_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, w.Lmax, S)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if n_copies == 1 else None
+    counts = byte_counts(w, xs[0].seqlens_host, S)
+    kv_bytes = sum(x.kv_bytes() for x in xs) / n_copies
+
+    def call(x):
+        fd.fd_decode(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for i in range(max(3, args.warmup)):
+        call(xs[i % n_copies])
+    torch.cuda.synchronize(dev)
+
+    # ---- main timed region: K calls, one event pair per call -------------
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(i & 255)
+            ev[i][0].record(stream)
+            call(xs[i % n_copies])
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        # keep the sampler on the same work for >= 1.5 s so clocks are seen under load
+        t_min = time.perf_counter() + 1.5
+        j = 0
+        while time.perf_counter() < t_min:
+            for _ in range(50):
+                call(xs[j % n_copies])
+                j += 1
+            torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - t_wall
+    barrier()
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    us_per_call = ms_max * 1e3 / args.steps
+    gbs = world * kv_bytes * args.steps / (ms_max * 1e-3) / 1e9
+
+    # ---- per-stage device time (split kernel alone, then combine alone) ----
+    ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+             torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        x = xs[i % n_copies]
+        if flush is not None:
+            flush.fill_(i & 255)
+        ev_s[i][0].record(stream)
+        fd.fd_split(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream)
+        ev_s[i][1].record(stream)
+        fd.fd_combine(w.B, w.Hq, w.Hkv, w.D, w.Lmax, x.seqlens, out, lse, ws, S, stream)
+        ev_s[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    split_us = 1e3 * sum(a.elapsed_time(b) for a, b, _ in ev_s) / args.steps
+    combine_us = 1e3 * sum(b.elapsed_time(c) for _, b, c in ev_s) / args.steps
+
+    # ---- end to end: host buffers in, host buffers out ---------------------
+    e2e = None
+    if not args.no_e2e:
+        x = xs[0]
+        hq, hk, hv = x.q.cpu().pin_memory(), x.k.cpu().pin_memory(), x.v.cpu().pin_memory()
+        hs = x.seqlens.cpu().pin_memory()
+        dq, dk, dv, dsq = (torch.empty_like(t) for t in (x.q, x.k, x.v, x.seqlens))
+        ho = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32).pin_memory()
+        hl = torch.empty((w.B, w.Hq), dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs))
+        d2h = ho.numel() * 4 + hl.numel() * 4
+        e_steps = max(3, min(args.steps, 20))
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dsq.copy_(hs, non_blocking=True)
+            fd.fd_decode(dq, dk, dv, dsq, x.scale, out, lse, ws, stream)
+            ho.copy_(out, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(ems, op=torch.distributed.ReduceOp.MAX)
+        e2e = {"value": world * x.kv_bytes() * e_steps / (float(ems.item()) * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
+               "us_per_call": float(ems.item()) * 1e3 / e_steps}
+
+    status = fd.fd_device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {fd.fd_strerror(status)}")
+
+    if rank != 0:
+        return 0
+    peak, peak_kind = peaks()
+    split_gbs = counts["split"] / (split_us * 1e-6) / 1e9
+    line = {
+        "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_max / args.steps, "us_per_call": us_per_call,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(w, S, l2_note),
+        "pct_of_nominal_hbm": 100.0 * gbs / world / NOMINAL_HBM_GBS,
+        "pct_of_measured_copy": 100.0 * gbs / world / peak,
+        "call_bytes_gbs": world * counts["total"] * args.steps / (ms_max * 1e-3) / 1e9,
+        "roofline": {"kernel": "fd_split_kernel", "bound": "hbm", "achieved": split_gbs, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": split_gbs / peak, "traffic": None,
+                     "bytes_per_launch": counts["split"], "us_per_launch": split_us,
+                     "combine_us_per_launch": combine_us},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "wall_s": wall,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        b, s, t, desc = oracle_sample(xs[0], budget_s=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": b / s / 1e9, "unit": "GB/s", "cores": t, "kind": "oracle",
+                                "sample": desc, "seconds": s}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["fd", "reference"], default="fd")
+    ap.add_argument("--config", choices=list(WORKLOADS), default=HEADLINE)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    w = WORKLOADS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    rank = int(os.environ.get("RANK", 0))
+    if world > 1 and args.impl == "fd":
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            return run_reference(args, w, rank, world)
+        return run_fd(args, w, rank, world)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

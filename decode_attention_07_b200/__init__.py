@@ -1,2 +1,10 @@
-"""B200-native split-KV decode attention (Flash-Decoding) behind a C ABI."""
+"""B200-native split-KV decode attention (Flash-Decoding) behind a C ABI.
+
+The computation lives in libfdecode.so (CUDA, sm_100a; declared in
+include/fd.h). This package is its thin binding (same entry-point names) plus
+the workload table and the seeded input generator."""
 from . import configs, inputs  # noqa: F401
+from ._lib import (  # noqa: F401
+    FdError, decode, fd_combine, fd_decode, fd_decode_splits, fd_device_status, fd_plan, fd_plan_for_sms,
+    fd_segments, fd_split, fd_strerror, fd_version, fd_workspace_bytes, lib, workspace_layout,
+)

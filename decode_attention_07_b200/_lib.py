@@ -1,0 +1,206 @@
+"""ctypes binding over libfdecode.so: the C ABI of include/fd.h with the same
+names, taking torch tensors. Argument marshalling only -- every step of the
+computation runs in the library's CUDA kernels. There is no fallback: if the
+library is missing or a call fails, an exception is raised."""
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(PKG, "libfdecode.so")
+
+FD_OK = 0
+FD_TILE_TOKENS = 64
+FD_MAX_SPLITS = 65535
+FD_MAX_GROUP = 16
+ERRORS = {
+    -1: "FD_ERR_NULL_POINTER", -2: "FD_ERR_SHAPE", -3: "FD_ERR_GROUP", -4: "FD_ERR_HEAD_DIM",
+    -5: "FD_ERR_ALIGNMENT", -6: "FD_ERR_WORKSPACE", -7: "FD_ERR_SPLITS", -8: "FD_ERR_DEVICE",
+    -9: "FD_ERR_LAUNCH", -10: "FD_ERR_TIMEOUT", -11: "FD_ERR_CAPACITY",
+}
+
+
+class FdError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {ERRORS.get(code, code)} ({fd_strerror(code)})")
+
+
+_lib = None
+_i, _p, _sz, _f = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfdecode.so (built in-tree by decode_attention_07_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIBRARY):
+            raise RuntimeError(f"{LIBRARY} is not built: run `python -c 'import __graft_entry__ as g; g.build()'`")
+        L = ctypes.CDLL(LIBRARY)
+        L.fd_plan.argtypes = [_i] * 5
+        L.fd_plan_for_sms.argtypes = [_i] * 6
+        L.fd_workspace_bytes.argtypes = [_i] * 6
+        L.fd_workspace_bytes.restype = _sz
+        compute = [_i] * 5 + [_p, _p, _p, _p, _f, _p, _p, _p, _sz]
+        L.fd_decode.argtypes = compute + [_p]
+        L.fd_decode_splits.argtypes = compute + [_i, _p]
+        L.fd_split.argtypes = compute + [_i, _p]
+        L.fd_combine.argtypes = [_i] * 5 + [_p, _p, _p, _p, _sz, _i, _p]
+        L.fd_segments.argtypes = [_i, _i, _i, _p, _i, _p, _p, _p, _p, _i]
+        L.fd_device_status.argtypes = [_p]
+        L.fd_strerror.argtypes = [_i]
+        L.fd_strerror.restype = ctypes.c_char_p
+        L.fd_version.argtypes = []
+        for name in ("fd_plan", "fd_plan_for_sms", "fd_decode", "fd_decode_splits", "fd_split", "fd_combine",
+                     "fd_segments", "fd_device_status", "fd_version"):
+            getattr(L, name).restype = _i
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str) -> int:
+    if rc < 0:
+        raise FdError(rc, what)
+    return rc
+
+
+def _stream(stream, device) -> int:
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _shapes(q, k_cache, v_cache):
+    if q.dim() != 3 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("expected q [B,Hq,D] and k_cache, v_cache [B,Hkv,Lmax,D]")
+    B, Hq, D = q.shape
+    B2, Hkv, Lmax, D2 = k_cache.shape
+    if B2 != B or D2 != D:
+        raise ValueError("q and the caches disagree on B or D")
+    for t, name in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    return B, Hq, Hkv, D, Lmax
+
+
+def _outputs(out, lse, B, Hq, D):
+    if out.shape != (B, Hq, D) or lse.shape != (B, Hq):
+        raise ValueError("out must be [B,Hq,D] and lse [B,Hq]")
+    for t, name in ((out, "out"), (lse, "lse")):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor")
+
+
+def _seqlens(seqlens, B):
+    if seqlens.shape != (B,) or seqlens.dtype != torch.int32 or not seqlens.is_cuda:
+        raise ValueError("seqlens must be an int32 CUDA tensor of shape [B]")
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
+# ---------------------------------------------------------------- the ABI --
+
+def fd_plan(B: int, Hq: int, Hkv: int, D: int, max_len: int) -> int:
+    return _check(lib().fd_plan(B, Hq, Hkv, D, max_len), "fd_plan")
+
+
+def fd_plan_for_sms(B: int, Hq: int, Hkv: int, D: int, max_len: int, num_sms: int) -> int:
+    return _check(lib().fd_plan_for_sms(B, Hq, Hkv, D, max_len, num_sms), "fd_plan_for_sms")
+
+
+def fd_workspace_bytes(B: int, Hq: int, Hkv: int, D: int, max_len: int, num_splits: int) -> int:
+    return int(lib().fd_workspace_bytes(B, Hq, Hkv, D, max_len, num_splits))
+
+
+def fd_decode(q, k_cache, v_cache, seqlens, scale, out, lse, workspace=None, stream=None):
+    B, Hq, Hkv, D, Lmax = _shapes(q, k_cache, v_cache)
+    _outputs(out, lse, B, Hq, D)
+    _seqlens(seqlens, B)
+    wp, wb = _ws(workspace)
+    _check(lib().fd_decode(B, Hq, Hkv, D, Lmax, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                           seqlens.data_ptr(), float(scale), out.data_ptr(), lse.data_ptr(), wp, wb,
+                           _stream(stream, q.device)), "fd_decode")
+
+
+def fd_decode_splits(q, k_cache, v_cache, seqlens, scale, out, lse, workspace, num_splits, stream=None):
+    B, Hq, Hkv, D, Lmax = _shapes(q, k_cache, v_cache)
+    _outputs(out, lse, B, Hq, D)
+    _seqlens(seqlens, B)
+    wp, wb = _ws(workspace)
+    _check(lib().fd_decode_splits(B, Hq, Hkv, D, Lmax, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                  seqlens.data_ptr(), float(scale), out.data_ptr(), lse.data_ptr(), wp, wb,
+                                  int(num_splits), _stream(stream, q.device)), "fd_decode_splits")
+
+
+def fd_split(q, k_cache, v_cache, seqlens, scale, out, lse, workspace, num_splits, stream=None):
+    B, Hq, Hkv, D, Lmax = _shapes(q, k_cache, v_cache)
+    _outputs(out, lse, B, Hq, D)
+    _seqlens(seqlens, B)
+    wp, wb = _ws(workspace)
+    _check(lib().fd_split(B, Hq, Hkv, D, Lmax, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                          seqlens.data_ptr(), float(scale), out.data_ptr(), lse.data_ptr(), wp, wb,
+                          int(num_splits), _stream(stream, q.device)), "fd_split")
+
+
+def fd_combine(B, Hq, Hkv, D, max_len, seqlens, out, lse, workspace, num_splits, stream=None):
+    _outputs(out, lse, B, Hq, D)
+    _seqlens(seqlens, B)
+    wp, wb = _ws(workspace)
+    _check(lib().fd_combine(B, Hq, Hkv, D, max_len, seqlens.data_ptr(), out.data_ptr(), lse.data_ptr(), wp, wb,
+                            int(num_splits), _stream(stream, out.device)), "fd_combine")
+
+
+def fd_segments(B: int, Hkv: int, max_len: int, seqlens_host, num_splits: int) -> dict:
+    """Where the split stage cuts each row (host computation). Returns numpy
+    arrays indexed by workspace slot: row (-1 = unused), begin, end, whole."""
+    lens = np.ascontiguousarray(np.asarray(seqlens_host, dtype=np.int32).reshape(B))
+    cap = num_splits + B * Hkv - 1
+    arrs = [np.zeros(cap, np.int32) for _ in range(4)]
+    n = _check(lib().fd_segments(B, Hkv, max_len, lens.ctypes.data, int(num_splits),
+                                 *(a.ctypes.data for a in arrs), cap), "fd_segments")
+    return dict(row=arrs[0][:n], begin=arrs[1][:n], end=arrs[2][:n], whole=arrs[3][:n])
+
+
+def fd_device_status(stream=None, device=None) -> int:
+    return lib().fd_device_status(_stream(stream, device))
+
+
+def fd_strerror(code: int) -> str:
+    return lib().fd_strerror(int(code)).decode()
+
+
+def fd_version() -> int:
+    return lib().fd_version()
+
+
+# ------------------------------------------------------------ convenience --
+
+def workspace_layout(B, Hq, Hkv, D, num_splits):
+    """(slots, g, byte offset of seg_lse) of the documented workspace layout."""
+    slots = num_splits + B * Hkv - 1
+    g = Hq // Hkv
+    off = (slots * g * D * 4 + 255) // 256 * 256
+    return slots, g, off
+
+
+def decode(q, k_cache, v_cache, seqlens, scale, num_splits=None, stream=None):
+    """Allocate out / lse / workspace with torch and run fd_decode (or
+    fd_decode_splits when num_splits is given). Returns (out, lse)."""
+    B, Hq, Hkv, D, Lmax = _shapes(q, k_cache, v_cache)
+    S = fd_plan(B, Hq, Hkv, D, Lmax) if num_splits is None else int(num_splits)
+    nbytes = fd_workspace_bytes(B, Hq, Hkv, D, Lmax, S)
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device) if nbytes else None
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    fd_decode_splits(q, k_cache, v_cache, seqlens, scale, out, lse, ws, S, stream)
+    return out, lse

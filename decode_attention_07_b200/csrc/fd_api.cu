@@ -1,0 +1,449 @@
+// fd_api.cu -- the C ABI declared in include/fd.h: argument checks, the
+// split planner, tensor-map encoding and the two launches.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "fd.h"
+#include "fd_combine.cuh"
+#include "fd_partition.cuh"
+#include "fd_split.cuh"
+
+namespace {
+
+constexpr int kVersion = 100;               // 0.1.0
+constexpr int kMinTilesPerSplit = 4;        // a split streams at least 256 tokens per kv head
+constexpr int kMaxDevices = 64;
+constexpr float kLog2e = 1.4426950408889634f;
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ----------------------------------------------------------- shape checks --
+int check_shape(int B, int Hq, int Hkv, int D, int max_len) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || max_len < 0) return FD_ERR_SHAPE;
+    if (Hq % Hkv != 0 || Hq / Hkv > FD_MAX_GROUP) return FD_ERR_GROUP;
+    if (D != 64 && D != 128) return FD_ERR_HEAD_DIM;
+    // sizes kept inside 32-bit grid/tensor-map dimensions and 64-bit run arithmetic
+    const long long rows = static_cast<long long>(B) * Hkv;
+    if (rows > 0x7fffffffLL || static_cast<long long>(B) * Hq > 0x7fffffffLL) return FD_ERR_SHAPE;
+    const long long tiles = rows * fd::tiles_of(max_len);
+    if (tiles > (1LL << 44)) return FD_ERR_SHAPE;
+    return FD_OK;
+}
+
+long long num_slots(int B, int Hkv, int num_splits) {
+    return static_cast<long long>(num_splits) + static_cast<long long>(B) * Hkv - 1;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t workspace_bytes(int B, int Hq, int Hkv, int D, int num_splits) {
+    if (num_splits <= 1) return 0;
+    const size_t slots = static_cast<size_t>(num_slots(B, Hkv, num_splits));
+    const size_t g = static_cast<size_t>(Hq / Hkv);
+    return align256(slots * g * D * sizeof(float)) + align256(slots * g * sizeof(float));
+}
+
+// ------------------------------------------------------------ device info --
+struct DeviceInfo {
+    bool queried = false;
+    int status = FD_OK;
+    int sms = 0;
+    bool split_attr_set = false;
+};
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+int current_device(int *dev) {
+    if (cudaGetDevice(dev) != cudaSuccess) {
+        cudaGetLastError();
+        return FD_ERR_DEVICE;
+    }
+    if (*dev < 0 || *dev >= kMaxDevices) return FD_ERR_DEVICE;
+    return FD_OK;
+}
+
+int device_sms(int *sms) {
+    int dev;
+    int rc = current_device(&dev);
+    if (rc != FD_OK) return rc;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo &d = g_devices[dev];
+    if (!d.queried) {
+        int major = 0, minor = 0, n = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            d.status = FD_ERR_DEVICE;
+        } else if (major != 10 || minor != 0) {
+            d.status = FD_ERR_DEVICE;   // built for sm_100a only
+        } else {
+            d.status = FD_OK;
+            d.sms = n;
+        }
+        d.queried = true;
+    }
+    *sms = d.sms;
+    return d.status;
+}
+
+// ------------------------------------------------------------ tensor maps --
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// K or V cache [B*Hkv rows][Lmax][D] bf16 as a 3-D tensor (D innermost);
+// box = 64 head-dim elements (128 bytes, 128-byte swizzle) x 64 tokens x 1 row.
+int encode_cache_map(CUtensorMap *map, const void *base, int D, int Lmax, long long rows) {
+    auto fn = encode_fn();
+    if (!fn) return FD_ERR_LAUNCH;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Lmax), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Lmax) * D * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(fd::kTileTokens), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FD_OK : FD_ERR_LAUNCH;
+}
+
+// ---------------------------------------------------------------- launches --
+template <int D, class Consumer>
+int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p, cudaStream_t st) {
+    constexpr int smem = fd::split_smem_bytes<D, Consumer::G>();
+    auto kern = fd::fd_split_kernel<D, Consumer>;
+    // the attribute is per function; setting it again is cheap and thread-safe
+    static std::once_flag once[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaError_t attr_err = cudaSuccess;
+    std::call_once(once[dev], [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (attr_err != cudaSuccess) {
+        cudaGetLastError();
+        return FD_ERR_LAUNCH;
+    }
+    kern<<<p.P, fd::kSplitThreads, smem, st>>>(tk, tv, p);
+    if (cudaGetLastError() != cudaSuccess) return FD_ERR_LAUNCH;
+    return FD_OK;
+}
+
+int launch_split(int D, int g, const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p,
+                 cudaStream_t st) {
+    if (D == 128) {
+        if (g == 1) return launch_split_t<128, fd::HeadConsumer<128>>(tk, tv, p, st);
+        if (g <= 8) return launch_split_t<128, fd::GroupConsumer<128, 1>>(tk, tv, p, st);
+        return launch_split_t<128, fd::GroupConsumer<128, 2>>(tk, tv, p, st);
+    }
+    if (g == 1) return launch_split_t<64, fd::HeadConsumer<64>>(tk, tv, p, st);
+    if (g <= 8) return launch_split_t<64, fd::GroupConsumer<64, 1>>(tk, tv, p, st);
+    return launch_split_t<64, fd::GroupConsumer<64, 2>>(tk, tv, p, st);
+}
+
+int launch_combine(int D, const fd::CombineParams &p, cudaStream_t st, bool after_split) {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(static_cast<unsigned>(p.B) * static_cast<unsigned>(p.Hkv));
+    cfg.blockDim = dim3(fd::kCombineThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_split ? 1 : 0;
+    cudaError_t e = D == 128 ? cudaLaunchKernelEx(&cfg, fd::fd_combine_kernel<128>, p)
+                             : cudaLaunchKernelEx(&cfg, fd::fd_combine_kernel<64>, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return FD_ERR_LAUNCH;
+    }
+    return FD_OK;
+}
+
+struct Problem {
+    int B, Hq, Hkv, D, max_len;
+    const uint16_t *q, *k, *v;
+    const int32_t *seqlens;
+    float scale;
+    float *out, *lse;
+    void *ws;
+    size_t ws_bytes;
+    int num_splits;
+    cudaStream_t stream;
+};
+
+// Checks shared by every compute entry point (no CUDA call).
+int check_problem(const Problem &pr, bool need_kv) {
+    int rc = check_shape(pr.B, pr.Hq, pr.Hkv, pr.D, pr.max_len);
+    if (rc != FD_OK) return rc;
+    if (pr.num_splits < 1 || pr.num_splits > FD_MAX_SPLITS) return FD_ERR_SPLITS;
+    if (!pr.seqlens || !pr.out || !pr.lse) return FD_ERR_NULL_POINTER;
+    // with max_len == 0 no token exists and q/k/v are never read (they may be NULL)
+    const bool reads_kv = need_kv && pr.max_len > 0;
+    if (reads_kv && (!pr.q || !pr.k || !pr.v)) return FD_ERR_NULL_POINTER;
+    if (!aligned(pr.seqlens, 4) || !aligned(pr.out, 4) || !aligned(pr.lse, 4)) return FD_ERR_ALIGNMENT;
+    if (reads_kv && (!aligned(pr.q, 16) || !aligned(pr.k, 16) || !aligned(pr.v, 16))) return FD_ERR_ALIGNMENT;
+    const size_t need = workspace_bytes(pr.B, pr.Hq, pr.Hkv, pr.D, pr.num_splits);
+    if (need > 0) {
+        if (!pr.ws || pr.ws_bytes < need) return FD_ERR_WORKSPACE;
+        if (!aligned(pr.ws, 16)) return FD_ERR_ALIGNMENT;
+    }
+    const long long tiles = static_cast<long long>(pr.B) * pr.Hkv * fd::tiles_of(pr.max_len);
+    if (tiles > 0 && (tiles * pr.num_splits) > (1LL << 62)) return FD_ERR_SHAPE;
+    return FD_OK;
+}
+
+void seg_pointers(const Problem &pr, float **so, float **sl) {
+    if (workspace_bytes(pr.B, pr.Hq, pr.Hkv, pr.D, pr.num_splits) == 0) {
+        *so = *sl = nullptr;
+        return;
+    }
+    const size_t slots = static_cast<size_t>(num_slots(pr.B, pr.Hkv, pr.num_splits));
+    const size_t g = static_cast<size_t>(pr.Hq / pr.Hkv);
+    *so = static_cast<float *>(pr.ws);
+    *sl = reinterpret_cast<float *>(static_cast<char *>(pr.ws) + align256(slots * g * pr.D * sizeof(float)));
+}
+
+int run_split(const Problem &pr) {
+    if (pr.max_len == 0) return FD_OK;   // no tokens anywhere: nothing to stream
+    int sms;
+    int rc = device_sms(&sms);
+    if (rc != FD_OK) return rc;
+    CUtensorMap tk, tv;
+    const long long rows = static_cast<long long>(pr.B) * pr.Hkv;
+    if ((rc = encode_cache_map(&tk, pr.k, pr.D, pr.max_len, rows)) != FD_OK) return rc;
+    if ((rc = encode_cache_map(&tv, pr.v, pr.D, pr.max_len, rows)) != FD_OK) return rc;
+    fd::SplitParams p;
+    p.q = pr.q;
+    p.seqlens = pr.seqlens;
+    p.out = pr.out;
+    p.lse = pr.lse;
+    seg_pointers(pr, &p.seg_out, &p.seg_lse);
+    p.B = pr.B;
+    p.Hq = pr.Hq;
+    p.Hkv = pr.Hkv;
+    p.g = pr.Hq / pr.Hkv;
+    p.Lmax = pr.max_len;
+    p.P = pr.num_splits;
+    p.scale_log2e = pr.scale * kLog2e;
+    return launch_split(pr.D, p.g, tk, tv, p, pr.stream);
+}
+
+int run_combine(const Problem &pr, bool after_split) {
+    int sms;
+    int rc = device_sms(&sms);
+    if (rc != FD_OK) return rc;
+    fd::CombineParams p;
+    p.seqlens = pr.seqlens;
+    p.out = pr.out;
+    p.lse = pr.lse;
+    float *so, *sl;
+    seg_pointers(pr, &so, &sl);
+    p.seg_out = so;
+    p.seg_lse = sl;
+    p.B = pr.B;
+    p.Hq = pr.Hq;
+    p.Hkv = pr.Hkv;
+    p.g = pr.Hq / pr.Hkv;
+    p.Lmax = pr.max_len;
+    p.P = pr.num_splits;
+    return launch_combine(pr.D, p, pr.stream, after_split && pr.max_len > 0);
+}
+
+Problem make_problem(int B, int Hq, int Hkv, int D, int max_len, const uint16_t *q, const uint16_t *k,
+                     const uint16_t *v, const int32_t *seqlens, float scale, float *out, float *lse, void *ws,
+                     size_t ws_bytes, int num_splits, void *stream) {
+    Problem pr;
+    pr.B = B;
+    pr.Hq = Hq;
+    pr.Hkv = Hkv;
+    pr.D = D;
+    pr.max_len = max_len;
+    pr.q = q;
+    pr.k = k;
+    pr.v = v;
+    pr.seqlens = seqlens;
+    pr.scale = scale;
+    pr.out = out;
+    pr.lse = lse;
+    pr.ws = ws;
+    pr.ws_bytes = ws_bytes;
+    pr.num_splits = num_splits;
+    pr.stream = static_cast<cudaStream_t>(stream);
+    return pr;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fd_plan_for_sms(int B, int Hq, int Hkv, int D, int max_len, int num_sms) {
+    int rc = check_shape(B, Hq, Hkv, D, max_len);
+    if (rc != FD_OK) return rc;
+    if (num_sms < 1) return FD_ERR_DEVICE;
+    const long long tiles = static_cast<long long>(B) * Hkv * fd::tiles_of(max_len);
+    long long want = (tiles + kMinTilesPerSplit - 1) / kMinTilesPerSplit;
+    if (want < 1) want = 1;
+    if (want > num_sms) want = num_sms;
+    if (want > FD_MAX_SPLITS) want = FD_MAX_SPLITS;
+    return static_cast<int>(want);
+}
+
+int fd_plan(int B, int Hq, int Hkv, int D, int max_len) {
+    int rc = check_shape(B, Hq, Hkv, D, max_len);
+    if (rc != FD_OK) return rc;
+    int sms;
+    rc = device_sms(&sms);
+    if (rc != FD_OK) return rc;
+    return fd_plan_for_sms(B, Hq, Hkv, D, max_len, sms);
+}
+
+size_t fd_workspace_bytes(int B, int Hq, int Hkv, int D, int max_len, int num_splits) {
+    if (check_shape(B, Hq, Hkv, D, max_len) != FD_OK) return 0;
+    if (num_splits < 1 || num_splits > FD_MAX_SPLITS) return 0;
+    return workspace_bytes(B, Hq, Hkv, D, num_splits);
+}
+
+int fd_decode_splits(int B, int Hq, int Hkv, int D, int max_len, const uint16_t *q, const uint16_t *k_cache,
+                     const uint16_t *v_cache, const int32_t *seqlens, float scale, float *out, float *lse,
+                     void *workspace, size_t workspace_bytes, int num_splits, void *stream) {
+    Problem pr = make_problem(B, Hq, Hkv, D, max_len, q, k_cache, v_cache, seqlens, scale, out, lse, workspace,
+                              workspace_bytes, num_splits, stream);
+    int rc = check_problem(pr, true);
+    if (rc != FD_OK) return rc;
+    if ((rc = run_split(pr)) != FD_OK) return rc;
+    return run_combine(pr, true);
+}
+
+int fd_decode(int B, int Hq, int Hkv, int D, int max_len, const uint16_t *q, const uint16_t *k_cache,
+              const uint16_t *v_cache, const int32_t *seqlens, float scale, float *out, float *lse,
+              void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = check_shape(B, Hq, Hkv, D, max_len);
+    if (rc != FD_OK) return rc;
+    const int S = fd_plan(B, Hq, Hkv, D, max_len);
+    if (S < 0) return S;
+    return fd_decode_splits(B, Hq, Hkv, D, max_len, q, k_cache, v_cache, seqlens, scale, out, lse, workspace,
+                            workspace_bytes, S, stream);
+}
+
+int fd_split(int B, int Hq, int Hkv, int D, int max_len, const uint16_t *q, const uint16_t *k_cache,
+             const uint16_t *v_cache, const int32_t *seqlens, float scale, float *out, float *lse,
+             void *workspace, size_t workspace_bytes, int num_splits, void *stream) {
+    Problem pr = make_problem(B, Hq, Hkv, D, max_len, q, k_cache, v_cache, seqlens, scale, out, lse, workspace,
+                              workspace_bytes, num_splits, stream);
+    int rc = check_problem(pr, true);
+    if (rc != FD_OK) return rc;
+    return run_split(pr);
+}
+
+int fd_combine(int B, int Hq, int Hkv, int D, int max_len, const int32_t *seqlens, float *out, float *lse,
+               const void *workspace, size_t workspace_bytes, int num_splits, void *stream) {
+    Problem pr = make_problem(B, Hq, Hkv, D, max_len, nullptr, nullptr, nullptr, seqlens, 0.f, out, lse,
+                              const_cast<void *>(workspace), workspace_bytes, num_splits, stream);
+    int rc = check_problem(pr, false);
+    if (rc != FD_OK) return rc;
+    return run_combine(pr, false);
+}
+
+int fd_segments(int B, int Hkv, int max_len, const int32_t *seqlens_host, int num_splits, int32_t *seg_row,
+                int32_t *seg_begin, int32_t *seg_end, int32_t *seg_whole, int capacity) {
+    if (B < 1 || Hkv < 1 || max_len < 0) return FD_ERR_SHAPE;
+    if (static_cast<long long>(B) * Hkv > 0x7fffffffLL) return FD_ERR_SHAPE;
+    if (num_splits < 1 || num_splits > FD_MAX_SPLITS) return FD_ERR_SPLITS;
+    if (!seqlens_host || !seg_row || !seg_begin || !seg_end || !seg_whole) return FD_ERR_NULL_POINTER;
+    const long long slots = num_slots(B, Hkv, num_splits);
+    if (slots > 0x7fffffffLL) return FD_ERR_SHAPE;
+    if (capacity < slots) return FD_ERR_CAPACITY;
+    for (long long s = 0; s < slots; ++s) {
+        seg_row[s] = -1;
+        seg_begin[s] = seg_end[s] = 0;
+        seg_whole[s] = 0;
+    }
+    long long total = 0;
+    for (int b = 0; b < B; ++b) total += fd::tiles_of(fd::clamp_len(seqlens_host[b], max_len));
+    const long long N = total * Hkv;
+    long long before = 0;
+    for (int b = 0; b < B; ++b) {
+        const int L = fd::clamp_len(seqlens_host[b], max_len);
+        const int n = fd::tiles_of(L);
+        for (int h = 0; h < Hkv; ++h) {
+            if (n == 0) continue;
+            const long long u = static_cast<long long>(b) * Hkv + h;
+            const long long first = before * Hkv + static_cast<long long>(h) * n;
+            const int i0 = fd::run_of_tile(first, N, num_splits);
+            const int i1 = fd::run_of_tile(first + n - 1, N, num_splits);
+            for (int i = i0; i <= i1; ++i) {
+                const long long lo = fd::run_begin(i, N, num_splits), hi = fd::run_begin(i + 1, N, num_splits);
+                const long long t0 = (lo > first ? lo : first) - first;
+                const long long t1 = (hi < first + n ? hi : first + n) - first;
+                const long long s = i + u;
+                seg_row[s] = static_cast<int32_t>(u);
+                seg_begin[s] = static_cast<int32_t>(t0 * fd::kTileTokens);
+                const long long e = t1 * fd::kTileTokens;
+                seg_end[s] = static_cast<int32_t>(e < L ? e : L);
+                seg_whole[s] = i0 == i1 ? 1 : 0;
+            }
+        }
+        before += n;
+    }
+    return static_cast<int>(slots);
+}
+
+int fd_device_status(void *stream) {
+    int dev;
+    if (current_device(&dev) != FD_OK) return FD_ERR_DEVICE;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return FD_ERR_LAUNCH;
+    }
+    int word = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&word, fd::g_fd_error_word, sizeof word) != cudaSuccess ||
+        cudaMemcpyToSymbol(fd::g_fd_error_word, &zero, sizeof zero) != cudaSuccess) {
+        cudaGetLastError();
+        return FD_ERR_LAUNCH;
+    }
+    return word;
+}
+
+const char *fd_strerror(int code) {
+    switch (code) {
+        case FD_OK: return "ok";
+        case FD_ERR_NULL_POINTER: return "a required pointer is NULL";
+        case FD_ERR_SHAPE: return "invalid or too large B / Hq / Hkv / max_len";
+        case FD_ERR_GROUP: return "Hq must be a multiple of Hkv with Hq/Hkv <= 16";
+        case FD_ERR_HEAD_DIM: return "head dimension D must be 64 or 128";
+        case FD_ERR_ALIGNMENT: return "pointer misaligned (q/k/v/workspace need 16 bytes, seqlens/out/lse 4)";
+        case FD_ERR_WORKSPACE: return "workspace missing or smaller than fd_workspace_bytes()";
+        case FD_ERR_SPLITS: return "num_splits out of range [1, 65535]";
+        case FD_ERR_DEVICE: return "no usable CUDA device of compute capability 10.0";
+        case FD_ERR_LAUNCH: return "kernel launch or tensor-map encoding failed";
+        case FD_ERR_TIMEOUT: return "a device-side wait gave up; outputs of that call are invalid";
+        case FD_ERR_CAPACITY: return "output arrays too small";
+        default: return "unknown error code";
+    }
+}
+
+int fd_version(void) { return kVersion; }
+
+}  // extern "C"

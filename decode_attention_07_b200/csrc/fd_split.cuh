@@ -1,0 +1,577 @@
+// fd_split.cuh -- the split stage of decode attention (one thread block per run
+// of key/value tiles; see fd_partition.cuh for how runs are cut).
+//
+// "Flash-Decoding for long-context inference", section "A faster attention
+// for decoding: Flash-Decoding": each split computes the attention of the
+// query with its chunk of keys/values and writes one extra scalar per row,
+// the log-sum-exp; the softmax can be built up tile by tile ("the
+// attention/softmax can be calculated iteratively"), which is what the
+// running max / running sum below do.
+//
+// Block layout (160 threads, one block per SM):
+//   warp 4      producer: one lane streams K and V tiles (64 tokens x D bf16
+//               each) from HBM into a ring of shared-memory stages with 3-D
+//               TMA loads, 128-byte swizzled; mbarrier completion.
+//   warps 0..3  consumers: warp w owns tokens [16w, 16w+16) of every tile.
+//               Per tile: logits for its 16 tokens, online-softmax update of
+//               the running max m and sum l per query head, and the
+//               rescaled accumulation of p * v; at the end of a row segment
+//               the four warps' (m, l, o) are merged through shared memory
+//               and written out (whole row) or to the workspace (segment).
+// Two consumer forms:
+//   * grouped heads (g = Hq/Hkv >= 2): the g query heads that share one kv
+//     head form a small dense contraction, run on tensor cores with
+//     mma.sync m16n8k16 (bf16 in, fp32 accumulate): S^T[16 tok x 8 heads] =
+//     K[16 x D] Q^T and O^T[D x 8 heads] += V^T[D x 16 tok] P^T, P split
+//     into a bf16 high part and a bf16 remainder so P V keeps ~16 bits of P.
+//     Every K/V byte is read once for the whole group.
+//   * one head per kv head (g = 1): CUDA-core dot products, 16 (D=128) or 8
+//     (D=64) lanes per token, reduced with warp shuffles.
+#pragma once
+
+#include "fd_partition.cuh"
+#include "fd_ptx.cuh"
+
+namespace fd {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kSplitThreads = kConsumerThreads + 32;
+constexpr int kWarpTokens = 16;                  // tokens of a tile owned by one consumer warp
+constexpr int kBoxBytes = kTileTokens * 128;     // one TMA box: 64 rows x 128 bytes (64 bf16)
+constexpr uint64_t kWaitLimitNs = 2000000000ull; // a bounded wait gives up after 2 s
+constexpr float kLn2 = 0.693147180559945309f;
+
+// Sticky per-device error word (FD_ERR_TIMEOUT when a wait gave up).
+__device__ int g_fd_error_word;
+
+struct SplitParams {
+    const uint16_t *q;        // [B, Hq, D]
+    const int32_t *seqlens;   // [B]
+    float *out;               // [B, Hq, D]
+    float *lse;               // [B, Hq]
+    float *seg_out;           // [slots, g, D]
+    float *seg_lse;           // [slots, g]
+    int B, Hq, Hkv, g, Lmax, P;
+    float scale_log2e;        // scale * log2(e): logits are kept in base 2
+};
+
+template <int D>
+struct SplitConfig {
+    static constexpr int kBoxes = D / 64;                        // 128-byte boxes per row
+    static constexpr int kTileBytes = kTileTokens * D * 2;       // one K (or V) tile
+    static constexpr int kStages = D == 128 ? 4 : 8;             // 128 KiB of ring either way
+    static constexpr int kRingBytes = kStages * 2 * kTileBytes;
+};
+
+// Shared-memory bytes of one split block (plus 1 KiB for 1024-byte alignment).
+template <int D, int G>
+constexpr int split_smem_bytes() {
+    return 1024 + SplitConfig<D>::kRingBytes + kConsumerWarps * (G * D + 2 * G) * 4 +
+           2 * SplitConfig<D>::kStages * 8 + 64;
+}
+
+struct Cursor {
+    int b, h, tile, n;   // row (b, h), tile index inside the row, tiles of sequence b
+};
+
+struct StartInfo {
+    long long count;     // tiles in this block's run
+    int b, h, tile, n;
+    int abort;           // set when a bounded wait gave up
+};
+
+// Bounded mbarrier wait. Returns false if the block is aborting or the limit
+// passes (then it marks the abort and the device error word).
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            atomicExch(&g_fd_error_word, -10 /* FD_ERR_TIMEOUT */);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ int row_tiles(const int32_t *seqlens, int b, int Lmax) {
+    return tiles_of(clamp_len(__ldg(seqlens + b), Lmax));
+}
+
+// Next row with at least one tile (only called while tiles remain).
+__device__ __forceinline__ void next_row(Cursor &c, const SplitParams &p) {
+    c.tile = 0;
+    if (++c.h == p.Hkv) {
+        c.h = 0;
+        do {
+            ++c.b;
+            c.n = row_tiles(p.seqlens, c.b, p.Lmax);
+        } while (c.n == 0);
+    }
+}
+
+// Warp 0: total tile count and this block's starting row / tile.
+__device__ __forceinline__ void find_start(const SplitParams &p, StartInfo *info) {
+    const int lane = threadIdx.x & 31;
+    long long total = 0;
+    for (int base = 0; base < p.B; base += 32) {
+        int n = base + lane < p.B ? row_tiles(p.seqlens, base + lane, p.Lmax) : 0;
+        for (int s = 16; s > 0; s >>= 1) n += __shfl_xor_sync(0xffffffffu, n, s);
+        total += n;
+    }
+    const long long N = total * p.Hkv;
+    const long long t0 = run_begin(blockIdx.x, N, p.P);
+    const long long t1 = run_begin(blockIdx.x + 1, N, p.P);
+    int b = 0, h = 0, tile = 0, n = 0;
+    if (t1 > t0) {
+        long long before = 0;   // Hkv * (tiles of sequences before this chunk)
+        for (int base = 0; base < p.B; base += 32) {
+            const int nb = base + lane < p.B ? row_tiles(p.seqlens, base + lane, p.Lmax) : 0;
+            int incl = nb;
+            for (int s = 1; s < 32; s <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, s);
+                if (lane >= s) incl += y;
+            }
+            const long long after = before + static_cast<long long>(p.Hkv) * incl;
+            const unsigned hit = __ballot_sync(0xffffffffu, base + lane < p.B && after > t0);
+            if (hit) {
+                const int src = __ffs(hit) - 1;
+                b = base + src;
+                n = __shfl_sync(0xffffffffu, nb, src);
+                const long long row0 = __shfl_sync(0xffffffffu, after, src) - static_cast<long long>(p.Hkv) * n;
+                const long long off = t0 - row0;
+                h = static_cast<int>(off / n);
+                tile = static_cast<int>(off % n);
+                break;
+            }
+            before += static_cast<long long>(p.Hkv) * __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
+    if (lane == 0) {
+        info->count = t1 - t0;
+        info->b = b;
+        info->h = h;
+        info->tile = tile;
+        info->n = n;
+        info->abort = 0;
+    }
+}
+
+// ------------------------------------------------------------ merge + store --
+// Per-warp partial results in shared memory: o[G][D], then m[G], l[G] (m in
+// base-2 units). All 128 consumer threads merge the four warps and store.
+template <int D, int G>
+__device__ __forceinline__ void merge_and_store(const float *merge, const SplitParams &p, const Cursor &c,
+                                                bool whole, int slot) {
+    constexpr int kWarpFloats = G * D + 2 * G;
+    const int tid = threadIdx.x;
+    for (int idx = tid; idx < p.g * D; idx += kConsumerThreads) {
+        const int head = idx / D, d = idx - head * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge[w * kWarpFloats + G * D + head]);
+        float o = 0.f, lse_nat = -INFINITY;
+        if (M != -INFINITY) {
+            float acc = 0.f, lsum = 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float *wb = merge + w * kWarpFloats;
+                const float e = ex2(wb[G * D + head] - M);
+                lsum += e * wb[G * D + G + head];
+                acc += e * wb[head * D + d];
+            }
+            o = acc / lsum;
+            lse_nat = (M + lg2(lsum)) * kLn2;
+        }
+        if (whole) {
+            const size_t row = static_cast<size_t>(c.b) * p.Hq + static_cast<size_t>(c.h) * p.g + head;
+            p.out[row * D + d] = o;
+            if (d == 0) p.lse[row] = lse_nat;
+        } else {
+            const size_t row = static_cast<size_t>(slot) * p.g + head;
+            p.seg_out[row * D + d] = o;
+            if (d == 0) p.seg_lse[row] = lse_nat;
+        }
+    }
+}
+
+// ------------------------------------------------- grouped-head consumer --
+template <int D, int NT>
+struct GroupConsumer {
+    static constexpr int KS = D / 16;   // k-steps of the logit contraction
+    static constexpr int MT = D / 16;   // m-tiles of the P V contraction
+    static constexpr int G = 8 * NT;    // heads held (padded)
+
+    uint32_t qf[NT][KS][2];             // Q^T as the B operand, per n-tile
+    float m[NT][2], l[NT][2];           // running max (base 2) / partial sum for heads 2c, 2c+1
+    float o[NT][MT][4];                 // O^T accumulators
+
+    __device__ __forceinline__ void begin_row(const SplitParams &p, const Cursor &c) {
+        const int lane = threadIdx.x & 31;
+        const int r0 = lane >> 2, cc = lane & 3;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int head = nt * 8 + r0;
+            const bool ok = head < p.g;
+            const uint16_t *qrow =
+                p.q + (static_cast<size_t>(c.b) * p.Hq + static_cast<size_t>(c.h) * p.g + (ok ? head : 0)) * D;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                qf[nt][ks][0] = ok ? __ldg(reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 2 * cc)) : 0u;
+                qf[nt][ks][1] = ok ? __ldg(reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 2 * cc + 8)) : 0u;
+            }
+            m[nt][0] = m[nt][1] = -INFINITY;
+            l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+        }
+    }
+
+    static __device__ __forceinline__ uint32_t keep_tokens(uint32_t w, int t, int valid) {
+        return w & ((t < valid ? 0x0000ffffu : 0u) | (t + 1 < valid ? 0xffff0000u : 0u));
+    }
+
+    // One tile: `valid` = tokens of this warp's 16 that are inside the row.
+    __device__ __forceinline__ void tile(uint32_t k_smem, uint32_t v_smem, int valid, float scale_log2e) {
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        const int mi = lane >> 3, rr = lane & 7;
+        const int r0 = lane >> 2, cc = lane & 3;
+
+        // S^T = K Q^T over this warp's 16 tokens
+        float s[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+        const int krow = kWarpTokens * warp + rr + 8 * (mi & 1);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            const int d = 16 * ks + 8 * (mi >> 1);
+            const uint32_t addr = k_smem + (d >> 6) * kBoxBytes + krow * 128 + ((((d & 63) >> 3) ^ rr) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(addr, a0, a1, a2, a3);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+        }
+
+        // online softmax per head column; P^T fragments (high + remainder)
+        uint32_t bh[NT][2], bl[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float x0 = s[nt][0] * scale_log2e, x1 = s[nt][1] * scale_log2e;
+            float x2 = s[nt][2] * scale_log2e, x3 = s[nt][3] * scale_log2e;
+            if (r0 >= valid) x0 = x1 = -INFINITY;
+            if (r0 + 8 >= valid) x2 = x3 = -INFINITY;
+            float ma = fmaxf(x0, x2), mb = fmaxf(x1, x3);
+#pragma unroll
+            for (int sh = 4; sh < 32; sh <<= 1) {
+                ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, sh));
+                mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, sh));
+            }
+            const float na = fmaxf(m[nt][0], ma), nb = fmaxf(m[nt][1], mb);
+            const float ua = na == -INFINITY ? 0.f : na, ub = nb == -INFINITY ? 0.f : nb;
+            const float alpha_a = ex2(m[nt][0] - ua), alpha_b = ex2(m[nt][1] - ub);
+            const float p0 = ex2(x0 - ua), p2 = ex2(x2 - ua), p1 = ex2(x1 - ub), p3 = ex2(x3 - ub);
+            l[nt][0] = l[nt][0] * alpha_a + (p0 + p2);
+            l[nt][1] = l[nt][1] * alpha_b + (p1 + p3);
+            m[nt][0] = na;
+            m[nt][1] = nb;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                o[nt][mt][0] *= alpha_a;
+                o[nt][mt][2] *= alpha_a;
+                o[nt][mt][1] *= alpha_b;
+                o[nt][mt][3] *= alpha_b;
+            }
+            const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+            const uint32_t l01 = pack_bf16x2(p0 - bf16lo_to_f32(h01), p1 - bf16hi_to_f32(h01));
+            const uint32_t l23 = pack_bf16x2(p2 - bf16lo_to_f32(h23), p3 - bf16hi_to_f32(h23));
+            bh[nt][0] = movmatrix_trans(h01);
+            bh[nt][1] = movmatrix_trans(h23);
+            bl[nt][0] = movmatrix_trans(l01);
+            bl[nt][1] = movmatrix_trans(l23);
+        }
+
+        // O^T += V^T P^T
+        const int vrow = kWarpTokens * warp + 8 * (mi >> 1) + rr;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int d = 16 * mt + 8 * (mi & 1);
+            const uint32_t addr = v_smem + (d >> 6) * kBoxBytes + vrow * 128 + ((((d & 63) >> 3) ^ rr) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_trans(addr, a0, a1, a2, a3);
+            if (valid < kWarpTokens) {   // rows past the end may hold anything (NaN): zero them
+                a0 = keep_tokens(a0, 2 * cc, valid);
+                a1 = keep_tokens(a1, 2 * cc, valid);
+                a2 = keep_tokens(a2, 8 + 2 * cc, valid);
+                a3 = keep_tokens(a3, 8 + 2 * cc, valid);
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                mma_bf16_16816(o[nt][mt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
+                mma_bf16_16816(o[nt][mt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+            }
+        }
+    }
+
+    __device__ __forceinline__ void to_smem(float *wb) {
+        const int lane = threadIdx.x & 31;
+        const int r0 = lane >> 2, cc = lane & 3;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int sh = 4; sh < 32; sh <<= 1) l[nt][e] += __shfl_xor_sync(0xffffffffu, l[nt][e], sh);
+            const int ha = nt * 8 + 2 * cc, hb = ha + 1;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int d0 = 16 * mt + r0, d1 = d0 + 8;
+                wb[ha * D + d0] = o[nt][mt][0];
+                wb[hb * D + d0] = o[nt][mt][1];
+                wb[ha * D + d1] = o[nt][mt][2];
+                wb[hb * D + d1] = o[nt][mt][3];
+            }
+            if (r0 == 0) {
+                wb[G * D + ha] = m[nt][0];
+                wb[G * D + hb] = m[nt][1];
+                wb[G * D + G + ha] = l[nt][0];
+                wb[G * D + G + hb] = l[nt][1];
+            }
+        }
+    }
+};
+
+// ------------------------------------------------ one-head (MHA) consumer --
+template <int D>
+struct HeadConsumer {
+    static constexpr int G = 1;
+    static constexpr int LPT = D / 8;          // lanes per token (16 bytes = 8 bf16 each)
+    static constexpr int TPI = 32 / LPT;       // tokens per warp-wide load
+    static constexpr int ITER = kWarpTokens / TPI;
+
+    float qv[8];                               // q[d0 .. d0+7] of this lane's 16-byte chunk
+    float m, l;                                // running max (base 2, warp-uniform) / lane partial sum
+    float acc[8];                              // sum of p * v over this lane's tokens, chunk d0..d0+7
+
+    __device__ __forceinline__ void begin_row(const SplitParams &p, const Cursor &c) {
+        const int lane = threadIdx.x & 31;
+        const int d0 = 8 * (lane % LPT);
+        const uint16_t *qrow = p.q + (static_cast<size_t>(c.b) * p.Hq + c.h) * D;
+        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(qrow + d0));
+        qv[0] = bf16lo_to_f32(w.x); qv[1] = bf16hi_to_f32(w.x);
+        qv[2] = bf16lo_to_f32(w.y); qv[3] = bf16hi_to_f32(w.y);
+        qv[4] = bf16lo_to_f32(w.z); qv[5] = bf16hi_to_f32(w.z);
+        qv[6] = bf16lo_to_f32(w.w); qv[7] = bf16hi_to_f32(w.w);
+        m = -INFINITY;
+        l = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+    }
+
+    static __device__ __forceinline__ uint4 lds128(uint32_t addr) {
+        uint4 r;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                     : "r"(addr)
+                     : "memory");
+        return r;
+    }
+
+    __device__ __forceinline__ void tile(uint32_t k_smem, uint32_t v_smem, int valid, float scale_log2e) {
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        const int half = lane / LPT, chunk = lane % LPT;
+        const int d0 = 8 * chunk;
+        const uint32_t col = (d0 >> 6) * kBoxBytes;
+        const int j = (d0 & 63) >> 3;
+
+        // partial dots over this lane's 8 dims for tokens TPI*it + half
+        float pd[ITER];
+#pragma unroll
+        for (int it = 0; it < ITER; ++it) {
+            const int r = kWarpTokens * warp + TPI * it + half;
+            const uint4 w = lds128(k_smem + col + r * 128 + ((j ^ (r & 7)) << 4));
+            float a = qv[0] * bf16lo_to_f32(w.x);
+            a = fmaf(qv[1], bf16hi_to_f32(w.x), a);
+            a = fmaf(qv[2], bf16lo_to_f32(w.y), a);
+            a = fmaf(qv[3], bf16hi_to_f32(w.y), a);
+            a = fmaf(qv[4], bf16lo_to_f32(w.z), a);
+            a = fmaf(qv[5], bf16hi_to_f32(w.z), a);
+            a = fmaf(qv[6], bf16lo_to_f32(w.w), a);
+            a = fmaf(qv[7], bf16hi_to_f32(w.w), a);
+            pd[it] = a;
+        }
+        // reduce across the LPT lanes of each token while spreading tokens
+        // over lanes: after the halving steps lane keeps token index
+        // (lane % LPT) / 2; the last step leaves the full dot in both lanes
+        // of each pair.
+#pragma unroll
+        for (int n = ITER; n > 1; n >>= 1) {
+            const bool up = (lane & n) != 0;
+#pragma unroll
+            for (int k = 0; k < n / 2; ++k) {
+                const float send = up ? pd[k] : pd[k + n / 2];
+                const float keep = up ? pd[k + n / 2] : pd[k];
+                pd[k] = keep + __shfl_xor_sync(0xffffffffu, send, n);
+            }
+        }
+        float x = pd[0] + __shfl_xor_sync(0xffffffffu, pd[0], 1);
+        const int my_it = chunk >> 1;
+        x *= scale_log2e;
+        if (TPI * my_it + half >= valid) x = -INFINITY;
+
+        float mx = x;
+#pragma unroll
+        for (int sh = 1; sh < 32; sh <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, sh));
+        const float mn = fmaxf(m, mx);
+        const float mu = mn == -INFINITY ? 0.f : mn;
+        const float alpha = ex2(m - mu);
+        const float pv = ex2(x - mu);
+        l = l * alpha + ((lane & 1) ? 0.f : pv);
+        m = mn;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] *= alpha;
+
+#pragma unroll
+        for (int it = 0; it < ITER; ++it) {
+            const float pt = __shfl_sync(0xffffffffu, pv, half * LPT + 2 * it);
+            const int t = TPI * it + half;
+            if (t < valid) {
+                const int r = kWarpTokens * warp + t;
+                const uint4 w = lds128(v_smem + col + r * 128 + ((j ^ (r & 7)) << 4));
+                acc[0] = fmaf(pt, bf16lo_to_f32(w.x), acc[0]);
+                acc[1] = fmaf(pt, bf16hi_to_f32(w.x), acc[1]);
+                acc[2] = fmaf(pt, bf16lo_to_f32(w.y), acc[2]);
+                acc[3] = fmaf(pt, bf16hi_to_f32(w.y), acc[3]);
+                acc[4] = fmaf(pt, bf16lo_to_f32(w.z), acc[4]);
+                acc[5] = fmaf(pt, bf16hi_to_f32(w.z), acc[5]);
+                acc[6] = fmaf(pt, bf16lo_to_f32(w.w), acc[6]);
+                acc[7] = fmaf(pt, bf16hi_to_f32(w.w), acc[7]);
+            }
+        }
+    }
+
+    __device__ __forceinline__ void to_smem(float *wb) {
+        const int lane = threadIdx.x & 31;
+#pragma unroll
+        for (int s = LPT; s < 32; s <<= 1)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], s);
+        float ls = l;
+#pragma unroll
+        for (int s = 1; s < 32; s <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, s);
+        if (lane < LPT) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) wb[8 * lane + k] = acc[k];
+        }
+        if (lane == 0) {
+            wb[D] = m;
+            wb[D + 1] = ls;
+        }
+    }
+};
+
+// ------------------------------------------------------------------ kernel --
+template <int D, class Consumer>
+__global__ void __launch_bounds__(kSplitThreads, 1)
+    fd_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const SplitParams p) {
+    using Cfg = SplitConfig<D>;
+    constexpr int G = Consumer::G;
+    constexpr int kWarpFloats = G * D + 2 * G;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *ring = smem;
+    float *merge = reinterpret_cast<float *>(ring + Cfg::kRingBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(merge + kConsumerWarps * kWarpFloats);
+    uint64_t *empty = full + Cfg::kStages;
+    StartInfo *info = reinterpret_cast<StartInfo *>(empty + Cfg::kStages);
+
+    // Let the combine kernel (launched behind this one) be scheduled early;
+    // it waits for this grid's completion before reading anything.
+    grid_dependents_launch();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 0) find_start(p, info);
+    __syncthreads();
+
+    long long remaining = info->count;
+    if (remaining <= 0) return;
+    Cursor c{info->b, info->h, info->tile, info->n};
+    volatile int *abort = &info->abort;
+
+    if (warp == kConsumerWarps) {
+        // ---------------------------------------------------- producer --
+        if (lane != 0) return;
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        const uint64_t policy = l2_policy_evict_first();
+        int stage = 0;
+        uint32_t phase = 0;
+        while (remaining > 0) {
+            const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
+            const int z = c.b * p.Hkv + c.h;
+            for (int k = 0; k < seg; ++k) {
+                if (!wait_bounded(&empty[stage], phase ^ 1u, abort)) return;
+                uint8_t *kt = ring + stage * 2 * Cfg::kTileBytes;
+                uint8_t *vt = kt + Cfg::kTileBytes;
+                mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kTileBytes);
+                const int y = (c.tile + k) * kTileTokens;
+#pragma unroll
+                for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+                    tma_load_3d(kt + bx * kBoxBytes, &tm_k, &full[stage], 64 * bx, y, z, policy);
+                    tma_load_3d(vt + bx * kBoxBytes, &tm_v, &full[stage], 64 * bx, y, z, policy);
+                }
+                if (++stage == Cfg::kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            remaining -= seg;
+            if (remaining > 0) next_row(c, p);
+        }
+        return;
+    }
+
+    // -------------------------------------------------------- consumers --
+    Consumer cons;
+    float *wb = merge + warp * kWarpFloats;
+    int stage = 0;
+    uint32_t phase = 0;
+    while (remaining > 0) {
+        const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
+        const int L = clamp_len(__ldg(p.seqlens + c.b), p.Lmax);
+        const bool whole = c.tile == 0 && seg == c.n;
+        cons.begin_row(p, c);
+        for (int k = 0; k < seg; ++k) {
+            wait_bounded(&full[stage], phase, abort);   // on abort: keep going, outputs are flagged invalid
+            const uint32_t kt = smem_addr(ring + stage * 2 * Cfg::kTileBytes);
+            const int valid = L - ((c.tile + k) * kTileTokens + kWarpTokens * warp);
+            cons.tile(kt, kt + Cfg::kTileBytes, valid, p.scale_log2e);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == Cfg::kStages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        cons.to_smem(wb);
+        named_barrier_sync(1, kConsumerThreads);
+        merge_and_store<D, G>(merge, p, c, whole, blockIdx.x + c.b * p.Hkv + c.h);
+        named_barrier_sync(1, kConsumerThreads);
+        remaining -= seg;
+        if (remaining > 0) next_row(c, p);
+    }
+}
+
+}  // namespace fd

@@ -1,0 +1,171 @@
+/*
+ * fd.h -- split-KV decode attention ("Flash-Decoding") for NVIDIA B200, sm_100a.
+ *
+ * THE OPERATION
+ * "Flash-Decoding for long-context inference" (Tri Dao, Daniel Haziza,
+ * Francisco Massa, Grigory Sizov), section "Multi-head attention for
+ * decoding": while decoding, the query of the one new token of each sequence
+ * attends to every cached key/value of that sequence. For sequence b, query
+ * head i, key/value head j = i / (Hq / Hkv) and L = seqlens[b] cached tokens:
+ *
+ *     z_t       = scale * sum_d q[b,i,d] * k_cache[b,j,t,d]        (t < L)
+ *     lse[b,i]  = log( sum_t exp(z_t) )                            (natural log)
+ *     out[b,i,:]= sum_t exp(z_t - lse[b,i]) * v_cache[b,j,t,:]
+ *
+ * Section "A faster attention for decoding: Flash-Decoding" reaches that
+ * result by splitting the keys/values along the sequence, computing each
+ * split's attention together with one log-sum-exp scalar per row and split,
+ * and reducing over the splits with each one rescaled through its
+ * log-sum-exp. This library does the same on one GPU in two stages:
+ *   split   -- every (sequence, kv-head) row's cached tokens are laid end to
+ *              end in one stream of 64-token tiles, and the stream is cut into
+ *              num_splits equal runs of tiles, one per thread block. A run
+ *              that holds a whole row writes out/lse directly; a run that
+ *              holds part of a row writes that part's normalised output and
+ *              log-sum-exp (one "segment") to the workspace.
+ *   combine -- for each row cut into several segments, the LSE-weighted
+ *              reduction of its segments; rows with no tokens get out = 0,
+ *              lse = -inf.
+ * fd_decode runs both stages; fd_split and fd_combine run one each.
+ *
+ * LAYOUTS (all row-major, contiguous, device memory unless stated)
+ *   q        [B, Hq, D]          bf16 bit patterns (uint16_t), 16-byte aligned
+ *   k_cache  [B, Hkv, Lmax, D]   bf16, 16-byte aligned
+ *   v_cache  [B, Hkv, Lmax, D]   bf16, 16-byte aligned
+ *   seqlens  [B]                 int32 (device); values are clamped to [0, Lmax]
+ *   out      [B, Hq, D]          fp32, 4-byte aligned
+ *   lse      [B, Hq]             fp32 natural-log log-sum-exp, 4-byte aligned
+ *   workspace                    fd_workspace_bytes() bytes, 16-byte aligned
+ * Supported: D in {64, 128}; 1 <= Hq/Hkv <= 16; positions t >= seqlens[b]
+ * are never used (their contents, NaN included, cannot reach the output).
+ *
+ * OWNERSHIP AND ERRORS
+ * Every pointer is owned by the caller; the library allocates nothing and
+ * keeps no state between calls except a per-device cache of the SM count
+ * and a per-device error word (see fd_device_status). Calls are
+ * asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream)
+ * and never synchronise, except fd_device_status. Every entry point returns
+ * FD_OK (0) or a negative FD_ERR_* code; argument checks run before any CUDA
+ * call, so a rejected call launches nothing.
+ */
+#ifndef FD_H_
+#define FD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FD_API __attribute__((visibility("default")))
+#else
+#define FD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FD_OK                 0
+#define FD_ERR_NULL_POINTER  -1   /* a required pointer is NULL */
+#define FD_ERR_SHAPE         -2   /* B, Hq, Hkv < 1, max_len < 0, or sizes beyond the limits below */
+#define FD_ERR_GROUP         -3   /* Hq % Hkv != 0 or Hq / Hkv > 16 */
+#define FD_ERR_HEAD_DIM      -4   /* D is not 64 or 128 */
+#define FD_ERR_ALIGNMENT     -5   /* a pointer breaks the alignment listed above */
+#define FD_ERR_WORKSPACE     -6   /* workspace NULL or smaller than fd_workspace_bytes() */
+#define FD_ERR_SPLITS        -7   /* num_splits < 1 or > FD_MAX_SPLITS */
+#define FD_ERR_DEVICE        -8   /* no usable CUDA device, or not compute capability 10.0 */
+#define FD_ERR_LAUNCH        -9   /* a kernel launch (or tensor-map encode) failed */
+#define FD_ERR_TIMEOUT      -10   /* a device-side wait gave up (reported by fd_device_status) */
+#define FD_ERR_CAPACITY     -11   /* an output array passed to fd_segments is too small */
+
+#define FD_TILE_TOKENS     64     /* tokens per tile; split boundaries are multiples of this */
+#define FD_MAX_SPLITS      65535
+#define FD_MAX_GROUP       16
+
+/* Number of splits (thread blocks of the split stage) for a problem shape,
+ * sized to the current device's SM count: one block per SM while the batch
+ * holds at least 4 tiles (256 tokens) per block, fewer for small problems.
+ * Pure function of its arguments and the SM count (queried once per device).
+ * Returns num_splits >= 1, or a negative FD_ERR_* code.
+ * Reading of the page's dispatcher (the library picks Flash-Decoding or a
+ * plain single-pass kernel by problem size): num_splits = 1 is the
+ * unsplit case. */
+FD_API int fd_plan(int B, int Hq, int Hkv, int D, int max_len);
+
+/* fd_plan with the SM count given instead of queried; no CUDA call. */
+FD_API int fd_plan_for_sms(int B, int Hq, int Hkv, int D, int max_len, int num_sms);
+
+/* Workspace bytes that fd_decode / fd_split / fd_combine need for
+ * num_splits splits: room for (num_splits + B*Hkv - 1) segments of
+ * Hq/Hkv rows, each D fp32 outputs plus one fp32 log-sum-exp, laid out as
+ *     seg_out [num_segments][Hq/Hkv][D]  fp32, then (256-byte aligned)
+ *     seg_lse [num_segments][Hq/Hkv]     fp32.
+ * Returns 0 when num_splits == 1 (no row is ever cut) or the arguments are
+ * invalid. */
+FD_API size_t fd_workspace_bytes(int B, int Hq, int Hkv, int D, int max_len, int num_splits);
+
+/* Decode attention with num_splits = fd_plan(B, Hq, Hkv, D, max_len).
+ * Writes out and lse for every (b, i). Enqueues two kernels on `stream`. */
+FD_API int fd_decode(int B, int Hq, int Hkv, int D, int max_len,
+              const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+              const int32_t *seqlens, float scale,
+              float *out, float *lse,
+              void *workspace, size_t workspace_bytes, void *stream);
+
+/* fd_decode with an explicit num_splits in [1, FD_MAX_SPLITS]; every value
+ * gives the same result up to fp32 rounding (the split identity). */
+FD_API int fd_decode_splits(int B, int Hq, int Hkv, int D, int max_len,
+                     const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                     const int32_t *seqlens, float scale,
+                     float *out, float *lse,
+                     void *workspace, size_t workspace_bytes,
+                     int num_splits, void *stream);
+
+/* Split stage alone: for each run of tiles, writes out/lse of the rows it
+ * holds whole and the segments of the rows it holds in part. Rows with no
+ * tokens and rows cut into several segments are left for fd_combine. */
+FD_API int fd_split(int B, int Hq, int Hkv, int D, int max_len,
+             const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+             const int32_t *seqlens, float scale,
+             float *out, float *lse,
+             void *workspace, size_t workspace_bytes,
+             int num_splits, void *stream);
+
+/* Combine stage alone: reads the segments that fd_split wrote for the same
+ * (shape, seqlens, num_splits) and writes out/lse of every row cut into
+ * several segments (segment order fixed, so the result is deterministic),
+ * and out = 0, lse = -inf for rows with no tokens. */
+FD_API int fd_combine(int B, int Hq, int Hkv, int D, int max_len,
+               const int32_t *seqlens,
+               float *out, float *lse,
+               const void *workspace, size_t workspace_bytes,
+               int num_splits, void *stream);
+
+/* Host-side description of where the split stage cuts each row, for host
+ * seqlens (HOST memory, [B]). For every segment slot s < capacity:
+ * seg_row[s] = b*Hkv + j of the row it belongs to, or -1 if the slot is
+ * unused; [seg_begin[s], seg_end[s]) = its token range (clipped to the
+ * row's length). seg_whole[s] = 1 if the segment is its row's only one
+ * (then fd_split writes out/lse directly and the slot stays unused in the
+ * workspace). Returns the number of slots (num_splits + B*Hkv - 1), or
+ * FD_ERR_CAPACITY if capacity is smaller, or another FD_ERR_* code. */
+FD_API int fd_segments(int B, int Hkv, int max_len, const int32_t *seqlens_host, int num_splits,
+                int32_t *seg_row, int32_t *seg_begin, int32_t *seg_end, int32_t *seg_whole,
+                int capacity);
+
+/* Waits for `stream`, then returns and clears this device's error word:
+ * FD_OK, or FD_ERR_TIMEOUT if a kernel's bounded wait gave up (the kernel
+ * then returned early and its outputs are invalid). FD_ERR_LAUNCH if the
+ * stream itself reports an error. */
+FD_API int fd_device_status(void *stream);
+
+/* Text for an FD_* code (static storage). */
+FD_API const char *fd_strerror(int code);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+FD_API int fd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FD_H_ */
