@@ -36,6 +36,33 @@ NOMINAL_HBM_GBS = 8000.0
 L2_BYTES = 126 * 1024 * 1024
 
 
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources (decode_attention_07_b200/csrc/*, include/fd.h)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "decode_attention_07_b200", "csrc", "*")))
+    for f in files + [os.path.join(ROOT, "include", "fd.h")]:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    """Per-launch DRAM bytes (read + write) recorded in profiles/traffic.txt
+    for this workload, if the kernel sources are unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 4 and not line.startswith("#") and parts[0] == workload and parts[1] == want:
+                return int(parts[2]) + int(parts[3])
+    return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -129,36 +156,38 @@ def byte_counts(w, lens, S):
 
 def oracle_sample(x, budget_s=12.0, nthreads=0):
     """Time the CPU oracle on a bounded sample of the workload: whole
-    (sequence, kv-head) rows, all of their query heads, until about
-    `budget_s` seconds of work. Returns (kv_bytes_processed, seconds,
-    threads, description)."""
+    sequences (all kv heads and query heads; the oracle spreads the rows over
+    the host cores), longest first, until about `budget_s` seconds of work;
+    a sequence too long for the budget is cut to its first kv heads.
+    Returns (kv_bytes_processed, seconds, threads, description)."""
     import oracle
     w = x.workload
-    order = np.argsort(-x.seqlens_host, kind="stable")     # longest sequences first: full-length rows
+    orc = oracle.default()
+    order = np.argsort(-x.seqlens_host, kind="stable")
     done_bytes, spent, rows, threads = 0, 0.0, 0, 0
-    host = {}
     for b in order:
         L = int(min(max(x.seqlens_host[b], 0), w.Lmax))
         if L == 0:
             continue
-        for j in range(w.Hkv):
-            key = (int(b), j)
-            if key not in host:
-                host[key] = (bf16_bits(x.q[b:b + 1, j * w.g:(j + 1) * w.g]), bf16_bits(x.k[b:b + 1, j:j + 1, :L]),
-                             bf16_bits(x.v[b:b + 1, j:j + 1, :L]))
-            qh, kh, vh = host[key]
-            orc = oracle.default()
+        # kv heads per call: enough rows to occupy the cores, few enough to stay in budget
+        step = max(1, min(w.Hkv, (os.cpu_count() or 1) // max(1, w.g)))
+        for j0 in range(0, w.Hkv, step):
+            j1 = min(w.Hkv, j0 + step)
+            qh = bf16_bits(x.q[b:b + 1, j0 * w.g:j1 * w.g])
+            kh = bf16_bits(x.k[b:b + 1, j0:j1, :L])
+            vh = bf16_bits(x.v[b:b + 1, j0:j1, :L])
             t0 = time.perf_counter()
             orc.attention(qh, kh, vh, np.array([L], np.int32), x.scale, nthreads)
             spent += time.perf_counter() - t0
             threads = max(threads, orc.threads_used)
-            done_bytes += L * w.D * 2 * 2
-            rows += 1
+            done_bytes += (j1 - j0) * L * w.D * 2 * 2
+            rows += j1 - j0
             if spent >= budget_s:
                 break
         if spent >= budget_s:
             break
-    desc = f"{rows} (sequence, kv-head) rows x {w.g} query heads of {w.name} seed {x.seed}, longest sequences first"
+    desc = (f"{rows} (sequence, kv-head) rows x {w.g} query heads of {w.name} seed {x.seed}, "
+            f"longest sequences first; KV bytes of the sample / oracle seconds")
     return done_bytes, spent, threads, desc
 
 
@@ -189,6 +218,27 @@ def run_reference(args, w, rank, world):
     return 0
 
 
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank decodes its own independent batch: seed + rank."""
+    return int(seed) + int(rank)
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The slowest rank's value (device time is reported as the max over
+    ranks). Works on any process group: NCCL with a CUDA device, gloo on CPU."""
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized() and \
+            torch.distributed.get_world_size() > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_rank_step: float, steps: int, ms_max: float) -> float:
+    """Weak scaling: every rank moves the same bytes per step; the job's rate
+    is all ranks' bytes over the slowest rank's time."""
+    return world * bytes_per_rank_step * steps / (ms_max * 1e-3) / 1e9
+
+
 def config_dict(w, S, l2):
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "Lmax": w.Lmax,
             "ragged": w.ragged, "num_splits": S, "l2": l2, "description": w.description}
@@ -201,7 +251,7 @@ def run_fd(args, w, rank, world):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.Lmax)
-    xs = [make_inputs(w, args.seed + rank, device=dev)]
+    xs = [make_inputs(w, rank_seed(args.seed, rank), device=dev)]
     kv_per_copy = xs[0].kv_bytes()
     if kv_per_copy >= L2_BYTES:
         # rotate input copies so every call streams bytes that are not in L2
@@ -211,58 +261,60 @@ def run_fd(args, w, rank, world):
         n_copies = 1
         l2_note = "L2 flushed before every timed call (256 MiB write outside the timed events)"
     for c in range(1, n_copies):
-        xs.append(make_inputs(w, args.seed + rank + 1000 * c, device=dev))
+        xs.append(make_inputs(w, rank_seed(args.seed, rank) + 1000 * c, device=dev))
     nbytes = fd.fd_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, w.Lmax, S)
-    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=dev)      # row counters start at zero
     out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
     lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if n_copies == 1 else None
     counts = byte_counts(w, xs[0].seqlens_host, S)
     kv_bytes = sum(x.kv_bytes() for x in xs) / n_copies
-
-    def call(x):
-        fd.fd_decode(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, stream)
+    calls = [fd.prepare_decode(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream) for x in xs]
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
     for i in range(max(3, args.warmup)):
-        call(xs[i % n_copies])
+        calls[i % n_copies]()
     torch.cuda.synchronize(dev)
 
-    # ---- main timed region: K calls, one event pair per call -------------
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # ---- main timed region: K calls back to back, one event pair ---------
+    # (the small workload, whose inputs fit in L2, is instead flushed before
+    # each call and timed call by call, flush outside the events)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps if flush is not None else 1)]
     barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clocks:
         t_wall = time.perf_counter()
-        for i in range(args.steps):
-            if flush is not None:
+        if flush is None:
+            ev[0][0].record(stream)
+            for i in range(args.steps):
+                calls[i % n_copies]()
+            ev[0][1].record(stream)
+        else:
+            for i in range(args.steps):
                 flush.fill_(i & 255)
-            ev[i][0].record(stream)
-            call(xs[i % n_copies])
-            ev[i][1].record(stream)
+                ev[i][0].record(stream)
+                calls[0]()
+                ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
         # keep the sampler on the same work for >= 1.5 s so clocks are seen under load
-        t_min = time.perf_counter() + 1.5
+        t_min = time.perf_counter() + (0.0 if args.no_clock_window else 1.5)
         j = 0
         while time.perf_counter() < t_min:
             for _ in range(50):
-                call(xs[j % n_copies])
+                calls[j % n_copies]()
                 j += 1
             torch.cuda.synchronize(dev)
         wall = time.perf_counter() - t_wall
     barrier()
-    ms = sum(a.elapsed_time(b) for a, b in ev)
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev)
     us_per_call = ms_max * 1e3 / args.steps
-    gbs = world * kv_bytes * args.steps / (ms_max * 1e-3) / 1e9
+    gbs = whole_job_gbs(world, kv_bytes, args.steps, ms_max)
 
-    # ---- per-stage device time (split kernel alone, then combine alone) ----
+    # ---- the two stages as separate kernels (for the per-stage split) ------
     ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
              torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for i in range(args.steps):
@@ -296,7 +348,7 @@ def run_fd(args, w, rank, world):
             dk.copy_(hk, non_blocking=True)
             dv.copy_(hv, non_blocking=True)
             dsq.copy_(hs, non_blocking=True)
-            fd.fd_decode(dq, dk, dv, dsq, x.scale, out, lse, ws, stream)
+            fd.fd_decode_splits(dq, dk, dv, dsq, x.scale, out, lse, ws, S, stream)
             ho.copy_(out, non_blocking=True)
             hl.copy_(lse, non_blocking=True)
 
@@ -309,12 +361,10 @@ def run_fd(args, w, rank, world):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        ems = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(ems, op=torch.distributed.ReduceOp.MAX)
-        e2e = {"value": world * x.kv_bytes() * e_steps / (float(ems.item()) * 1e-3) / 1e9, "unit": "GB/s",
+        ems = max_over_ranks(e0.elapsed_time(e1), dev)
+        e2e = {"value": whole_job_gbs(world, x.kv_bytes(), e_steps, ems), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
-               "us_per_call": float(ems.item()) * 1e3 / e_steps}
+               "us_per_call": ems * 1e3 / e_steps}
 
     status = fd.fd_device_status(stream)
     if status != 0:
@@ -323,7 +373,7 @@ def run_fd(args, w, rank, world):
     if rank != 0:
         return 0
     peak, peak_kind = peaks()
-    split_gbs = counts["split"] / (split_us * 1e-6) / 1e9
+    kernel_gbs = counts["total"] / (us_per_call * 1e-6) / 1e9
     line = {
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_max / args.steps, "us_per_call": us_per_call,
@@ -332,11 +382,13 @@ def run_fd(args, w, rank, world):
         "pct_of_nominal_hbm": 100.0 * gbs / world / NOMINAL_HBM_GBS,
         "pct_of_measured_copy": 100.0 * gbs / world / peak,
         "call_bytes_gbs": world * counts["total"] * args.steps / (ms_max * 1e-3) / 1e9,
-        "roofline": {"kernel": "fd_split_kernel", "bound": "hbm", "achieved": split_gbs, "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": split_gbs / peak, "traffic": None,
-                     "bytes_per_launch": counts["split"], "us_per_launch": split_us,
-                     "combine_us_per_launch": combine_us},
-        "gpu_launches": 2 * args.steps,
+        "roofline": {"kernel": "fd_split_kernel (fused combine)", "bound": "hbm", "achieved": kernel_gbs,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": kernel_gbs / peak,
+                     "traffic": measured_traffic(w.name), "bytes_per_launch": counts["total"],
+                     "us_per_launch": us_per_call,
+                     "frac_of_nominal_8tbs": kernel_gbs / NOMINAL_HBM_GBS},
+        "stages_alone": {"split_us": split_us, "combine_us": combine_us},
+        "gpu_launches": args.steps,
         "clocks": clocks.summary(),
         "e2e": e2e,
         "wall_s": wall,
@@ -360,6 +412,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-clock-window", action="store_true",
+                    help="do not extend clock sampling past the timed region (for profiler runs)")
     args = ap.parse_args()
     w = WORKLOADS[args.config]
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -50,11 +50,12 @@ def lib() -> ctypes.CDLL:
         L.fd_combine.argtypes = [_i] * 5 + [_p, _p, _p, _p, _sz, _i, _p]
         L.fd_segments.argtypes = [_i, _i, _i, _p, _i, _p, _p, _p, _p, _i]
         L.fd_device_status.argtypes = [_p]
+        L.fd_workspace_init.argtypes = [_p, _sz, _p]
         L.fd_strerror.argtypes = [_i]
         L.fd_strerror.restype = ctypes.c_char_p
         L.fd_version.argtypes = []
         for name in ("fd_plan", "fd_plan_for_sms", "fd_decode", "fd_decode_splits", "fd_split", "fd_combine",
-                     "fd_segments", "fd_device_status", "fd_version"):
+                     "fd_segments", "fd_device_status", "fd_version", "fd_workspace_init"):
             getattr(L, name).restype = _i
         _lib = L
     return _lib
@@ -171,6 +172,12 @@ def fd_segments(B: int, Hkv: int, max_len: int, seqlens_host, num_splits: int) -
     return dict(row=arrs[0][:n], begin=arrs[1][:n], end=arrs[2][:n], whole=arrs[3][:n])
 
 
+def fd_workspace_init(workspace, stream=None):
+    wp, wb = _ws(workspace)
+    if wb:
+        _check(lib().fd_workspace_init(wp, wb, _stream(stream, workspace.device)), "fd_workspace_init")
+
+
 def fd_device_status(stream=None, device=None) -> int:
     return lib().fd_device_status(_stream(stream, device))
 
@@ -185,12 +192,36 @@ def fd_version() -> int:
 
 # ------------------------------------------------------------ convenience --
 
+def prepare_decode(q, k_cache, v_cache, seqlens, scale, out, lse, workspace=None, num_splits=None, stream=None):
+    """Check and marshal the arguments once; return a no-argument callable
+    that enqueues fd_decode_splits with those pointers (for decode loops that
+    reuse the same buffers). The planned split count is used by default."""
+    B, Hq, Hkv, D, Lmax = _shapes(q, k_cache, v_cache)
+    _outputs(out, lse, B, Hq, D)
+    _seqlens(seqlens, B)
+    S = fd_plan(B, Hq, Hkv, D, Lmax) if num_splits is None else int(num_splits)
+    wp, wb = _ws(workspace)
+    fn = lib().fd_decode_splits
+    args = (B, Hq, Hkv, D, Lmax, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+            ctypes.c_float(scale), out.data_ptr(), lse.data_ptr(), wp, wb, S, _stream(stream, q.device))
+
+    def call():
+        rc = fn(*args)
+        if rc != 0:
+            raise FdError(rc, "fd_decode_splits")
+
+    call.num_splits = S
+    return call
+
+
 def workspace_layout(B, Hq, Hkv, D, num_splits):
-    """(slots, g, byte offset of seg_lse) of the documented workspace layout."""
+    """(slots, g, byte offset of seg_lse, byte offset of the row counters) of
+    the documented workspace layout."""
     slots = num_splits + B * Hkv - 1
     g = Hq // Hkv
     off = (slots * g * D * 4 + 255) // 256 * 256
-    return slots, g, off
+    tick = off + (slots * g * 4 + 255) // 256 * 256
+    return slots, g, off, tick
 
 
 def decode(q, k_cache, v_cache, seqlens, scale, num_splits=None, stream=None):
@@ -199,7 +230,7 @@ def decode(q, k_cache, v_cache, seqlens, scale, num_splits=None, stream=None):
     B, Hq, Hkv, D, Lmax = _shapes(q, k_cache, v_cache)
     S = fd_plan(B, Hq, Hkv, D, Lmax) if num_splits is None else int(num_splits)
     nbytes = fd_workspace_bytes(B, Hq, Hkv, D, Lmax, S)
-    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device) if nbytes else None
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
     out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
     lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     fd_decode_splits(q, k_cache, v_cache, seqlens, scale, out, lse, ws, S, stream)

@@ -42,11 +42,26 @@ long long num_slots(int B, int Hkv, int num_splits) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-size_t workspace_bytes(int B, int Hq, int Hkv, int D, int num_splits) {
-    if (num_splits <= 1) return 0;
+// Workspace: seg_out [slots][g][D] fp32 | seg_lse [slots][g] fp32 | row tickets [B*Hkv] int32,
+// each part 256-byte aligned.
+struct WorkspaceLayout {
+    size_t seg_out, seg_lse, tickets, total;
+};
+
+WorkspaceLayout workspace_layout(int B, int Hq, int Hkv, int D, int num_splits) {
+    WorkspaceLayout w{0, 0, 0, 0};
+    if (num_splits <= 1) return w;
     const size_t slots = static_cast<size_t>(num_slots(B, Hkv, num_splits));
     const size_t g = static_cast<size_t>(Hq / Hkv);
-    return align256(slots * g * D * sizeof(float)) + align256(slots * g * sizeof(float));
+    w.seg_out = 0;
+    w.seg_lse = align256(slots * g * D * sizeof(float));
+    w.tickets = w.seg_lse + align256(slots * g * sizeof(float));
+    w.total = w.tickets + align256(static_cast<size_t>(B) * Hkv * sizeof(int));
+    return w;
+}
+
+size_t workspace_bytes(int B, int Hq, int Hkv, int D, int num_splits) {
+    return workspace_layout(B, Hq, Hkv, D, num_splits).total;
 }
 
 // ------------------------------------------------------------ device info --
@@ -54,7 +69,6 @@ struct DeviceInfo {
     bool queried = false;
     int status = FD_OK;
     int sms = 0;
-    bool split_attr_set = false;
 };
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_mutex;
@@ -126,37 +140,56 @@ int encode_cache_map(CUtensorMap *map, const void *base, int D, int Lmax, long l
 }
 
 // ---------------------------------------------------------------- launches --
-template <int D, class Consumer>
+template <int D, class Consumer, bool kFused>
 int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p, cudaStream_t st) {
-    constexpr int smem = fd::split_smem_bytes<D, Consumer::G>();
-    auto kern = fd::fd_split_kernel<D, Consumer>;
-    // the attribute is per function; setting it again is cheap and thread-safe
+    constexpr int smem = fd::SplitConfig<D, Consumer::G>::kSmemBytes;
+    auto kern = fd::fd_split_kernel<D, Consumer, kFused>;
+    // the attribute is per function and device; set it once per device
     static std::once_flag once[kMaxDevices];
+    static cudaError_t attr_err[kMaxDevices];
     int dev = 0;
-    cudaGetDevice(&dev);
-    cudaError_t attr_err = cudaSuccess;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return FD_ERR_DEVICE;
+    }
     std::call_once(once[dev], [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        attr_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     });
-    if (attr_err != cudaSuccess) {
+    if (attr_err[dev] != cudaSuccess) {
         cudaGetLastError();
         return FD_ERR_LAUNCH;
     }
-    kern<<<p.P, fd::kSplitThreads, smem, st>>>(tk, tv, p);
-    if (cudaGetLastError() != cudaSuccess) return FD_ERR_LAUNCH;
+    // programmatic dependent launch: the prologue overlaps the previous
+    // kernel's tail; the kernel waits for it before reading any input
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(static_cast<unsigned>(p.P));
+    cfg.blockDim = dim3(fd::kSplitThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tk, tv, p) != cudaSuccess) {
+        cudaGetLastError();
+        return FD_ERR_LAUNCH;
+    }
     return FD_OK;
 }
 
+template <bool kFused>
 int launch_split(int D, int g, const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p,
                  cudaStream_t st) {
     if (D == 128) {
-        if (g == 1) return launch_split_t<128, fd::HeadConsumer<128>>(tk, tv, p, st);
-        if (g <= 8) return launch_split_t<128, fd::GroupConsumer<128, 1>>(tk, tv, p, st);
-        return launch_split_t<128, fd::GroupConsumer<128, 2>>(tk, tv, p, st);
+        if (g == 1) return launch_split_t<128, fd::HeadConsumer<128>, kFused>(tk, tv, p, st);
+        if (g <= 8) return launch_split_t<128, fd::GroupConsumer<128, 1>, kFused>(tk, tv, p, st);
+        return launch_split_t<128, fd::GroupConsumer<128, 2>, kFused>(tk, tv, p, st);
     }
-    if (g == 1) return launch_split_t<64, fd::HeadConsumer<64>>(tk, tv, p, st);
-    if (g <= 8) return launch_split_t<64, fd::GroupConsumer<64, 1>>(tk, tv, p, st);
-    return launch_split_t<64, fd::GroupConsumer<64, 2>>(tk, tv, p, st);
+    if (g == 1) return launch_split_t<64, fd::HeadConsumer<64>, kFused>(tk, tv, p, st);
+    if (g <= 8) return launch_split_t<64, fd::GroupConsumer<64, 1>, kFused>(tk, tv, p, st);
+    return launch_split_t<64, fd::GroupConsumer<64, 2>, kFused>(tk, tv, p, st);
 }
 
 int launch_combine(int D, const fd::CombineParams &p, cudaStream_t st, bool after_split) {
@@ -201,7 +234,7 @@ int check_problem(const Problem &pr, bool need_kv) {
     // with max_len == 0 no token exists and q/k/v are never read (they may be NULL)
     const bool reads_kv = need_kv && pr.max_len > 0;
     if (reads_kv && (!pr.q || !pr.k || !pr.v)) return FD_ERR_NULL_POINTER;
-    if (!aligned(pr.seqlens, 4) || !aligned(pr.out, 4) || !aligned(pr.lse, 4)) return FD_ERR_ALIGNMENT;
+    if (!aligned(pr.seqlens, 4) || !aligned(pr.out, 16) || !aligned(pr.lse, 4)) return FD_ERR_ALIGNMENT;
     if (reads_kv && (!aligned(pr.q, 16) || !aligned(pr.k, 16) || !aligned(pr.v, 16))) return FD_ERR_ALIGNMENT;
     const size_t need = workspace_bytes(pr.B, pr.Hq, pr.Hkv, pr.D, pr.num_splits);
     if (need > 0) {
@@ -213,32 +246,41 @@ int check_problem(const Problem &pr, bool need_kv) {
     return FD_OK;
 }
 
-void seg_pointers(const Problem &pr, float **so, float **sl) {
-    if (workspace_bytes(pr.B, pr.Hq, pr.Hkv, pr.D, pr.num_splits) == 0) {
+void seg_pointers(const Problem &pr, float **so, float **sl, int **tickets) {
+    const WorkspaceLayout w = workspace_layout(pr.B, pr.Hq, pr.Hkv, pr.D, pr.num_splits);
+    if (w.total == 0) {
         *so = *sl = nullptr;
+        *tickets = nullptr;
         return;
     }
-    const size_t slots = static_cast<size_t>(num_slots(pr.B, pr.Hkv, pr.num_splits));
-    const size_t g = static_cast<size_t>(pr.Hq / pr.Hkv);
-    *so = static_cast<float *>(pr.ws);
-    *sl = reinterpret_cast<float *>(static_cast<char *>(pr.ws) + align256(slots * g * pr.D * sizeof(float)));
+    char *base = static_cast<char *>(pr.ws);
+    *so = reinterpret_cast<float *>(base + w.seg_out);
+    *sl = reinterpret_cast<float *>(base + w.seg_lse);
+    *tickets = reinterpret_cast<int *>(base + w.tickets);
 }
 
-int run_split(const Problem &pr) {
-    if (pr.max_len == 0) return FD_OK;   // no tokens anywhere: nothing to stream
+// The split kernel; `fused` adds the in-kernel combine (fd_decode), without it
+// the segments are left for fd_combine.
+int run_split(const Problem &pr, bool fused) {
     int sms;
     int rc = device_sms(&sms);
     if (rc != FD_OK) return rc;
     CUtensorMap tk, tv;
+    std::memset(&tk, 0, sizeof tk);
+    std::memset(&tv, 0, sizeof tv);
     const long long rows = static_cast<long long>(pr.B) * pr.Hkv;
-    if ((rc = encode_cache_map(&tk, pr.k, pr.D, pr.max_len, rows)) != FD_OK) return rc;
-    if ((rc = encode_cache_map(&tv, pr.v, pr.D, pr.max_len, rows)) != FD_OK) return rc;
+    if (pr.max_len > 0) {
+        if ((rc = encode_cache_map(&tk, pr.k, pr.D, pr.max_len, rows)) != FD_OK) return rc;
+        if ((rc = encode_cache_map(&tv, pr.v, pr.D, pr.max_len, rows)) != FD_OK) return rc;
+    } else if (!fused) {
+        return FD_OK;   // no tokens anywhere: the combine writes every row
+    }
     fd::SplitParams p;
     p.q = pr.q;
     p.seqlens = pr.seqlens;
     p.out = pr.out;
     p.lse = pr.lse;
-    seg_pointers(pr, &p.seg_out, &p.seg_lse);
+    seg_pointers(pr, &p.seg_out, &p.seg_lse, &p.row_tickets);
     p.B = pr.B;
     p.Hq = pr.Hq;
     p.Hkv = pr.Hkv;
@@ -246,7 +288,10 @@ int run_split(const Problem &pr) {
     p.Lmax = pr.max_len;
     p.P = pr.num_splits;
     p.scale_log2e = pr.scale * kLog2e;
-    return launch_split(pr.D, p.g, tk, tv, p, pr.stream);
+    // with max_len == 0 every block finds zero tiles and only writes empty rows;
+    // the (unused) tensor maps stay zeroed
+    return fused ? launch_split<true>(pr.D, p.g, tk, tv, p, pr.stream)
+                 : launch_split<false>(pr.D, p.g, tk, tv, p, pr.stream);
 }
 
 int run_combine(const Problem &pr, bool after_split) {
@@ -258,7 +303,8 @@ int run_combine(const Problem &pr, bool after_split) {
     p.out = pr.out;
     p.lse = pr.lse;
     float *so, *sl;
-    seg_pointers(pr, &so, &sl);
+    int *tickets;
+    seg_pointers(pr, &so, &sl, &tickets);
     p.seg_out = so;
     p.seg_lse = sl;
     p.B = pr.B;
@@ -331,8 +377,7 @@ int fd_decode_splits(int B, int Hq, int Hkv, int D, int max_len, const uint16_t 
                               workspace_bytes, num_splits, stream);
     int rc = check_problem(pr, true);
     if (rc != FD_OK) return rc;
-    if ((rc = run_split(pr)) != FD_OK) return rc;
-    return run_combine(pr, true);
+    return run_split(pr, true);
 }
 
 int fd_decode(int B, int Hq, int Hkv, int D, int max_len, const uint16_t *q, const uint16_t *k_cache,
@@ -353,7 +398,7 @@ int fd_split(int B, int Hq, int Hkv, int D, int max_len, const uint16_t *q, cons
                               workspace_bytes, num_splits, stream);
     int rc = check_problem(pr, true);
     if (rc != FD_OK) return rc;
-    return run_split(pr);
+    return run_split(pr, false);
 }
 
 int fd_combine(int B, int Hq, int Hkv, int D, int max_len, const int32_t *seqlens, float *out, float *lse,
@@ -362,7 +407,7 @@ int fd_combine(int B, int Hq, int Hkv, int D, int max_len, const int32_t *seqlen
                               const_cast<void *>(workspace), workspace_bytes, num_splits, stream);
     int rc = check_problem(pr, false);
     if (rc != FD_OK) return rc;
-    return run_combine(pr, false);
+    return run_combine(pr, true);
 }
 
 int fd_segments(int B, int Hkv, int max_len, const int32_t *seqlens_host, int num_splits, int32_t *seg_row,
@@ -394,6 +439,7 @@ int fd_segments(int B, int Hkv, int max_len, const int32_t *seqlens_host, int nu
             const int i1 = fd::run_of_tile(first + n - 1, N, num_splits);
             for (int i = i0; i <= i1; ++i) {
                 const long long lo = fd::run_begin(i, N, num_splits), hi = fd::run_begin(i + 1, N, num_splits);
+                if (lo == hi) continue;   // more runs than tiles: this run is empty
                 const long long t0 = (lo > first ? lo : first) - first;
                 const long long t1 = (hi < first + n ? hi : first + n) - first;
                 const long long s = i + u;
@@ -407,6 +453,18 @@ int fd_segments(int B, int Hkv, int max_len, const int32_t *seqlens_host, int nu
         before += n;
     }
     return static_cast<int>(slots);
+}
+
+int fd_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
+    if (workspace_bytes == 0) return FD_OK;
+    if (!workspace) return FD_ERR_NULL_POINTER;
+    int dev;
+    if (current_device(&dev) != FD_OK) return FD_ERR_DEVICE;
+    if (cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return FD_ERR_LAUNCH;
+    }
+    return FD_OK;
 }
 
 int fd_device_status(void *stream) {
@@ -433,7 +491,7 @@ const char *fd_strerror(int code) {
         case FD_ERR_SHAPE: return "invalid or too large B / Hq / Hkv / max_len";
         case FD_ERR_GROUP: return "Hq must be a multiple of Hkv with Hq/Hkv <= 16";
         case FD_ERR_HEAD_DIM: return "head dimension D must be 64 or 128";
-        case FD_ERR_ALIGNMENT: return "pointer misaligned (q/k/v/workspace need 16 bytes, seqlens/out/lse 4)";
+        case FD_ERR_ALIGNMENT: return "pointer misaligned (q/k/v/out/workspace need 16 bytes, seqlens/lse 4)";
         case FD_ERR_WORKSPACE: return "workspace missing or smaller than fd_workspace_bytes()";
         case FD_ERR_SPLITS: return "num_splits out of range [1, 65535]";
         case FD_ERR_DEVICE: return "no usable CUDA device of compute capability 10.0";

@@ -1,23 +1,31 @@
-// fd_split.cuh -- the split stage of decode attention (one thread block per run
-// of key/value tiles; see fd_partition.cuh for how runs are cut).
+// fd_split.cuh -- the split stage of decode attention, optionally with the
+// final reduction fused in (one thread block per run of key/value tiles; see
+// fd_partition.cuh for how runs are cut).
 //
 // "Flash-Decoding for long-context inference", section "A faster attention
 // for decoding: Flash-Decoding": each split computes the attention of the
 // query with its chunk of keys/values and writes one extra scalar per row,
 // the log-sum-exp; the softmax can be built up tile by tile ("the
 // attention/softmax can be calculated iteratively"), which is what the
-// running max / running sum below do.
+// running max / running sum below do. A final reduction rescales the splits
+// by their log-sum-exps (fd_merge.cuh).
 //
-// Block layout (160 threads, one block per SM):
-//   warp 4      producer: one lane streams K and V tiles (64 tokens x D bf16
+// Block layout (288 threads, one block per SM):
+//   warp 8      producer: one lane streams K and V tiles (64 tokens x D bf16
 //               each) from HBM into a ring of shared-memory stages with 3-D
-//               TMA loads, 128-byte swizzled; mbarrier completion.
-//   warps 0..3  consumers: warp w owns tokens [16w, 16w+16) of every tile.
-//               Per tile: logits for its 16 tokens, online-softmax update of
-//               the running max m and sum l per query head, and the
-//               rescaled accumulation of p * v; at the end of a row segment
-//               the four warps' (m, l, o) are merged through shared memory
-//               and written out (whole row) or to the workspace (segment).
+//               TMA loads, 128-byte swizzled, mbarrier completion.
+//   warps 0..7  consumers in two groups of four. Group q takes the tiles with
+//               sequence number = q (mod 2), so each SM sub-partition runs two
+//               independent chains; warp w of a group owns tokens
+//               [16w, 16w+16) of its tiles. Per tile: logits, online-softmax
+//               update of the running max m and sum l per query head, and
+//               the rescaled accumulation of p * v. At the end of a row
+//               segment the eight warps' (m, l, o) are merged through shared
+//               memory and written out (whole row) or to the workspace.
+//   fused form: after writing a segment, the block takes a ticket on its
+//               row (atomic counter in the workspace, no waiting); the block
+//               that completes the row merges all its segments and resets
+//               the counter. Rows with no tokens are written by block u % P.
 // Two consumer forms:
 //   * grouped heads (g = Hq/Hkv >= 2): the g query heads that share one kv
 //     head form a small dense contraction, run on tensor cores with
@@ -29,18 +37,21 @@
 //     (D=64) lanes per token, reduced with warp shuffles.
 #pragma once
 
+#include "fd_merge.cuh"
 #include "fd_partition.cuh"
 #include "fd_ptx.cuh"
 
 namespace fd {
 
-constexpr int kConsumerWarps = 4;
+constexpr int kGroups = 2;                        // consumer groups alternating tiles
+constexpr int kSliceWarps = 4;                    // warps per group (16 tokens each)
+constexpr int kConsumerWarps = kGroups * kSliceWarps;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kSplitThreads = kConsumerThreads + 32;
-constexpr int kWarpTokens = 16;                  // tokens of a tile owned by one consumer warp
-constexpr int kBoxBytes = kTileTokens * 128;     // one TMA box: 64 rows x 128 bytes (64 bf16)
-constexpr uint64_t kWaitLimitNs = 2000000000ull; // a bounded wait gives up after 2 s
-constexpr float kLn2 = 0.693147180559945309f;
+constexpr int kWarpTokens = 16;                   // tokens of a tile owned by one consumer warp
+constexpr int kBoxBytes = kTileTokens * 128;      // one TMA box: 64 rows x 128 bytes (64 bf16)
+constexpr int kSmemLimit = 232448;                // 227 KiB opt-in shared memory per block
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a bounded wait gives up after 2 s
 
 // Sticky per-device error word (FD_ERR_TIMEOUT when a wait gave up).
 __device__ int g_fd_error_word;
@@ -52,33 +63,43 @@ struct SplitParams {
     float *lse;               // [B, Hq]
     float *seg_out;           // [slots, g, D]
     float *seg_lse;           // [slots, g]
+    int *row_tickets;         // [B * Hkv], zero between calls (fused form only)
     int B, Hq, Hkv, g, Lmax, P;
     float scale_log2e;        // scale * log2(e): logits are kept in base 2
 };
 
-template <int D>
+template <int D, int G>
 struct SplitConfig {
-    static constexpr int kBoxes = D / 64;                        // 128-byte boxes per row
-    static constexpr int kTileBytes = kTileTokens * D * 2;       // one K (or V) tile
-    static constexpr int kStages = D == 128 ? 4 : 8;             // 128 KiB of ring either way
+    static constexpr int kBoxes = D / 64;                                  // 128-byte boxes per row
+    static constexpr int kTileBytes = kTileTokens * D * 2;                 // one K (or V) tile
+    static constexpr int kWarpFloats = G * D + 2 * G;                      // o, m, l of one warp
+    static constexpr int kMergeBytes = kConsumerWarps * kWarpFloats * 4;
+    static constexpr int kFixedBytes = 1024 + kMergeBytes + 256;           // alignment, merge, barriers
+    static constexpr int kFit = (kSmemLimit - kFixedBytes) / (2 * kTileBytes);
+    static constexpr int kCap = D == 128 ? 4 : 8;                          // 128 KiB of ring: measured best
+    // A multiple of kGroups, so each consumer group owns its own stages: a
+    // stage shared by both groups could be waited on two phases ahead of a
+    // tile still in flight, where a parity wait would pass on the older phase.
+    static constexpr int kStages = ((kFit < kCap ? kFit : kCap) / kGroups) * kGroups;
     static constexpr int kRingBytes = kStages * 2 * kTileBytes;
+    static constexpr int kSmemBytes = 1024 + kRingBytes + kMergeBytes + 256;
+    static_assert(kStages >= 4, "ring too shallow");
+    static_assert(kStages % kGroups == 0, "each consumer group must own whole stages");
+    static_assert(kSmemBytes <= kSmemLimit, "shared memory over the limit");
 };
 
-// Shared-memory bytes of one split block (plus 1 KiB for 1024-byte alignment).
-template <int D, int G>
-constexpr int split_smem_bytes() {
-    return 1024 + SplitConfig<D>::kRingBytes + kConsumerWarps * (G * D + 2 * G) * 4 +
-           2 * SplitConfig<D>::kStages * 8 + 64;
-}
-
 struct Cursor {
-    int b, h, tile, n;   // row (b, h), tile index inside the row, tiles of sequence b
+    int b, h, tile, n;        // row (b, h), tile index inside the row, tiles of sequence b
+    long long first;          // flat index of the row's first tile
 };
 
 struct StartInfo {
-    long long count;     // tiles in this block's run
+    long long count;          // tiles in this block's run
+    long long N;              // tiles in the whole batch
+    long long first;          // flat index of the start row's first tile
     int b, h, tile, n;
-    int abort;           // set when a bounded wait gave up
+    int abort;                // set when a bounded wait gave up
+    int last;                 // this block completes the current row (fused form)
 };
 
 // Bounded mbarrier wait. Returns false if the block is aborting or the limit
@@ -104,6 +125,7 @@ __device__ __forceinline__ int row_tiles(const int32_t *seqlens, int b, int Lmax
 
 // Next row with at least one tile (only called while tiles remain).
 __device__ __forceinline__ void next_row(Cursor &c, const SplitParams &p) {
+    c.first += c.n;
     c.tile = 0;
     if (++c.h == p.Hkv) {
         c.h = 0;
@@ -127,6 +149,7 @@ __device__ __forceinline__ void find_start(const SplitParams &p, StartInfo *info
     const long long t0 = run_begin(blockIdx.x, N, p.P);
     const long long t1 = run_begin(blockIdx.x + 1, N, p.P);
     int b = 0, h = 0, tile = 0, n = 0;
+    long long first = 0;
     if (t1 > t0) {
         long long before = 0;   // Hkv * (tiles of sequences before this chunk)
         for (int base = 0; base < p.B; base += 32) {
@@ -142,10 +165,11 @@ __device__ __forceinline__ void find_start(const SplitParams &p, StartInfo *info
                 const int src = __ffs(hit) - 1;
                 b = base + src;
                 n = __shfl_sync(0xffffffffu, nb, src);
-                const long long row0 = __shfl_sync(0xffffffffu, after, src) - static_cast<long long>(p.Hkv) * n;
-                const long long off = t0 - row0;
+                const long long seq0 = __shfl_sync(0xffffffffu, after, src) - static_cast<long long>(p.Hkv) * n;
+                const long long off = t0 - seq0;
                 h = static_cast<int>(off / n);
                 tile = static_cast<int>(off % n);
+                first = seq0 + static_cast<long long>(h) * n;
                 break;
             }
             before += static_cast<long long>(p.Hkv) * __shfl_sync(0xffffffffu, incl, 31);
@@ -153,20 +177,23 @@ __device__ __forceinline__ void find_start(const SplitParams &p, StartInfo *info
     }
     if (lane == 0) {
         info->count = t1 - t0;
+        info->N = N;
+        info->first = first;
         info->b = b;
         info->h = h;
         info->tile = tile;
         info->n = n;
         info->abort = 0;
+        info->last = 0;
     }
 }
 
 // ------------------------------------------------------------ merge + store --
 // Per-warp partial results in shared memory: o[G][D], then m[G], l[G] (m in
-// base-2 units). All 128 consumer threads merge the four warps and store.
+// base-2 units). All consumer threads merge the eight warps and store.
 template <int D, int G>
-__device__ __forceinline__ void merge_and_store(const float *merge, const SplitParams &p, const Cursor &c,
-                                                bool whole, int slot) {
+__device__ __forceinline__ void merge_warps_and_store(const float *merge, const SplitParams &p, const Cursor &c,
+                                                      bool whole, size_t slot) {
     constexpr int kWarpFloats = G * D + 2 * G;
     const int tid = threadIdx.x;
     for (int idx = tid; idx < p.g * D; idx += kConsumerThreads) {
@@ -181,18 +208,18 @@ __device__ __forceinline__ void merge_and_store(const float *merge, const SplitP
             for (int w = 0; w < kConsumerWarps; ++w) {
                 const float *wb = merge + w * kWarpFloats;
                 const float e = ex2(wb[G * D + head] - M);
-                lsum += e * wb[G * D + G + head];
-                acc += e * wb[head * D + d];
+                lsum = fmaf(e, wb[G * D + G + head], lsum);
+                acc = fmaf(e, wb[head * D + d], acc);
             }
             o = acc / lsum;
-            lse_nat = (M + lg2(lsum)) * kLn2;
+            lse_nat = (M + lg2(lsum)) * kLn2F;
         }
         if (whole) {
             const size_t row = static_cast<size_t>(c.b) * p.Hq + static_cast<size_t>(c.h) * p.g + head;
             p.out[row * D + d] = o;
             if (d == 0) p.lse[row] = lse_nat;
         } else {
-            const size_t row = static_cast<size_t>(slot) * p.g + head;
+            const size_t row = slot * p.g + head;
             p.seg_out[row * D + d] = o;
             if (d == 0) p.seg_lse[row] = lse_nat;
         }
@@ -235,17 +262,22 @@ struct GroupConsumer {
         return w & ((t < valid ? 0x0000ffffu : 0u) | (t + 1 < valid ? 0xffff0000u : 0u));
     }
 
-    // One tile: `valid` = tokens of this warp's 16 that are inside the row.
-    __device__ __forceinline__ void tile(uint32_t k_smem, uint32_t v_smem, int valid, float scale_log2e) {
-        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // One tile: `slice` = this warp's 16-token slice, `valid` = how many of
+    // those 16 tokens are inside the row.
+    __device__ __forceinline__ void tile(uint32_t k_smem, uint32_t v_smem, int slice, int valid,
+                                         float scale_log2e) {
+        const int lane = threadIdx.x & 31;
         const int mi = lane >> 3, rr = lane & 7;
         const int r0 = lane >> 2, cc = lane & 3;
 
-        // S^T = K Q^T over this warp's 16 tokens
-        float s[NT][4];
+        // S^T = K Q^T over this warp's 16 tokens (two accumulators: even and
+        // odd k-steps, to halve the dependent mma chain)
+        float s[NT][4], s2[NT][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-        const int krow = kWarpTokens * warp + rr + 8 * (mi & 1);
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
+        const int krow = kWarpTokens * slice + rr + 8 * (mi & 1);
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
             const int d = 16 * ks + 8 * (mi >> 1);
@@ -253,15 +285,20 @@ struct GroupConsumer {
             uint32_t a0, a1, a2, a3;
             ldsm_x4(addr, a0, a1, a2, a3);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+                if (ks & 1)
+                    mma_bf16_16816(s2[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+                else
+                    mma_bf16_16816(s[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+            }
         }
 
         // online softmax per head column; P^T fragments (high + remainder)
         uint32_t bh[NT][2], bl[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            float x0 = s[nt][0] * scale_log2e, x1 = s[nt][1] * scale_log2e;
-            float x2 = s[nt][2] * scale_log2e, x3 = s[nt][3] * scale_log2e;
+            float x0 = (s[nt][0] + s2[nt][0]) * scale_log2e, x1 = (s[nt][1] + s2[nt][1]) * scale_log2e;
+            float x2 = (s[nt][2] + s2[nt][2]) * scale_log2e, x3 = (s[nt][3] + s2[nt][3]) * scale_log2e;
             if (r0 >= valid) x0 = x1 = -INFINITY;
             if (r0 + 8 >= valid) x2 = x3 = -INFINITY;
             float ma = fmaxf(x0, x2), mb = fmaxf(x1, x3);
@@ -274,8 +311,8 @@ struct GroupConsumer {
             const float ua = na == -INFINITY ? 0.f : na, ub = nb == -INFINITY ? 0.f : nb;
             const float alpha_a = ex2(m[nt][0] - ua), alpha_b = ex2(m[nt][1] - ub);
             const float p0 = ex2(x0 - ua), p2 = ex2(x2 - ua), p1 = ex2(x1 - ub), p3 = ex2(x3 - ub);
-            l[nt][0] = l[nt][0] * alpha_a + (p0 + p2);
-            l[nt][1] = l[nt][1] * alpha_b + (p1 + p3);
+            l[nt][0] = fmaf(l[nt][0], alpha_a, p0 + p2);
+            l[nt][1] = fmaf(l[nt][1], alpha_b, p1 + p3);
             m[nt][0] = na;
             m[nt][1] = nb;
 #pragma unroll
@@ -295,7 +332,7 @@ struct GroupConsumer {
         }
 
         // O^T += V^T P^T
-        const int vrow = kWarpTokens * warp + 8 * (mi >> 1) + rr;
+        const int vrow = kWarpTokens * slice + 8 * (mi >> 1) + rr;
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
             const int d = 16 * mt + 8 * (mi & 1);
@@ -380,8 +417,9 @@ struct HeadConsumer {
         return r;
     }
 
-    __device__ __forceinline__ void tile(uint32_t k_smem, uint32_t v_smem, int valid, float scale_log2e) {
-        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __device__ __forceinline__ void tile(uint32_t k_smem, uint32_t v_smem, int slice, int valid,
+                                         float scale_log2e) {
+        const int lane = threadIdx.x & 31;
         const int half = lane / LPT, chunk = lane % LPT;
         const int d0 = 8 * chunk;
         const uint32_t col = (d0 >> 6) * kBoxBytes;
@@ -391,7 +429,7 @@ struct HeadConsumer {
         float pd[ITER];
 #pragma unroll
         for (int it = 0; it < ITER; ++it) {
-            const int r = kWarpTokens * warp + TPI * it + half;
+            const int r = kWarpTokens * slice + TPI * it + half;
             const uint4 w = lds128(k_smem + col + r * 128 + ((j ^ (r & 7)) << 4));
             float a = qv[0] * bf16lo_to_f32(w.x);
             a = fmaf(qv[1], bf16hi_to_f32(w.x), a);
@@ -422,14 +460,14 @@ struct HeadConsumer {
         x *= scale_log2e;
         if (TPI * my_it + half >= valid) x = -INFINITY;
 
-        float mx = x;
+        float mx = x;   // both lanes of a pair hold the same value: skip the xor-1 step
 #pragma unroll
-        for (int sh = 1; sh < 32; sh <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, sh));
+        for (int sh = 2; sh < 32; sh <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, sh));
         const float mn = fmaxf(m, mx);
         const float mu = mn == -INFINITY ? 0.f : mn;
         const float alpha = ex2(m - mu);
         const float pv = ex2(x - mu);
-        l = l * alpha + ((lane & 1) ? 0.f : pv);
+        l = fmaf(l, alpha, (lane & 1) ? 0.f : pv);
         m = mn;
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc[k] *= alpha;
@@ -439,7 +477,7 @@ struct HeadConsumer {
             const float pt = __shfl_sync(0xffffffffu, pv, half * LPT + 2 * it);
             const int t = TPI * it + half;
             if (t < valid) {
-                const int r = kWarpTokens * warp + t;
+                const int r = kWarpTokens * slice + t;
                 const uint4 w = lds128(v_smem + col + r * 128 + ((j ^ (r & 7)) << 4));
                 acc[0] = fmaf(pt, bf16lo_to_f32(w.x), acc[0]);
                 acc[1] = fmaf(pt, bf16hi_to_f32(w.x), acc[1]);
@@ -474,54 +512,60 @@ struct HeadConsumer {
 };
 
 // ------------------------------------------------------------------ kernel --
-template <int D, class Consumer>
+template <int D, class Consumer, bool kFused>
 __global__ void __launch_bounds__(kSplitThreads, 1)
     fd_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const SplitParams p) {
-    using Cfg = SplitConfig<D>;
     constexpr int G = Consumer::G;
-    constexpr int kWarpFloats = G * D + 2 * G;
+    using Cfg = SplitConfig<D, G>;
+    constexpr int kWarpFloats = Cfg::kWarpFloats;
+    constexpr int kStages = Cfg::kStages;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *ring = smem;
     float *merge = reinterpret_cast<float *>(ring + Cfg::kRingBytes);
     uint64_t *full = reinterpret_cast<uint64_t *>(merge + kConsumerWarps * kWarpFloats);
-    uint64_t *empty = full + Cfg::kStages;
-    StartInfo *info = reinterpret_cast<StartInfo *>(empty + Cfg::kStages);
+    uint64_t *empty = full + kStages;
+    StartInfo *info = reinterpret_cast<StartInfo *>(empty + kStages);
 
-    // Let the combine kernel (launched behind this one) be scheduled early;
-    // it waits for this grid's completion before reading anything.
+    // A grid queued behind this one (the next call, or the standalone
+    // combine) may start its prologue now; it waits for this grid's
+    // completion before reading anything.
     grid_dependents_launch();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < Cfg::kStages; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
+            mbar_init(&empty[s], kSliceWarps);
         }
         fence_mbar_init();
     }
+    // Launched as a programmatic dependent of the previous kernel on the
+    // stream: everything above overlaps its tail; inputs are read only after it.
+    grid_dependency_wait();
     if (warp == 0) find_start(p, info);
     __syncthreads();
 
     long long remaining = info->count;
-    if (remaining <= 0) return;
-    Cursor c{info->b, info->h, info->tile, info->n};
+    Cursor c{info->b, info->h, info->tile, info->n, info->first};
+    const long long N = info->N;
     volatile int *abort = &info->abort;
 
     if (warp == kConsumerWarps) {
         // ---------------------------------------------------- producer --
-        if (lane != 0) return;
+        if (lane != 0 || remaining <= 0) return;
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
         const uint64_t policy = l2_policy_evict_first();
-        int stage = 0;
-        uint32_t phase = 0;
+        uint32_t seq = 0;
         while (remaining > 0) {
             const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
             const int z = c.b * p.Hkv + c.h;
-            for (int k = 0; k < seg; ++k) {
+            for (int k = 0; k < seg; ++k, ++seq) {
+                const int stage = static_cast<int>(seq % kStages);
+                const uint32_t phase = (seq / kStages) & 1u;
                 if (!wait_bounded(&empty[stage], phase ^ 1u, abort)) return;
                 uint8_t *kt = ring + stage * 2 * Cfg::kTileBytes;
                 uint8_t *vt = kt + Cfg::kTileBytes;
@@ -532,10 +576,6 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                     tma_load_3d(kt + bx * kBoxBytes, &tm_k, &full[stage], 64 * bx, y, z, policy);
                     tma_load_3d(vt + bx * kBoxBytes, &tm_v, &full[stage], 64 * bx, y, z, policy);
                 }
-                if (++stage == Cfg::kStages) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
             }
             remaining -= seg;
             if (remaining > 0) next_row(c, p);
@@ -544,33 +584,65 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     }
 
     // -------------------------------------------------------- consumers --
+    const int group = warp / kSliceWarps, slice = warp % kSliceWarps;
+    const int tid = threadIdx.x;
+    auto consumers_sync = [] { named_barrier_sync(1, kConsumerThreads); };
     Consumer cons;
     float *wb = merge + warp * kWarpFloats;
-    int stage = 0;
-    uint32_t phase = 0;
+    uint32_t seq = 0;
     while (remaining > 0) {
         const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
         const int L = clamp_len(__ldg(p.seqlens + c.b), p.Lmax);
         const bool whole = c.tile == 0 && seg == c.n;
         cons.begin_row(p, c);
-        for (int k = 0; k < seg; ++k) {
+        for (int k = 0; k < seg; ++k, ++seq) {
+            if (static_cast<int>(seq % kGroups) != group) continue;
+            const int stage = static_cast<int>(seq % kStages);
+            const uint32_t phase = (seq / kStages) & 1u;
             wait_bounded(&full[stage], phase, abort);   // on abort: keep going, outputs are flagged invalid
             const uint32_t kt = smem_addr(ring + stage * 2 * Cfg::kTileBytes);
-            const int valid = L - ((c.tile + k) * kTileTokens + kWarpTokens * warp);
-            cons.tile(kt, kt + Cfg::kTileBytes, valid, p.scale_log2e);
+            const int valid = L - ((c.tile + k) * kTileTokens + kWarpTokens * slice);
+            cons.tile(kt, kt + Cfg::kTileBytes, slice, valid, p.scale_log2e);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
-            if (++stage == Cfg::kStages) {
-                stage = 0;
-                phase ^= 1u;
-            }
         }
         cons.to_smem(wb);
-        named_barrier_sync(1, kConsumerThreads);
-        merge_and_store<D, G>(merge, p, c, whole, blockIdx.x + c.b * p.Hkv + c.h);
-        named_barrier_sync(1, kConsumerThreads);
+        consumers_sync();
+        const long long u = static_cast<long long>(c.b) * p.Hkv + c.h;
+        const size_t slot = static_cast<size_t>(blockIdx.x) + static_cast<size_t>(u);
+        merge_warps_and_store<D, G>(merge, p, c, whole, slot);
+        if (kFused && !whole) {
+            // ticket on the row; the block that completes it merges all segments
+            __threadfence();
+            consumers_sync();
+            if (tid == 0) {
+                const RowRuns rr = row_runs(c.first, c.n, N, p.P);
+                const int prev = atomicAdd(p.row_tickets + u, 1);
+                info->last = prev == rr.count - 1;
+            }
+            consumers_sync();
+            if (*reinterpret_cast<volatile int *>(&info->last)) {
+                __threadfence();
+                const RowRuns rr = row_runs(c.first, c.n, N, p.P);
+                const size_t row0 = static_cast<size_t>(c.b) * p.Hq + static_cast<size_t>(c.h) * p.g;
+                merge_row<D>(p.seg_out, p.seg_lse, p.g, u, rr, N, p.P, p.out + row0 * D, p.lse + row0, merge, tid,
+                             kConsumerThreads, consumers_sync);
+                if (tid == 0) p.row_tickets[u] = 0;   // every other segment has arrived: reset for the next call
+            }
+        }
+        consumers_sync();
         remaining -= seg;
         if (remaining > 0) next_row(c, p);
+    }
+
+    if (kFused) {
+        // rows without tokens: out = 0, lse = -inf, written by block u % P
+        for (long long u = blockIdx.x; u < static_cast<long long>(p.B) * p.Hkv; u += p.P) {
+            const int b = static_cast<int>(u / p.Hkv), h = static_cast<int>(u % p.Hkv);
+            if (clamp_len(__ldg(p.seqlens + b), p.Lmax) != 0) continue;
+            const size_t row0 = static_cast<size_t>(b) * p.Hq + static_cast<size_t>(h) * p.g;
+            write_empty_row<D>(p.out + row0 * D, p.lse + row0, p.g, tid, kConsumerThreads);
+        }
     }
 }
 

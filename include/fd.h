@@ -16,7 +16,7 @@
  * result by splitting the keys/values along the sequence, computing each
  * split's attention together with one log-sum-exp scalar per row and split,
  * and reducing over the splits with each one rescaled through its
- * log-sum-exp. This library does the same on one GPU in two stages:
+ * log-sum-exp. This library does the same on one GPU:
  *   split   -- every (sequence, kv-head) row's cached tokens are laid end to
  *              end in one stream of 64-token tiles, and the stream is cut into
  *              num_splits equal runs of tiles, one per thread block. A run
@@ -26,16 +26,22 @@
  *   combine -- for each row cut into several segments, the LSE-weighted
  *              reduction of its segments; rows with no tokens get out = 0,
  *              lse = -inf.
- * fd_decode runs both stages; fd_split and fd_combine run one each.
+ * fd_decode runs both in ONE kernel: after writing a segment, a block takes a
+ * ticket on its row (an atomic counter in the workspace; nothing waits), and
+ * the block that completes the row performs its reduction. fd_split and
+ * fd_combine run the two stages as separate kernels (same arithmetic, same
+ * results bit for bit).
  *
  * LAYOUTS (all row-major, contiguous, device memory unless stated)
  *   q        [B, Hq, D]          bf16 bit patterns (uint16_t), 16-byte aligned
  *   k_cache  [B, Hkv, Lmax, D]   bf16, 16-byte aligned
  *   v_cache  [B, Hkv, Lmax, D]   bf16, 16-byte aligned
  *   seqlens  [B]                 int32 (device); values are clamped to [0, Lmax]
- *   out      [B, Hq, D]          fp32, 4-byte aligned
+ *   out      [B, Hq, D]          fp32, 16-byte aligned
  *   lse      [B, Hq]             fp32 natural-log log-sum-exp, 4-byte aligned
- *   workspace                    fd_workspace_bytes() bytes, 16-byte aligned
+ *   workspace                    fd_workspace_bytes() bytes, 16-byte aligned; must be
+ *                                zero before its first use by fd_decode (fd_workspace_init);
+ *                                every completed fd_decode leaves its counters at zero again
  * Supported: D in {64, 128}; 1 <= Hq/Hkv <= 16; positions t >= seqlens[b]
  * are never used (their contents, NaN included, cannot reach the output).
  *
@@ -96,15 +102,20 @@ FD_API int fd_plan_for_sms(int B, int Hq, int Hkv, int D, int max_len, int num_s
 
 /* Workspace bytes that fd_decode / fd_split / fd_combine need for
  * num_splits splits: room for (num_splits + B*Hkv - 1) segments of
- * Hq/Hkv rows, each D fp32 outputs plus one fp32 log-sum-exp, laid out as
- *     seg_out [num_segments][Hq/Hkv][D]  fp32, then (256-byte aligned)
- *     seg_lse [num_segments][Hq/Hkv]     fp32.
+ * Hq/Hkv rows, each D fp32 outputs plus one fp32 log-sum-exp, and one int32
+ * counter per (sequence, kv-head) row, laid out as (each part 256-byte aligned)
+ *     seg_out [num_segments][Hq/Hkv][D]  fp32
+ *     seg_lse [num_segments][Hq/Hkv]     fp32
+ *     tickets [B*Hkv]                    int32 (fd_decode only)
  * Returns 0 when num_splits == 1 (no row is ever cut) or the arguments are
  * invalid. */
 FD_API size_t fd_workspace_bytes(int B, int Hq, int Hkv, int D, int max_len, int num_splits);
 
 /* Decode attention with num_splits = fd_plan(B, Hq, Hkv, D, max_len).
- * Writes out and lse for every (b, i). Enqueues two kernels on `stream`. */
+ * Writes out and lse for every (b, i). Enqueues one kernel on `stream`.
+ * Calls that share a workspace must not overlap on the device. After a call
+ * that failed on the device (fd_device_status != FD_OK) re-zero the
+ * workspace with fd_workspace_init before using it again. */
 FD_API int fd_decode(int B, int Hq, int Hkv, int D, int max_len,
               const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
               const int32_t *seqlens, float scale,
@@ -120,9 +131,10 @@ FD_API int fd_decode_splits(int B, int Hq, int Hkv, int D, int max_len,
                      void *workspace, size_t workspace_bytes,
                      int num_splits, void *stream);
 
-/* Split stage alone: for each run of tiles, writes out/lse of the rows it
- * holds whole and the segments of the rows it holds in part. Rows with no
- * tokens and rows cut into several segments are left for fd_combine. */
+/* Split stage alone (one kernel): for each run of tiles, writes out/lse of
+ * the rows it holds whole and the segments of the rows it holds in part.
+ * Rows with no tokens and rows cut into several segments are left for
+ * fd_combine. Does not use the workspace counters. */
 FD_API int fd_split(int B, int Hq, int Hkv, int D, int max_len,
              const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
              const int32_t *seqlens, float scale,
@@ -130,10 +142,11 @@ FD_API int fd_split(int B, int Hq, int Hkv, int D, int max_len,
              void *workspace, size_t workspace_bytes,
              int num_splits, void *stream);
 
-/* Combine stage alone: reads the segments that fd_split wrote for the same
- * (shape, seqlens, num_splits) and writes out/lse of every row cut into
- * several segments (segment order fixed, so the result is deterministic),
- * and out = 0, lse = -inf for rows with no tokens. */
+/* Combine stage alone (one kernel): reads the segments that fd_split wrote
+ * for the same (shape, seqlens, num_splits) and writes out/lse of every row
+ * cut into several segments (segment order fixed, so the result is
+ * deterministic), and out = 0, lse = -inf for rows with no tokens. Launched
+ * as a programmatic dependent of the preceding kernel on the stream. */
 FD_API int fd_combine(int B, int Hq, int Hkv, int D, int max_len,
                const int32_t *seqlens,
                float *out, float *lse,
@@ -151,6 +164,10 @@ FD_API int fd_combine(int B, int Hq, int Hkv, int D, int max_len,
 FD_API int fd_segments(int B, int Hkv, int max_len, const int32_t *seqlens_host, int num_splits,
                 int32_t *seg_row, int32_t *seg_begin, int32_t *seg_end, int32_t *seg_whole,
                 int capacity);
+
+/* Zero `workspace_bytes` bytes of workspace on `stream` (cudaMemsetAsync).
+ * Needed once after allocation, before the first fd_decode. */
+FD_API int fd_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /* Waits for `stream`, then returns and clears this device's error word:
  * FD_OK, or FD_ERR_TIMEOUT if a kernel's bounded wait gave up (the kernel

@@ -80,8 +80,10 @@ def test_plan_small_and_edge_shapes():
 def test_workspace_bytes_formula():
     for (B, Hq, Hkv, D, S) in [(1, 32, 32, 128, 148), (1, 64, 8, 128, 148), (64, 32, 8, 128, 148),
                                (32, 32, 8, 128, 148), (1, 4, 4, 64, 16), (3, 12, 4, 64, 5)]:
-        slots, g, off = fd.workspace_layout(B, Hq, Hkv, D, S)
-        want = off + (slots * g * 4 + 255) // 256 * 256
+        slots, g, off, tick = fd.workspace_layout(B, Hq, Hkv, D, S)
+        assert off == (slots * g * D * 4 + 255) // 256 * 256
+        assert tick == off + (slots * g * 4 + 255) // 256 * 256
+        want = tick + (B * Hkv * 4 + 255) // 256 * 256
         assert fd.fd_workspace_bytes(B, Hq, Hkv, D, 1000, S) == want
         assert fd.fd_workspace_bytes(B, Hq, Hkv, D, 1000, 1) == 0
     assert fd.fd_workspace_bytes(1, 3, 2, 64, 10, 4) == 0          # invalid shape
@@ -106,12 +108,16 @@ def test_bad_arguments_return_codes_without_a_device():
     assert split(q=None) == -1 and split(k=None) == -1 and split(out=None) == -1 and split(s=None) == -1
     assert split(k=ctypes.c_void_p(a16 + 8)) == -5
     assert split(out=ctypes.c_void_p(a16 + 2)) == -5
+    assert split(out=ctypes.c_void_p(a16 + 4)) == -5      # out needs 16 bytes (vector stores)
+    assert split(lse=ctypes.c_void_p(a16 + 4)) != -5      # lse needs 4
     assert split(S=0) == -7 and split(S=70000) == -7
     assert split(S=4, ws=None) == -6
     assert split(S=4, wsb=16) == -6
     assert split(S=4, ws=ctypes.c_void_p(a16 + 4)) == -5
     assert L.fd_combine(1, 4, 4, 64, 64, None, p, p, p, 4096, 4, None) == -1
     assert L.fd_split(1, 4, 4, 64, 64, p, p, p, p, 0.1, p, p, None, 0, 2, None) == -6
+    assert L.fd_workspace_init(None, 16, None) == -1
+    assert L.fd_workspace_init(None, 0, None) == 0
     # a valid call reaches the device query and fails there on a CPU-only host
     if not os.path.exists("/dev/nvidia0"):
         assert split() == -8
@@ -150,6 +156,7 @@ def segments_rule(B, Hkv, Lmax, seqlens, P):
     (3, 2, 500, [500, 1, 0], 7), (5, 3, 4096, [4096, 64, 65, 4000, 2], 148),
     (4, 8, 65536, [65536, 1, 30000, 12345], 148), (2, 1, 300, [999, -5], 3),
     (6, 2, 256, [0, 0, 256, 0, 130, 0], 11), (1, 1, 64, [64], 300),
+    (3, 2, 5000, [5000, 1234, 3], 400), (2, 3, 640, [640, 300], 61),   # more runs than tiles
 ])
 def test_segments_match_the_documented_partition(case):
     B, Hkv, Lmax, lens, P = case

@@ -172,6 +172,7 @@ def test_guard_bands_untouched():
     S = 37
     nbytes = fd.fd_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, w.Lmax, S)
     ws = torch.full((nbytes + 4096,), 0xA5, dtype=torch.uint8, device="cuda")
+    ws[:nbytes].zero_()                      # the row counters start at zero
     out_buf = torch.full((w.B * w.Hq * w.D + 1024,), 12345.0, device="cuda")
     lse_buf = torch.full((w.B * w.Hq + 1024,), 12345.0, device="cuda")
     out = out_buf[:w.B * w.Hq * w.D].view(w.B, w.Hq, w.D)
@@ -226,7 +227,7 @@ def test_split_stage_segments_against_oracle(g, D, S):
     lse = torch.full((w.B, w.Hq), 777.0, device="cuda")
     fd.fd_split(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S)
     torch.cuda.synchronize()
-    slots, gg, off = fd.workspace_layout(w.B, w.Hq, w.Hkv, w.D, S)
+    slots, gg, off, _ = fd.workspace_layout(w.B, w.Hq, w.Hkv, w.D, S)
     seg_out = ws[:slots * gg * w.D * 4].view(torch.float32).view(slots, gg, w.D).cpu().numpy()
     seg_lse = ws[off:off + slots * gg * 4].view(torch.float32).view(slots, gg).cpu().numpy()
     ref = segment_oracle(x, seg)
@@ -253,7 +254,7 @@ def test_combine_stage_alone_on_oracle_partials(g, D, S):
     w = x.workload
     seg = fd.fd_segments(w.B, w.Hkv, w.Lmax, x.seqlens_host, S)
     ref = segment_oracle(x, seg)
-    slots, gg, off = fd.workspace_layout(w.B, w.Hq, w.Hkv, w.D, S)
+    slots, gg, off, _ = fd.workspace_layout(w.B, w.Hq, w.Hkv, w.D, S)
     so = np.zeros((slots, gg, w.D), np.float32)
     sl = np.zeros((slots, gg), np.float32)
     for s, (o, l) in ref.items():
@@ -284,3 +285,43 @@ def test_combine_stage_alone_on_oracle_partials(g, D, S):
         ro, rl = oracle.combine(po, pl)
         compare(out[b, rows], lse[b, rows], ro, rl, f"combine row {u}", out_tol=1e-5, lse_rel=1e-6)
     assert multi > 0
+
+
+@pytest.mark.parametrize("g,D,S", [(1, 128, 37), (8, 128, 148), (4, 64, 23), (16, 128, 61)])
+def test_fused_equals_two_stages(g, D, S):
+    """fd_decode (split with the reduction fused in) gives bitwise the same
+    out/lse as fd_split followed by fd_combine."""
+    x = mid_case(g, D)
+    w = x.workload
+    nbytes = fd.fd_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, w.Lmax, S)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    o1 = torch.empty((w.B, w.Hq, w.D), device="cuda")
+    l1 = torch.empty((w.B, w.Hq), device="cuda")
+    fd.fd_decode_splits(x.q, x.k, x.v, x.seqlens, x.scale, o1, l1, ws, S)
+    o2 = torch.full_like(o1, 5.0)
+    l2 = torch.full_like(l1, 5.0)
+    ws2 = torch.zeros_like(ws)
+    fd.fd_split(x.q, x.k, x.v, x.seqlens, x.scale, o2, l2, ws2, S)
+    fd.fd_combine(w.B, w.Hq, w.Hkv, w.D, w.Lmax, x.seqlens, o2, l2, ws2, S)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_workspace_reuse_leaves_counters_at_zero():
+    """One workspace across calls with different inputs and lengths: every
+    call is right, and the row counters are back at zero after each."""
+    w = Workload("reuse", B=4, Hq=16, Hkv=4, D=128, Lmax=3000, ragged=False, sigma_k=2.0, nan_pad=True)
+    S = 97
+    nbytes = fd.fd_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, w.Lmax, S)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    fd.fd_workspace_init(ws)
+    _, _, _, tick = fd.workspace_layout(w.B, w.Hq, w.Hkv, w.D, S)
+    out = torch.empty((w.B, w.Hq, w.D), device="cuda")
+    lse = torch.empty((w.B, w.Hq), device="cuda")
+    for seed, lens in ((1, [3000, 17, 0, 2999]), (2, [64, 3000, 1500, 1]), (3, [0, 0, 0, 700])):
+        x = make_inputs(w, seed, device="cuda", seqlens=lens)
+        fd.fd_decode_splits(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S)
+        torch.cuda.synchronize()
+        ref_o, ref_l = oracle_rows(x)
+        compare(out, lse, ref_o, ref_l, f"reuse seed {seed}")
+        assert torch.all(ws[tick:tick + 4 * w.B * w.Hkv] == 0)
