@@ -18,8 +18,9 @@ FD_MAX_GROUP = 16
 ERRORS = {
     -1: "FD_ERR_NULL_POINTER", -2: "FD_ERR_SHAPE", -3: "FD_ERR_GROUP", -4: "FD_ERR_HEAD_DIM",
     -5: "FD_ERR_ALIGNMENT", -6: "FD_ERR_WORKSPACE", -7: "FD_ERR_SPLITS", -8: "FD_ERR_DEVICE",
-    -9: "FD_ERR_LAUNCH", -10: "FD_ERR_TIMEOUT", -11: "FD_ERR_CAPACITY",
+    -9: "FD_ERR_LAUNCH", -10: "FD_ERR_TIMEOUT", -11: "FD_ERR_CAPACITY", -12: "FD_ERR_STATIC_LIMIT",
 }
+FD_STATIC_SCRATCH_BYTES = 8 << 20
 
 
 class FdError(RuntimeError):
@@ -51,11 +52,12 @@ def lib() -> ctypes.CDLL:
         L.fd_segments.argtypes = [_i, _i, _i, _p, _i, _p, _p, _p, _p, _i]
         L.fd_device_status.argtypes = [_p]
         L.fd_workspace_init.argtypes = [_p, _sz, _p]
+        L.fd_decode_static.argtypes = [_i] * 5 + [_p, _p, _p, _p, _f, _p, _p, _p]
         L.fd_strerror.argtypes = [_i]
         L.fd_strerror.restype = ctypes.c_char_p
         L.fd_version.argtypes = []
         for name in ("fd_plan", "fd_plan_for_sms", "fd_decode", "fd_decode_splits", "fd_split", "fd_combine",
-                     "fd_segments", "fd_device_status", "fd_version", "fd_workspace_init"):
+                     "fd_segments", "fd_device_status", "fd_version", "fd_workspace_init", "fd_decode_static"):
             getattr(L, name).restype = _i
         _lib = L
     return _lib
@@ -170,6 +172,17 @@ def fd_segments(B: int, Hkv: int, max_len: int, seqlens_host, num_splits: int) -
     n = _check(lib().fd_segments(B, Hkv, max_len, lens.ctypes.data, int(num_splits),
                                  *(a.ctypes.data for a in arrs), cap), "fd_segments")
     return dict(row=arrs[0][:n], begin=arrs[1][:n], end=arrs[2][:n], whole=arrs[3][:n])
+
+
+def fd_decode_static(q, k_cache, v_cache, seqlens, scale, out, lse, stream=None):
+    """fd_decode without a workspace argument: the library's fixed device
+    scratch buffer is used instead (see include/fd.h)."""
+    B, Hq, Hkv, D, Lmax = _shapes(q, k_cache, v_cache)
+    _outputs(out, lse, B, Hq, D)
+    _seqlens(seqlens, B)
+    _check(lib().fd_decode_static(B, Hq, Hkv, D, Lmax, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                  seqlens.data_ptr(), float(scale), out.data_ptr(), lse.data_ptr(),
+                                  _stream(stream, q.device)), "fd_decode_static")
 
 
 def fd_workspace_init(workspace, stream=None):

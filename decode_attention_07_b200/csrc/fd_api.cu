@@ -339,6 +339,32 @@ Problem make_problem(int B, int Hq, int Hkv, int D, int max_len, const uint16_t 
     return pr;
 }
 
+// ------------------------------------------------- fixed scratch buffer --
+// Workspace of fd_decode_static: one buffer per device, lives as long as the
+// module. Host code must not use the symbol itself as a device address; it
+// asks the runtime for the address once per device (static_scratch below).
+static __device__ __align__(256) unsigned char g_fd_static_scratch[FD_STATIC_SCRATCH_BYTES];
+
+void *g_static_scratch_ptr[kMaxDevices];
+cudaError_t g_static_scratch_err[kMaxDevices];
+std::once_flag g_static_scratch_once[kMaxDevices];
+
+// Device address of this device's fixed scratch buffer (looked up on first use).
+int static_scratch(void **ptr) {
+    int dev;
+    int rc = current_device(&dev);
+    if (rc != FD_OK) return rc;
+    std::call_once(g_static_scratch_once[dev], [dev] {
+        g_static_scratch_err[dev] = cudaGetSymbolAddress(&g_static_scratch_ptr[dev], g_fd_static_scratch);
+    });
+    if (g_static_scratch_err[dev] != cudaSuccess || g_static_scratch_ptr[dev] == nullptr) {
+        cudaGetLastError();
+        return FD_ERR_LAUNCH;
+    }
+    *ptr = g_static_scratch_ptr[dev];
+    return FD_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -455,6 +481,34 @@ int fd_segments(int B, int Hkv, int max_len, const int32_t *seqlens_host, int nu
     return static_cast<int>(slots);
 }
 
+int fd_decode_static(int B, int Hq, int Hkv, int D, int max_len, const uint16_t *q, const uint16_t *k_cache,
+                     const uint16_t *v_cache, const int32_t *seqlens, float scale, float *out, float *lse,
+                     void *stream) {
+    // argument checks first (no CUDA call): validate as an unsplit call, which needs no workspace
+    Problem pr = make_problem(B, Hq, Hkv, D, max_len, q, k_cache, v_cache, seqlens, scale, out, lse, nullptr, 0, 1,
+                              stream);
+    int rc = check_problem(pr, true);
+    if (rc != FD_OK) return rc;
+    const int S = fd_plan(B, Hq, Hkv, D, max_len);
+    if (S < 0) return S;
+    const WorkspaceLayout w = workspace_layout(B, Hq, Hkv, D, S);
+    if (w.total > FD_STATIC_SCRATCH_BYTES) return FD_ERR_STATIC_LIMIT;
+    void *scratch = nullptr;
+    if (w.total > 0) {
+        if ((rc = static_scratch(&scratch)) != FD_OK) return rc;
+        // the per-row counters must start at zero; the segments need no clearing
+        char *tickets = static_cast<char *>(scratch) + w.tickets;
+        if (cudaMemsetAsync(tickets, 0, w.total - w.tickets, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+            cudaGetLastError();
+            return FD_ERR_LAUNCH;
+        }
+    }
+    pr.ws = scratch;
+    pr.ws_bytes = w.total;
+    pr.num_splits = S;
+    return run_split(pr, true);
+}
+
 int fd_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
     if (workspace_bytes == 0) return FD_OK;
     if (!workspace) return FD_ERR_NULL_POINTER;
@@ -498,6 +552,8 @@ const char *fd_strerror(int code) {
         case FD_ERR_LAUNCH: return "kernel launch or tensor-map encoding failed";
         case FD_ERR_TIMEOUT: return "a device-side wait gave up; outputs of that call are invalid";
         case FD_ERR_CAPACITY: return "output arrays too small";
+        case FD_ERR_STATIC_LIMIT:
+            return "problem needs more scratch than fd_decode_static's fixed 8 MiB buffer; use fd_decode with a workspace";
         default: return "unknown error code";
     }
 }

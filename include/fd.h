@@ -82,10 +82,12 @@ extern "C" {
 #define FD_ERR_LAUNCH        -9   /* a kernel launch (or tensor-map encode) failed */
 #define FD_ERR_TIMEOUT      -10   /* a device-side wait gave up (reported by fd_device_status) */
 #define FD_ERR_CAPACITY     -11   /* an output array passed to fd_segments is too small */
+#define FD_ERR_STATIC_LIMIT -12   /* fd_decode_static: the problem needs more scratch than its fixed buffer */
 
 #define FD_TILE_TOKENS     64     /* tokens per tile; split boundaries are multiples of this */
 #define FD_MAX_SPLITS      65535
 #define FD_MAX_GROUP       16
+#define FD_STATIC_SCRATCH_BYTES (8u << 20)   /* fixed device scratch behind fd_decode_static */
 
 /* Number of splits (thread blocks of the split stage) for a problem shape,
  * sized to the current device's SM count: one block per SM while the batch
@@ -164,6 +166,31 @@ FD_API int fd_combine(int B, int Hq, int Hkv, int D, int max_len,
 FD_API int fd_segments(int B, int Hkv, int max_len, const int32_t *seqlens_host, int num_splits,
                 int32_t *seg_row, int32_t *seg_begin, int32_t *seg_end, int32_t *seg_whole,
                 int capacity);
+
+/* fd_decode for callers that cannot allocate device memory. The paper has
+ * no counterpart to this entry point; it exists for code that is handed its
+ * input and output buffers but owns no allocator -- for example a plugin
+ * inside a serving engine that plans every device byte itself and forbids
+ * allocation on its execution path, or a decode loop that must not call
+ * cudaMalloc because cudaMalloc can synchronise the device.
+ * Same inputs, outputs, layouts and result as fd_decode with the planned
+ * split count; there is no workspace argument. Instead the library keeps one
+ * file-scope device buffer of FD_STATIC_SCRATCH_BYTES (8 MiB), which every
+ * GPU that loads the library holds until the process exits. A problem whose
+ * fd_workspace_bytes() exceeds it is rejected with FD_ERR_STATIC_LIMIT
+ * before anything is launched. Nothing is allocated: no cudaMalloc, no
+ * cudaFree, no allocating library call.
+ * The first call on each device looks up the buffer's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture. Every call clears the buffer's per-row counters
+ * (cudaMemsetAsync on `stream`) and then reuses it, so the buffer keeps the
+ * last call's segments. All calls on one device share the one buffer: two
+ * calls that can overlap on the GPU (different streams, no ordering between
+ * them) race on it and give wrong results. */
+FD_API int fd_decode_static(int B, int Hq, int Hkv, int D, int max_len,
+                            const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                            const int32_t *seqlens, float scale,
+                            float *out, float *lse, void *stream);
 
 /* Zero `workspace_bytes` bytes of workspace on `stream` (cudaMemsetAsync).
  * Needed once after allocation, before the first fd_decode. */
