@@ -38,7 +38,6 @@ __global__ void __launch_bounds__(kCombineThreads) fd_combine_kernel(const Combi
         total += __shfl_xor_sync(0xffffffffu, total, s);
     }
     __shared__ long long red[2][kCombineThreads / 32];
-    __shared__ float s_lse[16];
     if (lane == 0) {
         red[0][warp] = before;
         red[1][warp] = total;
@@ -64,8 +63,7 @@ __global__ void __launch_bounds__(kCombineThreads) fd_combine_kernel(const Combi
     const long long first = before * p.Hkv + static_cast<long long>(h) * n_b;
     const RowRuns rr = row_runs(first, n_b, N, p.P);
     if (rr.i0 == rr.i1) return;   // one segment: the split stage wrote this row
-    merge_row<D>(p.seg_out, p.seg_lse, p.g, u, rr, N, p.P, p.out + row0 * D, p.lse + row0, s_lse, tid,
-                 kCombineThreads, [] { __syncthreads(); });
+    merge_row<D>(p.seg_out, p.seg_lse, p.g, u, rr, N, p.P, p.out + row0 * D, p.lse + row0, tid, kCombineThreads);
 }
 
 }  // namespace fd

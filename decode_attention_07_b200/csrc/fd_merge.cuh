@@ -39,55 +39,79 @@ __device__ __forceinline__ RowRuns row_runs(long long first, int n, long long N,
     return r;
 }
 
-// Merge row u's segments into out_row[g][D] / lse_row[g]. Called by `nthreads`
-// threads (tid = 0..nthreads-1, whole warps) that share `s_lse` (>= g floats
-// of shared memory) and the barrier `bar`. Reads go to L2 (.cg): the segments
-// were written by other blocks of the same grid.
-template <int D, class Bar>
-__device__ __forceinline__ void merge_row(const float *seg_out, const float *seg_lse, int g, long long u,
-                                          const RowRuns &rr, long long N, int P, float *out_row, float *lse_row,
-                                          float *s_lse, int tid, int nthreads, Bar bar) {
-    const int lane = tid & 31, warp = tid >> 5, nwarps = nthreads >> 5;
-    const int nseg = rr.i1 - rr.i0 + 1;
-    const size_t slot0 = static_cast<size_t>(rr.i0) + static_cast<size_t>(u);
+// One float4 of the merged output of a row: head `head`, columns 4*d4..4*d4+3.
+// Walks the segments once, in slot order, with a running maximum
+//     M <- max(M, lse_s);  S = sum exp(lse_s - M);  acc = sum exp(lse_s - M) O_s
+// and returns acc / S (and LSE = M + log S through *lse). Loads are issued
+// eight segments at a time before any of them is used, so a row costs one L2
+// round trip per eight segments. Reads go to L2 (.cg): the segments were
+// written by other blocks of the same grid.
+template <int D>
+__device__ __forceinline__ float4 merge_row_vec(const float *seg_out, const float *seg_lse, int g, size_t slot0,
+                                                int nseg, int i0, long long N, int P, int head, int d4,
+                                                float *lse) {
+    constexpr int kChunk = 8;
     const bool maybe_empty = N < P;
-
-    for (int head = warp; head < g; head += nwarps) {
-        float mx = -INFINITY;
-        for (int s = lane; s < nseg; s += 32)
-            if (!maybe_empty || !run_is_empty(rr.i0 + s, N, P))
-                mx = fmaxf(mx, __ldcg(seg_lse + (slot0 + s) * g + head));
-        for (int sh = 16; sh > 0; sh >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, sh));
-        float sum = 0.f;
-        if (mx != -INFINITY)
-            for (int s = lane; s < nseg; s += 32)
-                if (!maybe_empty || !run_is_empty(rr.i0 + s, N, P))
-                    sum += ex2((__ldcg(seg_lse + (slot0 + s) * g + head) - mx) * kLog2eF);
-        for (int sh = 16; sh > 0; sh >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, sh);
-        if (lane == 0) s_lse[head] = mx == -INFINITY ? -INFINITY : mx + lg2(sum) * kLn2F;
-    }
-    bar();
-
-    constexpr int kVec = D / 4;   // float4 outputs per head
-    for (int idx = tid; idx < g * kVec; idx += nthreads) {
-        const int head = idx / kVec, d4 = idx - head * kVec;
-        const float LSE = s_lse[head];
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (LSE != -INFINITY) {
-#pragma unroll 4
-            for (int s = 0; s < nseg; ++s) {
-                if (maybe_empty && run_is_empty(rr.i0 + s, N, P)) continue;
+    float M = -INFINITY, S = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < nseg; s0 += kChunk) {
+        float ls[kChunk];
+        float4 o[kChunk];
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) {
+            const int s = s0 + j;
+            ls[j] = -INFINITY;
+            o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (s < nseg && !(maybe_empty && run_is_empty(i0 + s, N, P))) {
                 const size_t r = (slot0 + s) * g + head;
-                const float w = ex2((__ldcg(seg_lse + r) - LSE) * kLog2eF);
-                const float4 o = __ldcg(reinterpret_cast<const float4 *>(seg_out + r * D) + d4);
-                acc.x = fmaf(w, o.x, acc.x);
-                acc.y = fmaf(w, o.y, acc.y);
-                acc.z = fmaf(w, o.z, acc.z);
-                acc.w = fmaf(w, o.w, acc.w);
+                ls[j] = __ldcg(seg_lse + r);
+                o[j] = __ldcg(reinterpret_cast<const float4 *>(seg_out + r * D) + d4);
             }
         }
-        reinterpret_cast<float4 *>(out_row + head * D)[d4] = acc;
-        if (d4 == 0) lse_row[head] = LSE;
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) {
+            if (ls[j] == -INFINITY) continue;
+            if (ls[j] > M) {   // new maximum: rescale what has been summed so far
+                const float c = ex2((M - ls[j]) * kLog2eF);
+                S *= c;
+                acc.x *= c;
+                acc.y *= c;
+                acc.z *= c;
+                acc.w *= c;
+                M = ls[j];
+            }
+            const float w = ex2((ls[j] - M) * kLog2eF);
+            S += w;
+            acc.x = fmaf(w, o[j].x, acc.x);
+            acc.y = fmaf(w, o[j].y, acc.y);
+            acc.z = fmaf(w, o[j].z, acc.z);
+            acc.w = fmaf(w, o[j].w, acc.w);
+        }
+    }
+    if (M == -INFINITY) {
+        *lse = -INFINITY;
+        return make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const float inv = 1.f / S;
+    *lse = M + lg2(S) * kLn2F;
+    return make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+}
+
+// Merge row u's segments into out_row[g][D] / lse_row[g] with `nthreads`
+// threads (tid = 0..nthreads-1), one float4 output per thread and step.
+template <int D>
+__device__ __forceinline__ void merge_row(const float *seg_out, const float *seg_lse, int g, long long u,
+                                          const RowRuns &rr, long long N, int P, float *out_row, float *lse_row,
+                                          int tid, int nthreads) {
+    const int nseg = rr.i1 - rr.i0 + 1;
+    const size_t slot0 = static_cast<size_t>(rr.i0) + static_cast<size_t>(u);
+    constexpr int kVec = D / 4;
+    for (int idx = tid; idx < g * kVec; idx += nthreads) {
+        const int head = idx / kVec, d4 = idx - head * kVec;
+        float lse;
+        const float4 v = merge_row_vec<D>(seg_out, seg_lse, g, slot0, nseg, rr.i0, N, P, head, d4, &lse);
+        reinterpret_cast<float4 *>(out_row + head * D)[d4] = v;
+        if (d4 == 0) lse_row[head] = lse;
     }
 }
 

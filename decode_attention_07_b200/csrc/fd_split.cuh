@@ -10,22 +10,28 @@
 // running max / running sum below do. A final reduction rescales the splits
 // by their log-sum-exps (fd_merge.cuh).
 //
-// Block layout (288 threads, one block per SM):
+// Block layout (352 threads, one block per SM):
 //   warp 8      producer: one lane streams K and V tiles (64 tokens x D bf16
 //               each) from HBM into a ring of shared-memory stages with 3-D
-//               TMA loads, 128-byte swizzled, mbarrier completion.
+//               TMA loads, 128-byte swizzled, mbarrier completion; with each
+//               group's first tile of a row segment it also bulk-copies that
+//               row's query heads into the stage.
 //   warps 0..7  consumers in two groups of four. Group q takes the tiles with
 //               sequence number = q (mod 2), so each SM sub-partition runs two
 //               independent chains; warp w of a group owns tokens
 //               [16w, 16w+16) of its tiles. Per tile: logits, online-softmax
 //               update of the running max m and sum l per query head, and
 //               the rescaled accumulation of p * v. At the end of a row
-//               segment the eight warps' (m, l, o) are merged through shared
-//               memory and written out (whole row) or to the workspace.
-//   fused form: after writing a segment, the block takes a ticket on its
-//               row (atomic counter in the workspace, no waiting); the block
-//               that completes the row merges all its segments and resets
-//               the counter. Rows with no tokens are written by block u % P.
+//               segment each warp only copies its (m, l, o) into one of two
+//               shared-memory merge buffers and goes on.
+//   warps 9,10  finishers: merge the eight warps' states of each segment and
+//               store the result (whole row) or the segment (workspace), off
+//               the consumers' path. Fused form: after storing a segment they
+//               take a ticket on its row (atomic counter in the workspace, no
+//               waiting); the block that completes a row queues it, and at
+//               the end of its run all consumer and finisher threads merge
+//               the queued rows' segments and reset their counters. Rows
+//               with no tokens are written by block u % P.
 // Two consumer forms:
 //   * grouped heads (g = Hq/Hkv >= 2): the g query heads that share one kv
 //     head form a small dense contraction, run on tensor cores with
@@ -47,7 +53,13 @@ constexpr int kGroups = 2;                        // consumer groups alternating
 constexpr int kSliceWarps = 4;                    // warps per group (16 tokens each)
 constexpr int kConsumerWarps = kGroups * kSliceWarps;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kSplitThreads = kConsumerThreads + 32;
+constexpr int kProducerWarp = kConsumerWarps;     // warp 8
+constexpr int kFinisherWarps = 2;                 // warps 9, 10
+constexpr int kFinisherThreads = kFinisherWarps * 32;
+constexpr int kSplitThreads = kConsumerThreads + 32 + kFinisherThreads;
+constexpr int kWorkerThreads = kConsumerThreads + kFinisherThreads;   // all but the producer
+constexpr int kPendingMax = 4;                    // rows a block can complete (a run cuts at most 2)
+constexpr int kBarFinishers = 1, kBarWorkers = 2; // named barrier ids
 constexpr int kWarpTokens = 16;                   // tokens of a tile owned by one consumer warp
 constexpr int kBoxBytes = kTileTokens * 128;      // one TMA box: 64 rows x 128 bytes (64 bf16)
 constexpr int kSmemLimit = 232448;                // 227 KiB opt-in shared memory per block
@@ -72,19 +84,21 @@ template <int D, int G>
 struct SplitConfig {
     static constexpr int kBoxes = D / 64;                                  // 128-byte boxes per row
     static constexpr int kTileBytes = kTileTokens * D * 2;                 // one K (or V) tile
+    static constexpr int kQSlotBytes = (G * D * 2 + 1023) / 1024 * 1024;   // query heads of a row
+    static constexpr int kStageBytes = 2 * kTileBytes + kQSlotBytes;       // multiple of 1024 (swizzle)
+    static constexpr int kStages = D == 128 ? 4 : 8;                       // 128 KiB of K/V: measured best
+    static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kWarpFloats = G * D + 2 * G;                      // o, m, l of one warp
-    static constexpr int kMergeBytes = kConsumerWarps * kWarpFloats * 4;
-    static constexpr int kFixedBytes = 1024 + kMergeBytes + 256;           // alignment, merge, barriers
-    static constexpr int kFit = (kSmemLimit - kFixedBytes) / (2 * kTileBytes);
-    static constexpr int kCap = D == 128 ? 4 : 8;                          // 128 KiB of ring: measured best
-    // A multiple of kGroups, so each consumer group owns its own stages: a
-    // stage shared by both groups could be waited on two phases ahead of a
-    // tile still in flight, where a parity wait would pass on the older phase.
-    static constexpr int kStages = ((kFit < kCap ? kFit : kCap) / kGroups) * kGroups;
-    static constexpr int kRingBytes = kStages * 2 * kTileBytes;
-    static constexpr int kSmemBytes = 1024 + kRingBytes + kMergeBytes + 256;
-    static_assert(kStages >= 4, "ring too shallow");
+    static constexpr int kMergeFloats = kConsumerWarps * kWarpFloats;      // one merge buffer
+    static constexpr int kCtrlBytes = 2048;                                // barriers, start info, queue, weights
+    static constexpr int kMergeBufs =
+        1024 + kRingBytes + 2 * kMergeFloats * 4 + kCtrlBytes <= kSmemLimit ? 2 : 1;
+    static constexpr int kSmemBytes = 1024 + kRingBytes + kMergeBufs * kMergeFloats * 4 + kCtrlBytes;
+    // Each consumer group owns whole stages: a stage shared by both groups
+    // could be waited on two phases ahead of a tile still in flight, where a
+    // parity wait would pass on the older phase.
     static_assert(kStages % kGroups == 0, "each consumer group must own whole stages");
+    static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
     static_assert(kSmemBytes <= kSmemLimit, "shared memory over the limit");
 };
 
@@ -93,13 +107,20 @@ struct Cursor {
     long long first;          // flat index of the row's first tile
 };
 
+struct PendingRow {
+    long long first;          // flat index of the row's first tile
+    int b, h, n;              // the row and its tile count
+};
+
 struct StartInfo {
     long long count;          // tiles in this block's run
     long long N;              // tiles in the whole batch
     long long first;          // flat index of the start row's first tile
     int b, h, tile, n;
     int abort;                // set when a bounded wait gave up
-    int last;                 // this block completes the current row (fused form)
+    int last_buf;             // merge buffer holding the run's last segment
+    int npending;             // rows this block completed (fused form)
+    PendingRow pending[kPendingMax];
 };
 
 // Bounded mbarrier wait. Returns false if the block is aborting or the limit
@@ -139,9 +160,11 @@ __device__ __forceinline__ void next_row(Cursor &c, const SplitParams &p) {
 // Warp 0: total tile count and this block's starting row / tile.
 __device__ __forceinline__ void find_start(const SplitParams &p, StartInfo *info) {
     const int lane = threadIdx.x & 31;
+    // the first 32 sequences are read once and kept for the second pass
+    const int n_first = lane < p.B ? row_tiles(p.seqlens, lane, p.Lmax) : 0;
     long long total = 0;
     for (int base = 0; base < p.B; base += 32) {
-        int n = base + lane < p.B ? row_tiles(p.seqlens, base + lane, p.Lmax) : 0;
+        int n = base == 0 ? n_first : (base + lane < p.B ? row_tiles(p.seqlens, base + lane, p.Lmax) : 0);
         for (int s = 16; s > 0; s >>= 1) n += __shfl_xor_sync(0xffffffffu, n, s);
         total += n;
     }
@@ -153,7 +176,7 @@ __device__ __forceinline__ void find_start(const SplitParams &p, StartInfo *info
     if (t1 > t0) {
         long long before = 0;   // Hkv * (tiles of sequences before this chunk)
         for (int base = 0; base < p.B; base += 32) {
-            const int nb = base + lane < p.B ? row_tiles(p.seqlens, base + lane, p.Lmax) : 0;
+            const int nb = base == 0 ? n_first : (base + lane < p.B ? row_tiles(p.seqlens, base + lane, p.Lmax) : 0);
             int incl = nb;
             for (int s = 1; s < 32; s <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, incl, s);
@@ -184,44 +207,59 @@ __device__ __forceinline__ void find_start(const SplitParams &p, StartInfo *info
         info->tile = tile;
         info->n = n;
         info->abort = 0;
-        info->last = 0;
+        info->last_buf = 0;
+        info->npending = 0;
     }
 }
 
 // ------------------------------------------------------------ merge + store --
 // Per-warp partial results in shared memory: o[G][D], then m[G], l[G] (m in
-// base-2 units). All consumer threads merge the eight warps and store.
-template <int D, int G>
-__device__ __forceinline__ void merge_warps_and_store(const float *merge, const SplitParams &p, const Cursor &c,
-                                                      bool whole, size_t slot) {
+// base-2 units). `nthreads` threads (barrier `bar`) merge the eight warps:
+// first one thread per head turns the warps' (m, l) into normalised weights
+// w[head][warp] = 2^(m_w - M) / sum_w' 2^(m_w' - M) l_w' and the log-sum-exp,
+// then every output is sum_w w[head][w] * o_w.
+template <int D, int G, class Bar>
+__device__ __forceinline__ void merge_warps_and_store(const float *merge, float *weights, const SplitParams &p,
+                                                      const Cursor &c, bool whole, size_t slot, int tid,
+                                                      int nthreads, Bar bar) {
     constexpr int kWarpFloats = G * D + 2 * G;
-    const int tid = threadIdx.x;
-    for (int idx = tid; idx < p.g * D; idx += kConsumerThreads) {
-        const int head = idx / D, d = idx - head * D;
+    float *lse_h = weights + G * kConsumerWarps;   // [G] natural-log lse per head
+    for (int head = tid; head < p.g; head += nthreads) {
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge[w * kWarpFloats + G * D + head]);
-        float o = 0.f, lse_nat = -INFINITY;
-        if (M != -INFINITY) {
-            float acc = 0.f, lsum = 0.f;
+        if (M == -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) weights[head * kConsumerWarps + w] = 0.f;
+            lse_h[head] = -INFINITY;
+        } else {
+            float e[kConsumerWarps], lsum = 0.f;
 #pragma unroll
             for (int w = 0; w < kConsumerWarps; ++w) {
-                const float *wb = merge + w * kWarpFloats;
-                const float e = ex2(wb[G * D + head] - M);
-                lsum = fmaf(e, wb[G * D + G + head], lsum);
-                acc = fmaf(e, wb[head * D + d], acc);
+                e[w] = ex2(merge[w * kWarpFloats + G * D + head] - M);
+                lsum = fmaf(e[w], merge[w * kWarpFloats + G * D + G + head], lsum);
             }
-            o = acc / lsum;
-            lse_nat = (M + lg2(lsum)) * kLn2F;
+            const float inv = 1.f / lsum;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) weights[head * kConsumerWarps + w] = e[w] * inv;
+            lse_h[head] = (M + lg2(lsum)) * kLn2F;
         }
+    }
+    bar();
+    for (int idx = tid; idx < p.g * D; idx += nthreads) {
+        const int head = idx / D, d = idx - head * D;
+        float o = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w)
+            o = fmaf(weights[head * kConsumerWarps + w], merge[w * kWarpFloats + head * D + d], o);
         if (whole) {
             const size_t row = static_cast<size_t>(c.b) * p.Hq + static_cast<size_t>(c.h) * p.g + head;
             p.out[row * D + d] = o;
-            if (d == 0) p.lse[row] = lse_nat;
+            if (d == 0) p.lse[row] = lse_h[head];
         } else {
             const size_t row = slot * p.g + head;
             p.seg_out[row * D + d] = o;
-            if (d == 0) p.seg_lse[row] = lse_nat;
+            if (d == 0) p.seg_lse[row] = lse_h[head];
         }
     }
 }
@@ -237,24 +275,30 @@ struct GroupConsumer {
     float m[NT][2], l[NT][2];           // running max (base 2) / partial sum for heads 2c, 2c+1
     float o[NT][MT][4];                 // O^T accumulators
 
-    __device__ __forceinline__ void begin_row(const SplitParams &p, const Cursor &c) {
+    __device__ __forceinline__ void reset() {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            m[nt][0] = m[nt][1] = -INFINITY;
+            l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+        }
+    }
+
+    // Q^T fragments from the stage's copy of the row's g query heads ([g][D] bf16).
+    __device__ __forceinline__ void load_q(const uint8_t *qs, int g) {
         const int lane = threadIdx.x & 31;
         const int r0 = lane >> 2, cc = lane & 3;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int head = nt * 8 + r0;
-            const bool ok = head < p.g;
-            const uint16_t *qrow =
-                p.q + (static_cast<size_t>(c.b) * p.Hq + static_cast<size_t>(c.h) * p.g + (ok ? head : 0)) * D;
+            const bool ok = head < g;
+            const uint32_t *qrow = reinterpret_cast<const uint32_t *>(qs + (ok ? head : 0) * D * 2);
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
-                qf[nt][ks][0] = ok ? __ldg(reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 2 * cc)) : 0u;
-                qf[nt][ks][1] = ok ? __ldg(reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 2 * cc + 8)) : 0u;
+                qf[nt][ks][0] = ok ? qrow[8 * ks + cc] : 0u;
+                qf[nt][ks][1] = ok ? qrow[8 * ks + cc + 4] : 0u;
             }
-            m[nt][0] = m[nt][1] = -INFINITY;
-            l[nt][0] = l[nt][1] = 0.f;
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
         }
     }
 
@@ -393,19 +437,22 @@ struct HeadConsumer {
     float m, l;                                // running max (base 2, warp-uniform) / lane partial sum
     float acc[8];                              // sum of p * v over this lane's tokens, chunk d0..d0+7
 
-    __device__ __forceinline__ void begin_row(const SplitParams &p, const Cursor &c) {
-        const int lane = threadIdx.x & 31;
-        const int d0 = 8 * (lane % LPT);
-        const uint16_t *qrow = p.q + (static_cast<size_t>(c.b) * p.Hq + c.h) * D;
-        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(qrow + d0));
-        qv[0] = bf16lo_to_f32(w.x); qv[1] = bf16hi_to_f32(w.x);
-        qv[2] = bf16lo_to_f32(w.y); qv[3] = bf16hi_to_f32(w.y);
-        qv[4] = bf16lo_to_f32(w.z); qv[5] = bf16hi_to_f32(w.z);
-        qv[6] = bf16lo_to_f32(w.w); qv[7] = bf16hi_to_f32(w.w);
+    __device__ __forceinline__ void reset() {
         m = -INFINITY;
         l = 0.f;
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+    }
+
+    // q[d0 .. d0+7] from the stage's copy of the row's query head ([D] bf16).
+    __device__ __forceinline__ void load_q(const uint8_t *qs, int) {
+        const int lane = threadIdx.x & 31;
+        const int d0 = 8 * (lane % LPT);
+        const uint4 w = *reinterpret_cast<const uint4 *>(qs + d0 * 2);
+        qv[0] = bf16lo_to_f32(w.x); qv[1] = bf16hi_to_f32(w.x);
+        qv[2] = bf16lo_to_f32(w.y); qv[3] = bf16hi_to_f32(w.y);
+        qv[4] = bf16lo_to_f32(w.z); qv[5] = bf16hi_to_f32(w.z);
+        qv[6] = bf16lo_to_f32(w.w); qv[7] = bf16hi_to_f32(w.w);
     }
 
     static __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -518,29 +565,40 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                     const SplitParams p) {
     constexpr int G = Consumer::G;
     using Cfg = SplitConfig<D, G>;
-    constexpr int kWarpFloats = Cfg::kWarpFloats;
     constexpr int kStages = Cfg::kStages;
+    constexpr int kBufs = Cfg::kMergeBufs;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *ring = smem;
-    float *merge = reinterpret_cast<float *>(ring + Cfg::kRingBytes);
-    uint64_t *full = reinterpret_cast<uint64_t *>(merge + kConsumerWarps * kWarpFloats);
+    uint8_t *ring = smem;                                                  // stages: K tile | V tile | q slot
+    float *merge = reinterpret_cast<float *>(ring + Cfg::kRingBytes);      // kBufs x [8 warps][o, m, l]
+    uint64_t *full = reinterpret_cast<uint64_t *>(merge + kBufs * Cfg::kMergeFloats);
     uint64_t *empty = full + kStages;
-    StartInfo *info = reinterpret_cast<StartInfo *>(empty + kStages);
+    uint64_t *mfull = empty + kStages;                                     // merge buffer filled (8 warps)
+    uint64_t *mempty = mfull + kBufs;                                      // merge buffer drained (finishers)
+    StartInfo *info = reinterpret_cast<StartInfo *>(mempty + kBufs);
+    float *weights = reinterpret_cast<float *>(info + 1);                  // [G][8] merge weights, [G] lse
 
     // A grid queued behind this one (the next call, or the standalone
     // combine) may start its prologue now; it waits for this grid's
     // completion before reading anything.
     grid_dependents_launch();
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kSliceWarps);
         }
+        for (int b = 0; b < kBufs; ++b) {
+            mbar_init(&mfull[b], kConsumerWarps);
+            mbar_init(&mempty[b], kFinisherWarps);
+        }
         fence_mbar_init();
+    }
+    if (warp == kProducerWarp && lane == 0) {   // kernel parameters, not inputs: safe before the wait
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
     }
     // Launched as a programmatic dependent of the previous kernel on the
     // stream: everything above overlaps its tail; inputs are read only after it.
@@ -552,30 +610,32 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     Cursor c{info->b, info->h, info->tile, info->n, info->first};
     const long long N = info->N;
     volatile int *abort = &info->abort;
+    const uint32_t q_bytes = static_cast<uint32_t>(p.g) * D * 2;
 
-    if (warp == kConsumerWarps) {
+    if (warp == kProducerWarp) {
         // ---------------------------------------------------- producer --
         if (lane != 0 || remaining <= 0) return;
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
         const uint64_t policy = l2_policy_evict_first();
         uint32_t seq = 0;
         while (remaining > 0) {
             const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
             const int z = c.b * p.Hkv + c.h;
+            const uint16_t *q_row = p.q + (static_cast<size_t>(c.b) * p.Hq + static_cast<size_t>(c.h) * p.g) * D;
             for (int k = 0; k < seg; ++k, ++seq) {
                 const int stage = static_cast<int>(seq % kStages);
                 const uint32_t phase = (seq / kStages) & 1u;
                 if (!wait_bounded(&empty[stage], phase ^ 1u, abort)) return;
-                uint8_t *kt = ring + stage * 2 * Cfg::kTileBytes;
+                uint8_t *kt = ring + stage * Cfg::kStageBytes;
                 uint8_t *vt = kt + Cfg::kTileBytes;
-                mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kTileBytes);
+                const bool with_q = k < kGroups;   // each group's first tile of the segment
+                mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kTileBytes + (with_q ? q_bytes : 0u));
                 const int y = (c.tile + k) * kTileTokens;
 #pragma unroll
                 for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
                     tma_load_3d(kt + bx * kBoxBytes, &tm_k, &full[stage], 64 * bx, y, z, policy);
                     tma_load_3d(vt + bx * kBoxBytes, &tm_v, &full[stage], 64 * bx, y, z, policy);
                 }
+                if (with_q) bulk_load(vt + Cfg::kTileBytes, q_row, q_bytes, &full[stage]);
             }
             remaining -= seg;
             if (remaining > 0) next_row(c, p);
@@ -583,65 +643,136 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         return;
     }
 
-    // -------------------------------------------------------- consumers --
-    const int group = warp / kSliceWarps, slice = warp % kSliceWarps;
-    const int tid = threadIdx.x;
-    auto consumers_sync = [] { named_barrier_sync(1, kConsumerThreads); };
-    Consumer cons;
-    float *wb = merge + warp * kWarpFloats;
-    uint32_t seq = 0;
-    while (remaining > 0) {
-        const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
-        const int L = clamp_len(__ldg(p.seqlens + c.b), p.Lmax);
-        const bool whole = c.tile == 0 && seg == c.n;
-        cons.begin_row(p, c);
-        for (int k = 0; k < seg; ++k, ++seq) {
-            if (static_cast<int>(seq % kGroups) != group) continue;
-            const int stage = static_cast<int>(seq % kStages);
-            const uint32_t phase = (seq / kStages) & 1u;
-            wait_bounded(&full[stage], phase, abort);   // on abort: keep going, outputs are flagged invalid
-            const uint32_t kt = smem_addr(ring + stage * 2 * Cfg::kTileBytes);
-            const int valid = L - ((c.tile + k) * kTileTokens + kWarpTokens * slice);
-            cons.tile(kt, kt + Cfg::kTileBytes, slice, valid, p.scale_log2e);
+    Cursor last_c = c;          // the run's last segment: merged by all workers at the end
+    int last_seg = 0;
+    if (warp < kConsumerWarps) {
+        // ---------------------------------------------------- consumers --
+        const int group = warp / kSliceWarps, slice = warp % kSliceWarps;
+        Consumer cons;
+        uint32_t seq = 0, segctr = 0;
+        while (remaining > 0) {
+            const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
+            const int L = clamp_len(__ldg(p.seqlens + c.b), p.Lmax);
+            cons.reset();
+            for (int k = 0; k < seg; ++k, ++seq) {
+                if (static_cast<int>(seq % kGroups) != group) continue;
+                const int stage = static_cast<int>(seq % kStages);
+                const uint32_t phase = (seq / kStages) & 1u;
+                wait_bounded(&full[stage], phase, abort);   // on abort: keep going, outputs are flagged invalid
+                const uint8_t *st = ring + stage * Cfg::kStageBytes;
+                if (k < kGroups) cons.load_q(st + 2 * Cfg::kTileBytes, p.g);
+                const uint32_t kt = smem_addr(st);
+                const int valid = L - ((c.tile + k) * kTileTokens + kWarpTokens * slice);
+                cons.tile(kt, kt + Cfg::kTileBytes, slice, valid, p.scale_log2e);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
+            }
+            // hand this segment's state to the finishers and go on
+            const int buf = static_cast<int>(segctr % kBufs);
+            wait_bounded(&mempty[buf], ((segctr / kBufs) & 1u) ^ 1u, abort);
+            cons.to_smem(merge + buf * Cfg::kMergeFloats + warp * Cfg::kWarpFloats);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (lane == 0) mbar_arrive(&mfull[buf]);
+            if (tid == 0) info->last_buf = buf;
+            ++segctr;
+            last_c = c;
+            last_seg = seg;
+            remaining -= seg;
+            if (remaining > 0) next_row(c, p);
         }
-        cons.to_smem(wb);
-        consumers_sync();
-        const long long u = static_cast<long long>(c.b) * p.Hkv + c.h;
-        const size_t slot = static_cast<size_t>(blockIdx.x) + static_cast<size_t>(u);
-        merge_warps_and_store<D, G>(merge, p, c, whole, slot);
-        if (kFused && !whole) {
-            // ticket on the row; the block that completes it merges all segments
-            __threadfence();
-            consumers_sync();
-            if (tid == 0) {
-                const RowRuns rr = row_runs(c.first, c.n, N, p.P);
-                const int prev = atomicAdd(p.row_tickets + u, 1);
-                info->last = prev == rr.count - 1;
+    } else {
+        // ---------------------------------------------------- finishers --
+        const int ftid = tid - (kProducerWarp + 1) * 32;
+        uint32_t segctr = 0;
+        while (remaining > 0) {
+            const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
+            if (seg == remaining) {   // the last segment: left for all workers at the end
+                last_c = c;
+                last_seg = seg;
+                break;
             }
-            consumers_sync();
-            if (*reinterpret_cast<volatile int *>(&info->last)) {
+            const bool whole = c.tile == 0 && seg == c.n;
+            const long long u = static_cast<long long>(c.b) * p.Hkv + c.h;
+            const size_t slot = static_cast<size_t>(blockIdx.x) + static_cast<size_t>(u);
+            const int buf = static_cast<int>(segctr % kBufs);
+            wait_bounded(&mfull[buf], (segctr / kBufs) & 1u, abort);
+            merge_warps_and_store<D, G>(merge + buf * Cfg::kMergeFloats, weights, p, c, whole, slot, ftid,
+                                        kFinisherThreads, [] { named_barrier_sync(kBarFinishers, kFinisherThreads); });
+            named_barrier_sync(kBarFinishers, kFinisherThreads);   // every finisher is done with the buffer
+            if (lane == 0) mbar_arrive(&mempty[buf]);
+            if (kFused && !whole) {
+                // ticket on the row; the block that completes it merges the row later
                 __threadfence();
-                const RowRuns rr = row_runs(c.first, c.n, N, p.P);
-                const size_t row0 = static_cast<size_t>(c.b) * p.Hq + static_cast<size_t>(c.h) * p.g;
-                merge_row<D>(p.seg_out, p.seg_lse, p.g, u, rr, N, p.P, p.out + row0 * D, p.lse + row0, merge, tid,
-                             kConsumerThreads, consumers_sync);
-                if (tid == 0) p.row_tickets[u] = 0;   // every other segment has arrived: reset for the next call
+                named_barrier_sync(kBarFinishers, kFinisherThreads);
+                if (ftid == 0) {
+                    const RowRuns rr = row_runs(c.first, c.n, N, p.P);
+                    const int prev = atomicAdd(p.row_tickets + u, 1);
+                    if (prev == rr.count - 1 && info->npending < kPendingMax)
+                        info->pending[info->npending++] = PendingRow{c.first, c.b, c.h, c.n};
+                    __threadfence();   // acquire: the row's other segments are read after this
+                }
             }
+            ++segctr;
+            remaining -= seg;
+            if (remaining > 0) next_row(c, p);
         }
-        consumers_sync();
-        remaining -= seg;
-        if (remaining > 0) next_row(c, p);
     }
 
+    // ------------------------------------------ end of the run (all but the producer) --
+    // The consumers have dumped the last segment; the finishers have stored
+    // every earlier one. All 320 threads merge and store the last segment.
+    const int wtid = tid < kConsumerThreads ? tid : tid - 32;   // skip the producer warp
+    auto workers_sync = [] { named_barrier_sync(kBarWorkers, kWorkerThreads); };
+    workers_sync();
+    if (info->count > 0) {
+        const bool whole = last_c.tile == 0 && last_seg == last_c.n;
+        const long long u = static_cast<long long>(last_c.b) * p.Hkv + last_c.h;
+        const size_t slot = static_cast<size_t>(blockIdx.x) + static_cast<size_t>(u);
+        const int buf = static_cast<int>(info->last_buf);
+        merge_warps_and_store<D, G>(merge + buf * Cfg::kMergeFloats, weights, p, last_c, whole, slot, wtid,
+                                    kWorkerThreads, workers_sync);
+        if (kFused && !whole) {
+            // ticket on the row: the writes above happen before the fence by
+            // the block barrier; the fence orders them before the atomic
+            workers_sync();
+            if (wtid == 0) {
+                __threadfence();
+                const RowRuns rr = row_runs(last_c.first, last_c.n, N, p.P);
+                const int prev = atomicAdd(p.row_tickets + u, 1);
+                if (prev == rr.count - 1 && info->npending < kPendingMax)
+                    info->pending[info->npending++] = PendingRow{last_c.first, last_c.b, last_c.h, last_c.n};
+                __threadfence();
+            }
+        }
+        workers_sync();
+    }
     if (kFused) {
+        // all queued rows at once: one float4 output per thread and step
+        const int npending = *reinterpret_cast<volatile int *>(&info->npending);
+        constexpr int kVec = D / 4;
+        for (int idx = wtid; idx < npending * p.g * kVec; idx += kWorkerThreads) {
+            const int i = idx / (p.g * kVec), rem = idx - i * p.g * kVec;
+            const int head = rem / kVec, d4 = rem - head * kVec;
+            const PendingRow r = info->pending[i];
+            const long long u = static_cast<long long>(r.b) * p.Hkv + r.h;
+            const RowRuns rr = row_runs(r.first, r.n, N, p.P);
+            const size_t row0 = static_cast<size_t>(r.b) * p.Hq + static_cast<size_t>(r.h) * p.g;
+            float lse;
+            const float4 v = merge_row_vec<D>(p.seg_out, p.seg_lse, p.g, static_cast<size_t>(rr.i0) + u,
+                                              rr.i1 - rr.i0 + 1, rr.i0, N, p.P, head, d4, &lse);
+            reinterpret_cast<float4 *>(p.out + (row0 + head) * D)[d4] = v;
+            if (d4 == 0) p.lse[row0 + head] = lse;
+        }
+        if (wtid < npending) {   // every segment of that row has arrived: reset for the next call
+            const PendingRow r = info->pending[wtid];
+            p.row_tickets[static_cast<long long>(r.b) * p.Hkv + r.h] = 0;
+        }
         // rows without tokens: out = 0, lse = -inf, written by block u % P
         for (long long u = blockIdx.x; u < static_cast<long long>(p.B) * p.Hkv; u += p.P) {
             const int b = static_cast<int>(u / p.Hkv), h = static_cast<int>(u % p.Hkv);
             if (clamp_len(__ldg(p.seqlens + b), p.Lmax) != 0) continue;
             const size_t row0 = static_cast<size_t>(b) * p.Hq + static_cast<size_t>(h) * p.g;
-            write_empty_row<D>(p.out + row0 * D, p.lse + row0, p.g, tid, kConsumerThreads);
+            write_empty_row<D>(p.out + row0 * D, p.lse + row0, p.g, wtid, kWorkerThreads);
         }
     }
 }
