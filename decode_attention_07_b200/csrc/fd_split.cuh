@@ -60,6 +60,7 @@ constexpr int kSplitThreads = kConsumerThreads + 32 + kFinisherThreads;
 constexpr int kWorkerThreads = kConsumerThreads + kFinisherThreads;   // all but the producer
 constexpr int kPendingMax = 4;                    // rows a block can complete (a run cuts at most 2)
 constexpr int kBarFinishers = 1, kBarWorkers = 2; // named barrier ids
+constexpr int kPrefetchTiles = 8;                 // tiles guessed into L2 before the dependency wait
 constexpr int kWarpTokens = 16;                   // tokens of a tile owned by one consumer warp
 constexpr int kBoxBytes = kTileTokens * 128;      // one TMA box: 64 rows x 128 bytes (64 bf16)
 constexpr int kSmemLimit = 232448;                // 227 KiB opt-in shared memory per block
@@ -144,6 +145,17 @@ __device__ __forceinline__ int row_tiles(const int32_t *seqlens, int b, int Lmax
     return tiles_of(clamp_len(__ldg(seqlens + b), Lmax));
 }
 
+// L2-only read (no L1 line kept): for a guess made before the previous grid
+// has finished, which must not leave a stale copy behind for the real read.
+__device__ __forceinline__ int row_tiles_l2(const int32_t *seqlens, int b, int Lmax) {
+    return tiles_of(clamp_len(__ldcg(seqlens + b), Lmax));
+}
+
+template <bool kL2Only>
+__device__ __forceinline__ int tiles_at(const int32_t *seqlens, int b, int Lmax) {
+    return kL2Only ? row_tiles_l2(seqlens, b, Lmax) : row_tiles(seqlens, b, Lmax);
+}
+
 // Next row with at least one tile (only called while tiles remain).
 __device__ __forceinline__ void next_row(Cursor &c, const SplitParams &p) {
     c.first += c.n;
@@ -158,13 +170,14 @@ __device__ __forceinline__ void next_row(Cursor &c, const SplitParams &p) {
 }
 
 // Warp 0: total tile count and this block's starting row / tile.
+template <bool kGuess>
 __device__ __forceinline__ void find_start(const SplitParams &p, StartInfo *info) {
     const int lane = threadIdx.x & 31;
     // the first 32 sequences are read once and kept for the second pass
-    const int n_first = lane < p.B ? row_tiles(p.seqlens, lane, p.Lmax) : 0;
+    const int n_first = lane < p.B ? tiles_at<kGuess>(p.seqlens, lane, p.Lmax) : 0;
     long long total = 0;
     for (int base = 0; base < p.B; base += 32) {
-        int n = base == 0 ? n_first : (base + lane < p.B ? row_tiles(p.seqlens, base + lane, p.Lmax) : 0);
+        int n = base == 0 ? n_first : (base + lane < p.B ? tiles_at<kGuess>(p.seqlens, base + lane, p.Lmax) : 0);
         for (int s = 16; s > 0; s >>= 1) n += __shfl_xor_sync(0xffffffffu, n, s);
         total += n;
     }
@@ -176,7 +189,7 @@ __device__ __forceinline__ void find_start(const SplitParams &p, StartInfo *info
     if (t1 > t0) {
         long long before = 0;   // Hkv * (tiles of sequences before this chunk)
         for (int base = 0; base < p.B; base += 32) {
-            const int nb = base == 0 ? n_first : (base + lane < p.B ? row_tiles(p.seqlens, base + lane, p.Lmax) : 0);
+            const int nb = base == 0 ? n_first : (base + lane < p.B ? tiles_at<kGuess>(p.seqlens, base + lane, p.Lmax) : 0);
             int incl = nb;
             for (int s = 1; s < 32; s <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, incl, s);
@@ -600,10 +613,28 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
     }
+    // While the previous grid drains (HBM mostly idle), guess this block's
+    // first tiles from seqlens as read now and pull them into L2. L2 is the
+    // point of coherence, so a stale guess only wastes bandwidth; everything
+    // below is recomputed from the real inputs after the wait.
+    if (warp == 0) {
+        find_start<true>(p, info);
+        __syncwarp();
+        if (lane < 2 * kPrefetchTiles && info->count > 0) {
+            const int t = lane >> 1;
+            const int tile = info->tile + t;
+            if (t < info->count && tile < info->n) {
+                const CUtensorMap *map = (lane & 1) ? &tm_v : &tm_k;
+                const int z = info->b * p.Hkv + info->h;
+                for (int bx = 0; bx < D / 64; ++bx) tma_prefetch_l2_3d(map, 64 * bx, tile * kTileTokens, z);
+            }
+        }
+        __syncwarp();
+    }
     // Launched as a programmatic dependent of the previous kernel on the
     // stream: everything above overlaps its tail; inputs are read only after it.
     grid_dependency_wait();
-    if (warp == 0) find_start(p, info);
+    if (warp == 0) find_start<false>(p, info);
     __syncthreads();
 
     long long remaining = info->count;
