@@ -269,7 +269,17 @@ def run_fd(args, w, rank, world):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if n_copies == 1 else None
     counts = byte_counts(w, xs[0].seqlens_host, S)
     kv_bytes = sum(x.kv_bytes() for x in xs) / n_copies
-    calls = [fd.prepare_decode(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream) for x in xs]
+    if args.paged:
+        # the same logical caches, scattered into shuffled page pools
+        from decode_attention_07_b200.inputs import make_paged
+        pgs = [make_paged(x, args.paged, args.layout, seed=7 + i) for i, x in enumerate(xs)]
+        for x in xs:   # the contiguous copies are not used by the paged calls
+            x.k = x.v = None
+        torch.cuda.empty_cache()
+        calls = [fd.prepare_decode_paged(x.q, pg.k_pages, pg.v_pages, pg.block_table, x.seqlens, x.scale, out, lse,
+                                         ws, args.layout, S, stream) for x, pg in zip(xs, pgs)]
+    else:
+        calls = [fd.prepare_decode(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream) for x in xs]
 
     def barrier():
         if world > 1:
@@ -316,8 +326,8 @@ def run_fd(args, w, rank, world):
 
     # ---- the two stages as separate kernels (for the per-stage split) ------
     ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-             torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
+             torch.cuda.Event(enable_timing=True)) for _ in range(args.steps if not args.paged else 0)]
+    for i in range(len(ev_s)):
         x = xs[i % n_copies]
         if flush is not None:
             flush.fill_(i & 255)
@@ -327,12 +337,12 @@ def run_fd(args, w, rank, world):
         fd.fd_combine(w.B, w.Hq, w.Hkv, w.D, w.Lmax, x.seqlens, out, lse, ws, S, stream)
         ev_s[i][2].record(stream)
     torch.cuda.synchronize(dev)
-    split_us = 1e3 * sum(a.elapsed_time(b) for a, b, _ in ev_s) / args.steps
-    combine_us = 1e3 * sum(b.elapsed_time(c) for _, b, c in ev_s) / args.steps
+    split_us = 1e3 * sum(a.elapsed_time(b) for a, b, _ in ev_s) / max(1, len(ev_s)) if ev_s else None
+    combine_us = 1e3 * sum(b.elapsed_time(c) for _, b, c in ev_s) / max(1, len(ev_s)) if ev_s else None
 
     # ---- end to end: host buffers in, host buffers out ---------------------
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.paged:
         x = xs[0]
         hq, hk, hv = x.q.cpu().pin_memory(), x.k.cpu().pin_memory(), x.v.cpu().pin_memory()
         hs = x.seqlens.cpu().pin_memory()
@@ -378,13 +388,14 @@ def run_fd(args, w, rank, world):
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_max / args.steps, "us_per_call": us_per_call,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_dict(w, S, l2_note),
+        "config": dict(config_dict(w, S, l2_note), **({"paged": {"page_size": args.paged, "layout": args.layout}}
+                                                      if args.paged else {})),
         "pct_of_nominal_hbm": 100.0 * gbs / world / NOMINAL_HBM_GBS,
         "pct_of_measured_copy": 100.0 * gbs / world / peak,
         "call_bytes_gbs": world * counts["total"] * args.steps / (ms_max * 1e-3) / 1e9,
         "roofline": {"kernel": "fd_split_kernel (fused combine)", "bound": "hbm", "achieved": kernel_gbs,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": kernel_gbs / peak,
-                     "traffic": measured_traffic(w.name), "bytes_per_launch": counts["total"],
+                     "traffic": None if args.paged else measured_traffic(w.name), "bytes_per_launch": counts["total"],
                      "us_per_launch": us_per_call,
                      "frac_of_nominal_8tbs": kernel_gbs / NOMINAL_HBM_GBS},
         "stages_alone": {"split_us": split_us, "combine_us": combine_us},
@@ -393,7 +404,7 @@ def run_fd(args, w, rank, world):
         "e2e": e2e,
         "wall_s": wall,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not args.paged:
         b, s, t, desc = oracle_sample(xs[0], budget_s=args.cpu_seconds)
         line["cpu_baseline"] = {"value": b / s / 1e9, "unit": "GB/s", "cores": t, "kind": "oracle",
                                 "sample": desc, "seconds": s}
@@ -412,6 +423,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--paged", type=int, default=0, metavar="PAGE_SIZE",
+                    help="read the caches from a shuffled page pool with this page size (fd_decode_paged)")
+    ap.add_argument("--layout", choices=["HND", "NHD"], default="HND", help="page layout for --paged")
     ap.add_argument("--no-clock-window", action="store_true",
                     help="do not extend clock sampling past the timed region (for profiler runs)")
     args = ap.parse_args()

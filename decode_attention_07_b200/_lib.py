@@ -21,6 +21,8 @@ ERRORS = {
     -9: "FD_ERR_LAUNCH", -10: "FD_ERR_TIMEOUT", -11: "FD_ERR_CAPACITY", -12: "FD_ERR_STATIC_LIMIT",
 }
 FD_STATIC_SCRATCH_BYTES = 8 << 20
+FD_KV_HND, FD_KV_NHD = 0, 1
+LAYOUTS = {"HND": FD_KV_HND, "NHD": FD_KV_NHD}
 
 
 class FdError(RuntimeError):
@@ -53,11 +55,13 @@ def lib() -> ctypes.CDLL:
         L.fd_device_status.argtypes = [_p]
         L.fd_workspace_init.argtypes = [_p, _sz, _p]
         L.fd_decode_static.argtypes = [_i] * 5 + [_p, _p, _p, _p, _f, _p, _p, _p]
+        L.fd_decode_paged.argtypes = [_i] * 8 + [_p, _p, _p, _p, _p, _f, _p, _p, _p, _sz, _i, _p]
         L.fd_strerror.argtypes = [_i]
         L.fd_strerror.restype = ctypes.c_char_p
         L.fd_version.argtypes = []
         for name in ("fd_plan", "fd_plan_for_sms", "fd_decode", "fd_decode_splits", "fd_split", "fd_combine",
-                     "fd_segments", "fd_device_status", "fd_version", "fd_workspace_init", "fd_decode_static"):
+                     "fd_segments", "fd_device_status", "fd_version", "fd_workspace_init", "fd_decode_static",
+                     "fd_decode_paged"):
             getattr(L, name).restype = _i
         _lib = L
     return _lib
@@ -183,6 +187,72 @@ def fd_decode_static(q, k_cache, v_cache, seqlens, scale, out, lse, stream=None)
     _check(lib().fd_decode_static(B, Hq, Hkv, D, Lmax, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
                                   seqlens.data_ptr(), float(scale), out.data_ptr(), lse.data_ptr(),
                                   _stream(stream, q.device)), "fd_decode_static")
+
+
+def _paged_shapes(q, k_pages, v_pages, block_table, layout):
+    if layout not in LAYOUTS:
+        raise ValueError("layout must be 'HND' ([pages, Hkv, page_size, D]) or 'NHD' ([pages, page_size, Hkv, D])")
+    if q.dim() != 3 or k_pages.dim() != 4 or v_pages.shape != k_pages.shape or block_table.dim() != 2:
+        raise ValueError("expected q [B,Hq,D], k_pages/v_pages 4-D, block_table [B, max_pages]")
+    B, Hq, D = q.shape
+    if layout == "HND":
+        num_pages, Hkv, page_size, D2 = k_pages.shape
+    else:
+        num_pages, page_size, Hkv, D2 = k_pages.shape
+    if D2 != D or block_table.shape[0] != B:
+        raise ValueError("q, pages and block_table disagree on B or D")
+    for t, name in ((q, "q"), (k_pages, "k_pages"), (v_pages, "v_pages")):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if block_table.dtype != torch.int32 or not block_table.is_cuda or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous int32 CUDA tensor")
+    return B, Hq, Hkv, D, page_size, num_pages, block_table.shape[1]
+
+
+def fd_decode_paged(q, k_pages, v_pages, block_table, seqlens, scale, out, lse, workspace=None, layout="HND",
+                    num_splits=0, stream=None):
+    B, Hq, Hkv, D, page_size, num_pages, max_pages = _paged_shapes(q, k_pages, v_pages, block_table, layout)
+    _outputs(out, lse, B, Hq, D)
+    _seqlens(seqlens, B)
+    wp, wb = _ws(workspace)
+    _check(lib().fd_decode_paged(B, Hq, Hkv, D, page_size, num_pages, max_pages, LAYOUTS[layout], q.data_ptr(),
+                                 k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(), seqlens.data_ptr(),
+                                 float(scale), out.data_ptr(), lse.data_ptr(), wp, wb, int(num_splits),
+                                 _stream(stream, q.device)), "fd_decode_paged")
+
+
+def prepare_decode_paged(q, k_pages, v_pages, block_table, seqlens, scale, out, lse, workspace=None, layout="HND",
+                         num_splits=0, stream=None):
+    """Check and marshal once; return a no-argument callable that enqueues
+    fd_decode_paged with those pointers."""
+    B, Hq, Hkv, D, page_size, num_pages, max_pages = _paged_shapes(q, k_pages, v_pages, block_table, layout)
+    _outputs(out, lse, B, Hq, D)
+    _seqlens(seqlens, B)
+    wp, wb = _ws(workspace)
+    fn = lib().fd_decode_paged
+    args = (B, Hq, Hkv, D, page_size, num_pages, max_pages, LAYOUTS[layout], q.data_ptr(), k_pages.data_ptr(),
+            v_pages.data_ptr(), block_table.data_ptr(), seqlens.data_ptr(), ctypes.c_float(scale), out.data_ptr(),
+            lse.data_ptr(), wp, wb, int(num_splits), _stream(stream, q.device))
+
+    def call():
+        rc = fn(*args)
+        if rc != 0:
+            raise FdError(rc, "fd_decode_paged")
+
+    return call
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale, layout="HND", num_splits=None, stream=None):
+    """Allocate out / lse / workspace with torch and run fd_decode_paged."""
+    B, Hq, Hkv, D, page_size, num_pages, max_pages = _paged_shapes(q, k_pages, v_pages, block_table, layout)
+    Lmax = max_pages * page_size
+    S = fd_plan(B, Hq, Hkv, D, Lmax) if num_splits is None else int(num_splits)
+    nbytes = fd_workspace_bytes(B, Hq, Hkv, D, Lmax, S)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    fd_decode_paged(q, k_pages, v_pages, block_table, seqlens, scale, out, lse, ws, layout, S, stream)
+    return out, lse
 
 
 def fd_workspace_init(workspace, stream=None):

@@ -139,11 +139,51 @@ int encode_cache_map(CUtensorMap *map, const void *base, int D, int Lmax, long l
     return r == CUDA_SUCCESS ? FD_OK : FD_ERR_LAUNCH;
 }
 
+// Paged K or V pool as a 4-D tensor, head-dim innermost; the other three dims
+// in increasing-stride order. Head-major pages [num_pages][Hkv][page_size][D]:
+// {D, page_size, Hkv, num_pages}, box {64, rows, 1, 1}. Token-major pages
+// [num_pages][page_size][Hkv][D]: {D, Hkv, page_size, num_pages}, box
+// {64, 1, rows, 1}. rows = min(page_size, 64); 128-byte swizzle as above.
+int encode_paged_map(CUtensorMap *map, const void *base, int D, int page_size, int Hkv, long long num_pages,
+                     bool nhd) {
+    auto fn = encode_fn();
+    if (!fn) return FD_ERR_LAUNCH;
+    const cuuint64_t e = 2;   // bf16
+    const cuuint32_t rows = static_cast<cuuint32_t>(page_size < fd::kTileTokens ? page_size : fd::kTileTokens);
+    cuuint64_t dims[4], strides[3];
+    cuuint32_t box[4];
+    dims[0] = static_cast<cuuint64_t>(D);
+    dims[3] = static_cast<cuuint64_t>(num_pages);
+    box[0] = 64;
+    box[3] = 1;
+    if (nhd) {
+        dims[1] = static_cast<cuuint64_t>(Hkv);
+        dims[2] = static_cast<cuuint64_t>(page_size);
+        strides[0] = D * e;
+        strides[1] = static_cast<cuuint64_t>(Hkv) * D * e;
+        box[1] = 1;
+        box[2] = rows;
+    } else {
+        dims[1] = static_cast<cuuint64_t>(page_size);
+        dims[2] = static_cast<cuuint64_t>(Hkv);
+        strides[0] = D * e;
+        strides[1] = static_cast<cuuint64_t>(page_size) * D * e;
+        box[1] = rows;
+        box[2] = 1;
+    }
+    strides[2] = static_cast<cuuint64_t>(page_size) * Hkv * D * e;
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FD_OK : FD_ERR_LAUNCH;
+}
+
 // ---------------------------------------------------------------- launches --
-template <int D, class Consumer, bool kFused>
+template <int D, class Consumer, bool kFused, bool kPaged>
 int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p, cudaStream_t st) {
     constexpr int smem = fd::SplitConfig<D, Consumer::G>::kSmemBytes;
-    auto kern = fd::fd_split_kernel<D, Consumer, kFused>;
+    auto kern = fd::fd_split_kernel<D, Consumer, kFused, kPaged>;
     // the attribute is per function and device; set it once per device
     static std::once_flag once[kMaxDevices];
     static cudaError_t attr_err[kMaxDevices];
@@ -179,17 +219,17 @@ int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::Split
     return FD_OK;
 }
 
-template <bool kFused>
+template <bool kFused, bool kPaged = false>
 int launch_split(int D, int g, const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p,
                  cudaStream_t st) {
     if (D == 128) {
-        if (g == 1) return launch_split_t<128, fd::HeadConsumer<128>, kFused>(tk, tv, p, st);
-        if (g <= 8) return launch_split_t<128, fd::GroupConsumer<128, 1>, kFused>(tk, tv, p, st);
-        return launch_split_t<128, fd::GroupConsumer<128, 2>, kFused>(tk, tv, p, st);
+        if (g == 1) return launch_split_t<128, fd::HeadConsumer<128>, kFused, kPaged>(tk, tv, p, st);
+        if (g <= 8) return launch_split_t<128, fd::GroupConsumer<128, 1>, kFused, kPaged>(tk, tv, p, st);
+        return launch_split_t<128, fd::GroupConsumer<128, 2>, kFused, kPaged>(tk, tv, p, st);
     }
-    if (g == 1) return launch_split_t<64, fd::HeadConsumer<64>, kFused>(tk, tv, p, st);
-    if (g <= 8) return launch_split_t<64, fd::GroupConsumer<64, 1>, kFused>(tk, tv, p, st);
-    return launch_split_t<64, fd::GroupConsumer<64, 2>, kFused>(tk, tv, p, st);
+    if (g == 1) return launch_split_t<64, fd::HeadConsumer<64>, kFused, kPaged>(tk, tv, p, st);
+    if (g <= 8) return launch_split_t<64, fd::GroupConsumer<64, 1>, kFused, kPaged>(tk, tv, p, st);
+    return launch_split_t<64, fd::GroupConsumer<64, 2>, kFused, kPaged>(tk, tv, p, st);
 }
 
 int launch_combine(int D, const fd::CombineParams &p, cudaStream_t st, bool after_split) {
@@ -288,10 +328,48 @@ int run_split(const Problem &pr, bool fused) {
     p.Lmax = pr.max_len;
     p.P = pr.num_splits;
     p.scale_log2e = pr.scale * kLog2e;
+    p.block_table = nullptr;
+    p.max_pages = 0;
+    p.page_shift = 0;
+    p.kv_nhd = 0;
     // with max_len == 0 every block finds zero tiles and only writes empty rows;
     // the (unused) tensor maps stay zeroed
     return fused ? launch_split<true>(pr.D, p.g, tk, tv, p, pr.stream)
                  : launch_split<false>(pr.D, p.g, tk, tv, p, pr.stream);
+}
+
+struct PagedLayout {
+    const int32_t *block_table;
+    int page_size, num_pages, max_pages;
+    bool nhd;
+};
+
+int run_split_paged(const Problem &pr, const PagedLayout &pl) {
+    int sms;
+    int rc = device_sms(&sms);
+    if (rc != FD_OK) return rc;
+    CUtensorMap tk, tv;
+    if ((rc = encode_paged_map(&tk, pr.k, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
+    if ((rc = encode_paged_map(&tv, pr.v, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
+    fd::SplitParams p;
+    p.q = pr.q;
+    p.seqlens = pr.seqlens;
+    p.out = pr.out;
+    p.lse = pr.lse;
+    seg_pointers(pr, &p.seg_out, &p.seg_lse, &p.row_tickets);
+    p.B = pr.B;
+    p.Hq = pr.Hq;
+    p.Hkv = pr.Hkv;
+    p.g = pr.Hq / pr.Hkv;
+    p.Lmax = pr.max_len;
+    p.P = pr.num_splits;
+    p.scale_log2e = pr.scale * kLog2e;
+    p.block_table = pl.block_table;
+    p.max_pages = pl.max_pages;
+    p.page_shift = 0;
+    while ((1 << p.page_shift) < pl.page_size) ++p.page_shift;
+    p.kv_nhd = pl.nhd ? 1 : 0;
+    return launch_split<true, true>(pr.D, p.g, tk, tv, p, pr.stream);
 }
 
 int run_combine(const Problem &pr, bool after_split) {
@@ -479,6 +557,33 @@ int fd_segments(int B, int Hkv, int max_len, const int32_t *seqlens_host, int nu
         before += n;
     }
     return static_cast<int>(slots);
+}
+
+int fd_decode_paged(int B, int Hq, int Hkv, int D, int page_size, int num_pages, int max_pages_per_seq,
+                    int kv_layout, const uint16_t *q, const uint16_t *k_pages, const uint16_t *v_pages,
+                    const int32_t *block_table, const int32_t *seqlens, float scale, float *out, float *lse,
+                    void *workspace, size_t workspace_bytes, int num_splits, void *stream) {
+    if (page_size < 8 || page_size > 4096 || (page_size & (page_size - 1)) != 0) return FD_ERR_SHAPE;
+    if (num_pages < 1 || max_pages_per_seq < 1 || (max_pages_per_seq % 4) != 0) return FD_ERR_SHAPE;
+    if (kv_layout != FD_KV_HND && kv_layout != FD_KV_NHD) return FD_ERR_SHAPE;
+    const long long max_len = static_cast<long long>(max_pages_per_seq) * page_size;
+    if (max_len > 0x7fffffffLL) return FD_ERR_SHAPE;
+    int rc = check_shape(B, Hq, Hkv, D, static_cast<int>(max_len));
+    if (rc != FD_OK) return rc;
+    if (!block_table) return FD_ERR_NULL_POINTER;
+    if (!aligned(block_table, 16)) return FD_ERR_ALIGNMENT;
+    if (num_splits < 0) return FD_ERR_SPLITS;
+    Problem pr = make_problem(B, Hq, Hkv, D, static_cast<int>(max_len), q, k_pages, v_pages, seqlens, scale, out,
+                              lse, workspace, workspace_bytes, num_splits == 0 ? 1 : num_splits, stream);
+    if ((rc = check_problem(pr, true)) != FD_OK) return rc;   // pointer / alignment checks (no CUDA call)
+    if (num_splits == 0) {
+        const int S = fd_plan(B, Hq, Hkv, D, static_cast<int>(max_len));
+        if (S < 0) return S;
+        pr.num_splits = S;
+        if ((rc = check_problem(pr, true)) != FD_OK) return rc;   // workspace for the planned count
+    }
+    PagedLayout pl{block_table, page_size, num_pages, max_pages_per_seq, kv_layout == FD_KV_NHD};
+    return run_split_paged(pr, pl);
 }
 
 int fd_decode_static(int B, int Hq, int Hkv, int D, int max_len, const uint16_t *q, const uint16_t *k_cache,

@@ -79,7 +79,14 @@ struct SplitParams {
     int *row_tickets;         // [B * Hkv], zero between calls (fused form only)
     int B, Hq, Hkv, g, Lmax, P;
     float scale_log2e;        // scale * log2(e): logits are kept in base 2
+    // paged caches only
+    const int32_t *block_table;   // [B, max_pages]: page of each sequence's logical page
+    int max_pages;            // block-table row length (a multiple of 4)
+    int page_shift;           // log2(page_size)
+    int kv_nhd;               // 0: pages [num_pages, Hkv, page_size, D]; 1: [num_pages, page_size, Hkv, D]
 };
+
+constexpr int kPageWindow = 1024;                 // block-table entries staged in shared memory
 
 template <int D, int G>
 struct SplitConfig {
@@ -92,9 +99,11 @@ struct SplitConfig {
     static constexpr int kWarpFloats = G * D + 2 * G;                      // o, m, l of one warp
     static constexpr int kMergeFloats = kConsumerWarps * kWarpFloats;      // one merge buffer
     static constexpr int kCtrlBytes = 2048;                                // barriers, start info, queue, weights
+    static constexpr int kPageBytes = kPageWindow * 4;                     // block-table window (paged)
     static constexpr int kMergeBufs =
-        1024 + kRingBytes + 2 * kMergeFloats * 4 + kCtrlBytes <= kSmemLimit ? 2 : 1;
-    static constexpr int kSmemBytes = 1024 + kRingBytes + kMergeBufs * kMergeFloats * 4 + kCtrlBytes;
+        1024 + kRingBytes + 2 * kMergeFloats * 4 + kCtrlBytes + kPageBytes <= kSmemLimit ? 2 : 1;
+    static constexpr int kSmemBytes =
+        1024 + kRingBytes + kMergeBufs * kMergeFloats * 4 + kCtrlBytes + kPageBytes;
     // Each consumer group owns whole stages: a stage shared by both groups
     // could be waited on two phases ahead of a tile still in flight, where a
     // parity wait would pass on the older phase.
@@ -572,7 +581,7 @@ struct HeadConsumer {
 };
 
 // ------------------------------------------------------------------ kernel --
-template <int D, class Consumer, bool kFused>
+template <int D, class Consumer, bool kFused, bool kPaged = false>
 __global__ void __launch_bounds__(kSplitThreads, 1)
     fd_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const SplitParams p) {
@@ -589,8 +598,11 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     uint64_t *empty = full + kStages;
     uint64_t *mfull = empty + kStages;                                     // merge buffer filled (8 warps)
     uint64_t *mempty = mfull + kBufs;                                      // merge buffer drained (finishers)
-    StartInfo *info = reinterpret_cast<StartInfo *>(mempty + kBufs);
+    uint64_t *pbar = mempty + kBufs;                                       // block-table window landed
+    StartInfo *info = reinterpret_cast<StartInfo *>(pbar + 1);
     float *weights = reinterpret_cast<float *>(info + 1);                  // [G][8] merge weights, [G] lse
+    int32_t *page_win = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(merge) +
+                                                    kBufs * Cfg::kMergeFloats * 4 + Cfg::kCtrlBytes);
 
     // A grid queued behind this one (the next call, or the standalone
     // combine) may start its prologue now; it waits for this grid's
@@ -607,6 +619,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             mbar_init(&mfull[b], kConsumerWarps);
             mbar_init(&mempty[b], kFinisherWarps);
         }
+        mbar_init(pbar, 1);
         fence_mbar_init();
     }
     if (warp == kProducerWarp && lane == 0) {   // kernel parameters, not inputs: safe before the wait
@@ -617,7 +630,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     // first tiles from seqlens as read now and pull them into L2. L2 is the
     // point of coherence, so a stale guess only wastes bandwidth; everything
     // below is recomputed from the real inputs after the wait.
-    if (warp == 0) {
+    if (!kPaged && warp == 0) {
         find_start<true>(p, info);
         __syncwarp();
         if (lane < 2 * kPrefetchTiles && info->count > 0) {
@@ -647,11 +660,30 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         // ---------------------------------------------------- producer --
         if (lane != 0 || remaining <= 0) return;
         const uint64_t policy = l2_policy_evict_first();
+        // paged caches: a window of the current sequence's block-table row in
+        // shared memory, fetched with a 1-D bulk copy when a page falls outside it
+        int win_b = -1, win_lo = 0, win_hi = 0;
+        uint32_t win_phase = 0;
+        auto page_of = [&](int b, int lp, int *page) -> bool {
+            if (b != win_b || lp < win_lo || lp >= win_hi) {
+                win_b = b;
+                win_lo = lp & ~3;
+                win_hi = min(win_lo + kPageWindow, p.max_pages);
+                const uint32_t bytes = static_cast<uint32_t>(win_hi - win_lo) * 4u;
+                mbar_arrive_expect_tx(pbar, bytes);
+                bulk_load(page_win, p.block_table + static_cast<size_t>(b) * p.max_pages + win_lo, bytes, pbar);
+                if (!wait_bounded(pbar, win_phase, abort)) return false;
+                win_phase ^= 1u;
+            }
+            *page = page_win[lp - win_lo];
+            return true;
+        };
         uint32_t seq = 0;
         while (remaining > 0) {
             const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
             const int z = c.b * p.Hkv + c.h;
             const uint16_t *q_row = p.q + (static_cast<size_t>(c.b) * p.Hq + static_cast<size_t>(c.h) * p.g) * D;
+            const int L = kPaged ? clamp_len(__ldg(p.seqlens + c.b), p.Lmax) : 0;
             for (int k = 0; k < seg; ++k, ++seq) {
                 const int stage = static_cast<int>(seq % kStages);
                 const uint32_t phase = (seq / kStages) & 1u;
@@ -659,12 +691,43 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                 uint8_t *kt = ring + stage * Cfg::kStageBytes;
                 uint8_t *vt = kt + Cfg::kTileBytes;
                 const bool with_q = k < kGroups;   // each group's first tile of the segment
-                mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kTileBytes + (with_q ? q_bytes : 0u));
+                const uint32_t qb = with_q ? q_bytes : 0u;
                 const int y = (c.tile + k) * kTileTokens;
+                if (!kPaged) {
+                    mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kTileBytes + qb);
 #pragma unroll
-                for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-                    tma_load_3d(kt + bx * kBoxBytes, &tm_k, &full[stage], 64 * bx, y, z, policy);
-                    tma_load_3d(vt + bx * kBoxBytes, &tm_v, &full[stage], 64 * bx, y, z, policy);
+                    for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+                        tma_load_3d(kt + bx * kBoxBytes, &tm_k, &full[stage], 64 * bx, y, z, policy);
+                        tma_load_3d(vt + bx * kBoxBytes, &tm_v, &full[stage], 64 * bx, y, z, policy);
+                    }
+                } else {
+                    // the tile's tokens [y, y + 64) span one page (page_size >= 64) or
+                    // 64 / page_size pages; pages past the sequence's end are not loaded
+                    // (their rows are masked), so unused block-table entries never matter
+                    const int psize = 1 << p.page_shift;
+                    const int rows = psize < kTileTokens ? psize : kTileTokens;
+                    const int lp0 = y >> p.page_shift;
+                    const int npages_seq = (L + psize - 1) >> p.page_shift;
+                    const int nsub = psize >= kTileTokens ? 1 : min(kTileTokens >> p.page_shift, npages_seq - lp0);
+                    const int off = psize >= kTileTokens ? (y & (psize - 1)) : 0;
+                    int page[kTileTokens / 8];
+                    for (int j = 0; j < nsub; ++j)
+                        if (!page_of(c.b, lp0 + j, &page[j])) return;
+                    const uint32_t sub_bytes = static_cast<uint32_t>(rows) * 128u;
+                    mbar_arrive_expect_tx(&full[stage], 2u * nsub * sub_bytes * Cfg::kBoxes + qb);
+                    for (int j = 0; j < nsub; ++j) {
+#pragma unroll
+                        for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+                            const int dst = bx * kBoxBytes + j * rows * 128;
+                            if (p.kv_nhd) {
+                                tma_load_4d(kt + dst, &tm_k, &full[stage], 64 * bx, c.h, off, page[j], policy);
+                                tma_load_4d(vt + dst, &tm_v, &full[stage], 64 * bx, c.h, off, page[j], policy);
+                            } else {
+                                tma_load_4d(kt + dst, &tm_k, &full[stage], 64 * bx, off, c.h, page[j], policy);
+                                tma_load_4d(vt + dst, &tm_v, &full[stage], 64 * bx, off, c.h, page[j], policy);
+                            }
+                        }
+                    }
                 }
                 if (with_q) bulk_load(vt + Cfg::kTileBytes, q_row, q_bytes, &full[stage]);
             }

@@ -78,3 +78,55 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu", seqlens=None) -> Decod
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """The bf16 tensor's bit patterns as a host numpy uint16 array."""
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@dataclass
+class PagedInputs:
+    """The same logical cache as a DecodeInputs, stored in a pool of pages."""
+    k_pages: torch.Tensor        # HND: [num_pages, Hkv, page_size, D]; NHD: [num_pages, page_size, Hkv, D]
+    v_pages: torch.Tensor
+    block_table: torch.Tensor    # [B, max_pages] int32, same device
+    block_table_host: np.ndarray
+    page_size: int
+    layout: str
+
+
+def make_paged(x: DecodeInputs, page_size: int, layout: str = "HND", seed: int = 0, spare_pages: int = 3,
+               unused_entry: int = -1) -> PagedInputs:
+    """Scatter x's cache into a shuffled pool of pages (data movement only).
+
+    Sequence b needs ceil(seqlens[b] / page_size) pages; the pool holds those
+    plus `spare_pages` more, in an order drawn from a CPU generator seeded
+    `seed`. Block-table entries past a sequence's pages are `unused_entry`;
+    pool slots that no sequence position maps to are NaN."""
+    w = x.workload
+    dev = x.k.device
+    lens = np.clip(x.seqlens_host.astype(np.int64), 0, w.Lmax)
+    need = [int(-(-int(L) // page_size)) for L in lens]
+    max_pages = max(1, -(-w.Lmax // page_size))
+    max_pages = (max_pages + 3) // 4 * 4
+    total = sum(need) + spare_pages
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    order = torch.randperm(total, generator=g).numpy()
+    table = np.full((w.B, max_pages), unused_entry, dtype=np.int32)
+    shape = (total, w.Hkv, page_size, w.D) if layout == "HND" else (total, page_size, w.Hkv, w.D)
+    k_pages = torch.full(shape, float("nan"), dtype=torch.bfloat16, device=dev)
+    v_pages = torch.full(shape, float("nan"), dtype=torch.bfloat16, device=dev)
+    nxt = 0
+    for b in range(w.B):
+        n = need[b]
+        if n == 0:
+            continue
+        ids = order[nxt:nxt + n]
+        nxt += n
+        table[b, :n] = ids
+        span = n * page_size
+        for src, dst in ((x.k, k_pages), (x.v, v_pages)):
+            part = src[b, :, :min(span, w.Lmax)]                           # [Hkv, tokens, D]
+            if part.shape[1] < span:
+                pad = torch.full((w.Hkv, span - part.shape[1], w.D), float("nan"), dtype=part.dtype, device=dev)
+                part = torch.cat([part, pad], dim=1)
+            part = part.reshape(w.Hkv, n, page_size, w.D)
+            part = part.permute(1, 0, 2, 3) if layout == "HND" else part.permute(1, 2, 0, 3)
+            dst[torch.from_numpy(ids.astype(np.int64)).to(dev)] = part.contiguous()
+    return PagedInputs(k_pages, v_pages, torch.from_numpy(table).to(dev), table, page_size, layout)

@@ -88,6 +88,8 @@ extern "C" {
 #define FD_MAX_SPLITS      65535
 #define FD_MAX_GROUP       16
 #define FD_STATIC_SCRATCH_BYTES (8u << 20)   /* fixed device scratch behind fd_decode_static */
+#define FD_KV_HND           0     /* paged pool [num_pages][Hkv][page_size][D] */
+#define FD_KV_NHD           1     /* paged pool [num_pages][page_size][Hkv][D] */
 
 /* Number of splits (thread blocks of the split stage) for a problem shape,
  * sized to the current device's SM count: one block per SM while the batch
@@ -132,6 +134,27 @@ FD_API int fd_decode_splits(int B, int Hq, int Hkv, int D, int max_len,
                      float *out, float *lse,
                      void *workspace, size_t workspace_bytes,
                      int num_splits, void *stream);
+
+/* fd_decode_splits over a PAGED key/value cache. The page pools
+ * k_pages / v_pages hold num_pages pages of page_size tokens each, laid out
+ * head-major (kv_layout = FD_KV_HND: [num_pages][Hkv][page_size][D] bf16) or
+ * token-major (FD_KV_NHD: [num_pages][page_size][Hkv][D] bf16), 16-byte
+ * aligned. block_table ([B][max_pages_per_seq] int32, device, 16-byte
+ * aligned) gives the page that holds logical page p of sequence b: token t
+ * of sequence b is slot t % page_size of page block_table[b][t / page_size].
+ * Only the first ceil(seqlens[b] / page_size) entries of a row are read, so
+ * the rest may hold anything; an entry outside [0, num_pages) reads as a
+ * page of zeros. seqlens[b] is clamped to [0, max_pages_per_seq * page_size].
+ * page_size: a power of two in [8, 4096]; max_pages_per_seq: a multiple of 4.
+ * num_splits = 0 means fd_plan(B, Hq, Hkv, D, max_pages_per_seq * page_size);
+ * workspace as for fd_decode with max_len = max_pages_per_seq * page_size.
+ * The paged-KV layout is the one the "flash decoding论文" page lists among
+ * PaddleNLP's attention optimisations ("PageAttention"). */
+FD_API int fd_decode_paged(int B, int Hq, int Hkv, int D, int page_size, int num_pages, int max_pages_per_seq,
+                           int kv_layout, const uint16_t *q, const uint16_t *k_pages, const uint16_t *v_pages,
+                           const int32_t *block_table, const int32_t *seqlens, float scale,
+                           float *out, float *lse, void *workspace, size_t workspace_bytes,
+                           int num_splits, void *stream);
 
 /* Split stage alone (one kernel): for each run of tiles, writes out/lse of
  * the rows it holds whole and the segments of the rows it holds in part.

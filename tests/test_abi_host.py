@@ -124,6 +124,27 @@ def test_bad_arguments_return_codes_without_a_device():
         assert L.fd_decode(1, 4, 4, 64, 64, p, p, p, p, 0.125, p, p, None, 0, None) == -8
 
 
+def test_paged_argument_errors_without_a_device():
+    L = fd.lib()
+    buf = (ctypes.c_uint8 * 4096)()
+    a16 = (ctypes.addressof(buf) + 15) // 16 * 16
+    p = ctypes.c_void_p(a16)
+
+    def paged(page_size=16, num_pages=8, max_pages=4, layout=0, bt=p, S=1, B=1, Hq=4, Hkv=2, D=128):
+        return L.fd_decode_paged(B, Hq, Hkv, D, page_size, num_pages, max_pages, layout, p, p, p, bt, p, 0.1,
+                                 p, p, p, 4096, S, None)
+
+    assert paged(page_size=24) == -2 and paged(page_size=4) == -2 and paged(page_size=8192) == -2
+    assert paged(max_pages=6) == -2 and paged(max_pages=0) == -2 and paged(num_pages=0) == -2
+    assert paged(layout=2) == -2
+    assert paged(bt=None) == -1
+    assert paged(bt=ctypes.c_void_p(a16 + 4)) == -5
+    assert paged(S=-1) == -7
+    assert paged(Hq=3) == -3 and paged(D=96) == -4
+    if not os.path.exists("/dev/nvidia0"):
+        assert paged() == -8
+
+
 def segments_rule(B, Hkv, Lmax, seqlens, P):
     """Independent statement of the documented partition: rows u = b*Hkv + j
     in order, ceil(L_b/64) tiles each, run i = flat tiles
