@@ -39,6 +39,9 @@ class Oracle:
         lib.fdo_split_attention.argtypes = ([ctypes.c_int] * 5 + [_u16p, _u16p, _u16p, _i32p, ctypes.c_double,
                                             ctypes.c_int, _i32p, _f64p, _f64p,
                                             _f64p_or_null, _f64p_or_null, ctypes.c_int])
+        lib.fdo_attention_multi.restype = ctypes.c_int
+        lib.fdo_attention_multi.argtypes = [ctypes.c_int] * 6 + [_u16p, _u16p, _u16p, _i32p, ctypes.c_double,
+                                                                 _f64p, _f64p, ctypes.c_int]
         lib.fdo_combine.restype = ctypes.c_int
         lib.fdo_combine.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _f64p, _f64p, _f64p, _f64p]
         lib.fdo_mutant.restype = ctypes.c_int
@@ -74,6 +77,26 @@ class Oracle:
         rc = self.lib.fdo_attention(B, Hq, Hkv, D, Lmax, q, k, v, seqlens, float(scale), out, lse, int(nthreads))
         if rc <= 0:
             raise RuntimeError(f"fdo_attention failed ({rc})")
+        self.threads_used = rc
+        return out, lse
+
+    def attention_multi(self, q, k, v, seqlens, scale, nthreads=0):
+        """Several queries per sequence, causal among the new tokens.
+        q [B,q_len,Hq,D]; k/v [B,Hkv,Lmax,D]; query j of sequence b sees the
+        first seqlens[b] - (q_len - 1 - j) tokens. Returns (out [B,q_len,Hq,D],
+        lse [B,q_len,Hq]) as float64."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        k = np.ascontiguousarray(k, dtype=np.uint16)
+        v = np.ascontiguousarray(v, dtype=np.uint16)
+        seqlens = np.ascontiguousarray(seqlens, dtype=np.int32)
+        B, q_len, Hq, D = q.shape
+        _, Hkv, Lmax, _ = k.shape
+        out = np.zeros((B, q_len, Hq, D), np.float64)
+        lse = np.zeros((B, q_len, Hq), np.float64)
+        rc = self.lib.fdo_attention_multi(B, q_len, Hq, Hkv, D, Lmax, q, k, v, seqlens, float(scale), out, lse,
+                                          int(nthreads))
+        if rc <= 0:
+            raise RuntimeError(f"fdo_attention_multi failed ({rc})")
         self.threads_used = rc
         return out, lse
 
@@ -132,6 +155,10 @@ def combine(part_o, part_lse):
     return default().combine(part_o, part_lse)
 
 
+def attention_multi(q, k, v, seqlens, scale, nthreads=0):
+    return default().attention_multi(q, k, v, seqlens, scale, nthreads)
+
+
 LIBRARY = _build.LIBRARY
 SOURCE = _build.SOURCE
-__all__ = ["Oracle", "default", "attention", "split_attention", "combine", "LIBRARY", "SOURCE"]
+__all__ = ["Oracle", "default", "attention", "attention_multi", "split_attention", "combine", "LIBRARY", "SOURCE"]

@@ -19,6 +19,14 @@
  *    maximum before exp() is exact in real arithmetic; it only keeps exp()
  *    from overflowing in double for large logits.
  *
+ *  - Several queries per sequence ("flash decoding论文" page: with multi-turn
+ *    dialogue or speculative decoding several query vectors are computed in
+ *    parallel). Reading taken: sequence b holds L = seqlens[b] cached tokens
+ *    of which the last q_len are the new ones, in order; query j (0-based)
+ *    is the token at position L - q_len + j and attends causally to tokens
+ *    t < L - (q_len - 1 - j). fdo_attention_multi() is the same definition
+ *    with that length per query; q_len = 1 is fdo_attention().
+ *
  *  - Section "A faster attention for decoding: Flash-Decoding": the keys and
  *    values are cut into chunks along the sequence, the attention of the
  *    query with each chunk is computed on its own together with one extra
@@ -75,6 +83,8 @@ typedef struct {
     const int32_t *bounds;   /* nsplit + 1 token boundaries, ascending */
     double *part_o;          /* [B, Hq, nsplit, D] or NULL */
     double *part_lse;        /* [B, Hq, nsplit]    or NULL */
+    /* several queries per sequence (fdo_attention_multi) */
+    int q_len;
     /* thread partition */
     int nthreads, tid;
 } job_t;
@@ -85,15 +95,14 @@ static int clamp_len(int L, int Lmax) {
     return L;
 }
 
-/* Logits z_t = scale * <q, k_t> for t in [t0, t1) of one row. */
-static void row_logits(const job_t *J, int b, int i, int t0, int t1, double *z) {
+/* Logits z_t = scale * <qrow, k_t> for t in [t0, t1), query head i of sequence b. */
+static void row_logits(const job_t *J, int b, int i, const uint16_t *qrow, int t0, int t1, double *z) {
     const int g = J->Hq / J->Hkv;
 #if FDO_MUTANT == 2
     const int j = i % J->Hkv;                     /* planted: wrong group map */
 #else
     const int j = i / g;
 #endif
-    const uint16_t *qrow = J->q + ((size_t)b * J->Hq + i) * J->D;
     for (int t = t0; t < t1; ++t) {
         const uint16_t *krow = J->k + (((size_t)b * J->Hkv + j) * J->Lmax + t) * J->D;
         double dot = 0.0;
@@ -159,7 +168,7 @@ static void *attention_worker(void *arg) {
     for (int r = J->tid; r < rows; r += J->nthreads) {
         const int b = r / J->Hq, i = r % J->Hq;
         const int L = row_length(J, b);
-        row_logits(J, b, i, 0, L, z);
+        row_logits(J, b, i, J->q + (size_t)r * J->D, 0, L, z);
         J->lse[r] = row_softmax_sum(J, b, i, 0, L, z, J->out + (size_t)r * J->D);
     }
     free(z);
@@ -207,7 +216,7 @@ static void *split_worker(void *arg) {
             int t0 = J->bounds[s], t1 = J->bounds[s + 1];
             if (t0 > L) t0 = L;
             if (t1 > L) t1 = L;
-            row_logits(J, b, i, t0, t1, z);
+            row_logits(J, b, i, J->q + ((size_t)b * J->Hq + i) * J->D, t0, t1, z);
             pl[s] = row_softmax_sum(J, b, i, t0, t1, z, po + (size_t)s * J->D);
         }
         if (J->part_o) memcpy(J->part_o + (size_t)r * n * J->D, po, sizeof(double) * (size_t)n * J->D);
@@ -219,12 +228,11 @@ static void *split_worker(void *arg) {
     return NULL;
 }
 
-static int run_threads(job_t *proto, void *(*fn)(void *), int nthreads) {
+static int run_threads_rows(job_t *proto, void *(*fn)(void *), int nthreads, int rows) {
     if (nthreads <= 0) {
         long c = sysconf(_SC_NPROCESSORS_ONLN);
         nthreads = c > 0 ? (int)c : 1;
     }
-    const int rows = proto->B * proto->Hq;
     if (nthreads > rows) nthreads = rows > 0 ? rows : 1;
     job_t *jobs = (job_t *)malloc(sizeof(job_t) * (size_t)nthreads);
     pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
@@ -246,6 +254,10 @@ static int run_threads(job_t *proto, void *(*fn)(void *), int nthreads) {
     }
     free(jobs); free(th);
     return rc == 0 ? nthreads : rc;
+}
+
+static int run_threads(job_t *proto, void *(*fn)(void *), int nthreads) {
+    return run_threads_rows(proto, fn, nthreads, proto->B * proto->Hq);
 }
 
 static int check_shape(int B, int Hq, int Hkv, int D, int Lmax) {
@@ -270,6 +282,47 @@ int fdo_attention(int B, int Hq, int Hkv, int D, int Lmax,
     J.q = q; J.k = k; J.v = v; J.seqlens = seqlens; J.scale = scale;
     J.out = out; J.lse = lse;
     return run_threads(&J, attention_worker, nthreads);
+}
+
+/* --- several queries per sequence, causal among the new tokens --------- */
+
+static void *multi_worker(void *arg) {
+    const job_t *J = (const job_t *)arg;
+    double *z = (double *)malloc(sizeof(double) * (size_t)(J->Lmax > 0 ? J->Lmax : 1));
+    if (!z) return (void *)1;
+    /* q, out: [B, q_len, Hq, D]; lse: [B, q_len, Hq]. Row r = (b*q_len + j)*Hq + i. */
+    const int rows = J->B * J->q_len * J->Hq;
+    for (int r = J->tid; r < rows; r += J->nthreads) {
+        const int i = r % J->Hq, bj = r / J->Hq;
+        const int j = bj % J->q_len, b = bj / J->q_len;
+        int L = row_length(J, b);
+#if FDO_MUTANT == 8
+        L -= J->q_len - j;                           /* planted: query sees one token too few */
+#else
+        L -= J->q_len - 1 - j;                       /* query j sees t < L - (q_len - 1 - j) */
+#endif
+        if (L < 0) L = 0;
+        row_logits(J, b, i, J->q + (size_t)r * J->D, 0, L, z);
+        J->lse[r] = row_softmax_sum(J, b, i, 0, L, z, J->out + (size_t)r * J->D);
+    }
+    free(z);
+    return NULL;
+}
+
+/* Several queries per sequence: q [B,q_len,Hq,D], k/v [B,Hkv,Lmax,D], seqlens [B];
+ * out [B,q_len,Hq,D], lse [B,q_len,Hq]. Returns threads used or a negative value. */
+int fdo_attention_multi(int B, int q_len, int Hq, int Hkv, int D, int Lmax,
+                        const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        const int32_t *seqlens, double scale,
+                        double *out, double *lse, int nthreads) {
+    if (check_shape(B, Hq, Hkv, D, Lmax) || q_len < 1) return -1;
+    if (B == 0) return 1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.Lmax = Lmax;
+    J.q = q; J.k = k; J.v = v; J.seqlens = seqlens; J.scale = scale;
+    J.out = out; J.lse = lse; J.q_len = q_len;
+    return run_threads_rows(&J, multi_worker, nthreads, B * q_len * Hq);
 }
 
 /* Split-then-reduce form. bounds holds nsplit+1 ascending token positions;

@@ -286,6 +286,51 @@ def pin_group_mapping(orc):
             raise AssertionError(f"group mapping: kv head {j} differs")
 
 
+def pin_multi_query_decimal(orc):
+    """Several queries per sequence against 50-digit decimal evaluation:
+    query j of a sequence with L cached tokens sees its first
+    L - (q_len - 1 - j) tokens."""
+    rng = np.random.default_rng(77)
+    for trial in range(6):
+        q_len = 1 + trial % 4
+        Hkv, g = [1, 2][trial % 2], [1, 3][trial % 2]
+        Hq, D, Lmax = Hkv * g, 1 + trial % 3, 9
+        seqlens = np.array([9, q_len + (trial % 3)], np.int32)
+        scale = float(rng.uniform(0.3, 1.2))
+        q = to_bits(rng.standard_normal((2, q_len, Hq, D)))
+        _, k, v, _ = rand_case(rng, 2, Hq, Hkv, D, Lmax, seqlens, sigma=(1.0, 2.0, 1.0))
+        out, lse = orc.attention_multi(q, k, v, seqlens, scale)
+        qf, kf, vf = bits_to_f64(q), bits_to_f64(k), bits_to_f64(v)
+        for b in range(2):
+            for j in range(q_len):
+                Lq = int(seqlens[b]) - (q_len - 1 - j)
+                for i in range(Hq):
+                    eo, el = decimal_row(qf[b, j, i], kf[b, i // g], vf[b, i // g], Lq, scale)
+                    close(out[b, j, i], eo, 1e-12, f"multi-query out b={b} j={j} i={i}")
+                    close(lse[b, j, i], el, 1e-12, f"multi-query lse b={b} j={j} i={i}")
+
+
+def pin_multi_query_library_mask(orc):
+    """Several queries against torch scaled_dot_product_attention (float64)
+    with an explicit boolean mask built from the causal-offset rule."""
+    rng = np.random.default_rng(78)
+    B, q_len, Hq, Hkv, D, Lmax = 2, 4, 6, 2, 8, 30
+    seq = np.array([30, 11], np.int32)
+    q = to_bits(rng.standard_normal((B, q_len, Hq, D)))
+    _, k, v, seq = rand_case(rng, B, Hq, Hkv, D, Lmax, seq)
+    out, lse = orc.attention_multi(q, k, v, seq, 0.3)
+    qf, kf, vf = (torch.from_numpy(bits_to_f64(a)) for a in (q, k, v))
+    for b in range(B):
+        L = int(seq[b])
+        mask = torch.zeros((q_len, L), dtype=torch.bool)
+        for j in range(q_len):
+            mask[j, :L - (q_len - 1 - j)] = True
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            qf[b].permute(1, 0, 2)[None], kf[b, :, :L][None], vf[b, :, :L][None], attn_mask=mask, scale=0.3,
+            enable_gqa=True)                                            # [1, Hq, q_len, D]
+        close(out[b], ref[0].permute(1, 0, 2).numpy(), 1e-12, "multi-query sdpa out")
+
+
 ALL_PINS = [
     pin_brute_force_decimal,
     pin_worked_examples,
@@ -296,4 +341,6 @@ ALL_PINS = [
     pin_invariants,
     pin_padding_and_empty,
     pin_group_mapping,
+    pin_multi_query_decimal,
+    pin_multi_query_library_mask,
 ]

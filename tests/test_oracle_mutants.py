@@ -16,6 +16,7 @@ MUTANTS = {
     5: "keys used as values",
     6: "softmax weights not normalised",
     7: "split weights not rescaled by the total log-sum-exp",
+    8: "each of several queries sees one token too few",
 }
 
 
