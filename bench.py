@@ -133,15 +133,16 @@ class ClockSampler:
 
 # ------------------------------------------------------------ byte counts --
 
-def byte_counts(w, lens, S):
+def byte_counts(w, lens, S, q_len=1):
     """Algorithmic bytes of one call: K/V inside the sequences, q, and the
-    outputs / workspace segments each stage writes and reads."""
+    outputs / workspace segments each stage writes and reads (q_len queries
+    per sequence: q_len times the query and output bytes)."""
     lens = np.clip(lens.astype(np.int64), 0, w.Lmax)
     kv = int(lens.sum()) * w.Hkv * w.D * 2 * 2
-    q = w.B * w.Hq * w.D * 2
+    q = w.B * q_len * w.Hq * w.D * 2
     seg = fd.fd_segments(w.B, w.Hkv, w.Lmax, lens.astype(np.int32), S)
     used = seg["row"] >= 0
-    row_bytes = w.g * (w.D + 1) * 4
+    row_bytes = q_len * w.g * (w.D + 1) * 4
     n_whole = int(seg["whole"][used].sum())
     n_part = int(used.sum()) - n_whole
     multi_rows = len(set(seg["row"][used & (seg["whole"] == 0)].tolist()))
@@ -262,12 +263,19 @@ def run_fd(args, w, rank, world):
         l2_note = "L2 flushed before every timed call (256 MiB write outside the timed events)"
     for c in range(1, n_copies):
         xs.append(make_inputs(w, rank_seed(args.seed, rank) + 1000 * c, device=dev))
-    nbytes = fd.fd_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, w.Lmax, S)
+    Q = args.q_len
+    nbytes = fd.fd_workspace_bytes(w.B, w.Hq * Q, w.Hkv, w.D, w.Lmax, S)
     ws = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=dev)      # row counters start at zero
-    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
-    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    oshape = (w.B, w.Hq) if Q == 1 else (w.B, Q, w.Hq)
+    out = torch.empty(oshape + (w.D,), dtype=torch.float32, device=dev)
+    lse = torch.empty(oshape, dtype=torch.float32, device=dev)
+    if Q > 1:
+        # q_len new tokens per sequence: queries [B, q_len, Hq, D] drawn like q
+        for i, x in enumerate(xs):
+            g = torch.Generator(device=dev).manual_seed(rank_seed(args.seed, rank) + 77 + i)
+            x.q = (torch.randn((w.B, Q, w.Hq, w.D), generator=g, device=dev) * w.sigma_q).to(torch.bfloat16)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if n_copies == 1 else None
-    counts = byte_counts(w, xs[0].seqlens_host, S)
+    counts = byte_counts(w, xs[0].seqlens_host, S, Q)
     kv_bytes = sum(x.kv_bytes() for x in xs) / n_copies
     if args.paged:
         # the same logical caches, scattered into shuffled page pools
@@ -278,6 +286,8 @@ def run_fd(args, w, rank, world):
         torch.cuda.empty_cache()
         calls = [fd.prepare_decode_paged(x.q, pg.k_pages, pg.v_pages, pg.block_table, x.seqlens, x.scale, out, lse,
                                          ws, args.layout, S, stream) for x, pg in zip(xs, pgs)]
+    elif Q > 1:
+        calls = [fd.prepare_decode_multi(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream) for x in xs]
     else:
         calls = [fd.prepare_decode(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream) for x in xs]
 
@@ -326,7 +336,7 @@ def run_fd(args, w, rank, world):
 
     # ---- the two stages as separate kernels (for the per-stage split) ------
     ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-             torch.cuda.Event(enable_timing=True)) for _ in range(args.steps if not args.paged else 0)]
+             torch.cuda.Event(enable_timing=True)) for _ in range(args.steps if not args.paged and Q == 1 else 0)]
     for i in range(len(ev_s)):
         x = xs[i % n_copies]
         if flush is not None:
@@ -347,8 +357,8 @@ def run_fd(args, w, rank, world):
         hq, hk, hv = x.q.cpu().pin_memory(), x.k.cpu().pin_memory(), x.v.cpu().pin_memory()
         hs = x.seqlens.cpu().pin_memory()
         dq, dk, dv, dsq = (torch.empty_like(t) for t in (x.q, x.k, x.v, x.seqlens))
-        ho = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32).pin_memory()
-        hl = torch.empty((w.B, w.Hq), dtype=torch.float32).pin_memory()
+        ho = torch.empty(tuple(out.shape), dtype=torch.float32).pin_memory()
+        hl = torch.empty(tuple(lse.shape), dtype=torch.float32).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs))
         d2h = ho.numel() * 4 + hl.numel() * 4
         e_steps = max(3, min(args.steps, 20))
@@ -358,7 +368,10 @@ def run_fd(args, w, rank, world):
             dk.copy_(hk, non_blocking=True)
             dv.copy_(hv, non_blocking=True)
             dsq.copy_(hs, non_blocking=True)
-            fd.fd_decode_splits(dq, dk, dv, dsq, x.scale, out, lse, ws, S, stream)
+            if Q > 1:
+                fd.fd_decode_multi(dq, dk, dv, dsq, x.scale, out, lse, ws, S, stream)
+            else:
+                fd.fd_decode_splits(dq, dk, dv, dsq, x.scale, out, lse, ws, S, stream)
             ho.copy_(out, non_blocking=True)
             hl.copy_(lse, non_blocking=True)
 
@@ -389,13 +402,13 @@ def run_fd(args, w, rank, world):
         "warmup": max(3, args.warmup), "ms_per_step": ms_max / args.steps, "us_per_call": us_per_call,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(config_dict(w, S, l2_note), **({"paged": {"page_size": args.paged, "layout": args.layout}}
-                                                      if args.paged else {})),
+                                                      if args.paged else {}), **({"q_len": Q} if Q > 1 else {})),
         "pct_of_nominal_hbm": 100.0 * gbs / world / NOMINAL_HBM_GBS,
         "pct_of_measured_copy": 100.0 * gbs / world / peak,
         "call_bytes_gbs": world * counts["total"] * args.steps / (ms_max * 1e-3) / 1e9,
         "roofline": {"kernel": "fd_split_kernel (fused combine)", "bound": "hbm", "achieved": kernel_gbs,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": kernel_gbs / peak,
-                     "traffic": None if args.paged else measured_traffic(w.name), "bytes_per_launch": counts["total"],
+                     "traffic": None if args.paged or Q > 1 else measured_traffic(w.name), "bytes_per_launch": counts["total"],
                      "us_per_launch": us_per_call,
                      "frac_of_nominal_8tbs": kernel_gbs / NOMINAL_HBM_GBS},
         "stages_alone": {"split_us": split_us, "combine_us": combine_us},
@@ -404,7 +417,7 @@ def run_fd(args, w, rank, world):
         "e2e": e2e,
         "wall_s": wall,
     }
-    if world == 1 and not args.no_cpu_baseline and not args.paged:
+    if world == 1 and not args.no_cpu_baseline and not args.paged and Q == 1:
         b, s, t, desc = oracle_sample(xs[0], budget_s=args.cpu_seconds)
         line["cpu_baseline"] = {"value": b / s / 1e9, "unit": "GB/s", "cores": t, "kind": "oracle",
                                 "sample": desc, "seconds": s}
@@ -426,6 +439,8 @@ def main():
     ap.add_argument("--paged", type=int, default=0, metavar="PAGE_SIZE",
                     help="read the caches from a shuffled page pool with this page size (fd_decode_paged)")
     ap.add_argument("--layout", choices=["HND", "NHD"], default="HND", help="page layout for --paged")
+    ap.add_argument("--q-len", type=int, default=1,
+                    help="new tokens per sequence, each a query seeing the cache up to itself (fd_decode_multi)")
     ap.add_argument("--no-clock-window", action="store_true",
                     help="do not extend clock sampling past the timed region (for profiler runs)")
     args = ap.parse_args()

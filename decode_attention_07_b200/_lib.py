@@ -56,12 +56,13 @@ def lib() -> ctypes.CDLL:
         L.fd_workspace_init.argtypes = [_p, _sz, _p]
         L.fd_decode_static.argtypes = [_i] * 5 + [_p, _p, _p, _p, _f, _p, _p, _p]
         L.fd_decode_paged.argtypes = [_i] * 8 + [_p, _p, _p, _p, _p, _f, _p, _p, _p, _sz, _i, _p]
+        L.fd_decode_multi.argtypes = [_i] * 6 + [_p, _p, _p, _p, _f, _p, _p, _p, _sz, _i, _p]
         L.fd_strerror.argtypes = [_i]
         L.fd_strerror.restype = ctypes.c_char_p
         L.fd_version.argtypes = []
         for name in ("fd_plan", "fd_plan_for_sms", "fd_decode", "fd_decode_splits", "fd_split", "fd_combine",
                      "fd_segments", "fd_device_status", "fd_version", "fd_workspace_init", "fd_decode_static",
-                     "fd_decode_paged"):
+                     "fd_decode_paged", "fd_decode_multi"):
             getattr(L, name).restype = _i
         _lib = L
     return _lib
@@ -189,6 +190,26 @@ def fd_decode_static(q, k_cache, v_cache, seqlens, scale, out, lse, stream=None)
                                   _stream(stream, q.device)), "fd_decode_static")
 
 
+def fd_decode_multi(q, k_cache, v_cache, seqlens, scale, out, lse, workspace=None, num_splits=0, stream=None):
+    """Several queries per sequence: q [B, q_len, Hq, D], out [B, q_len, Hq, D],
+    lse [B, q_len, Hq]; query j sees the first seqlens[b] - (q_len-1-j) tokens.
+    num_splits 0 lets the library plan the split count."""
+    prepare_decode_multi(q, k_cache, v_cache, seqlens, scale, out, lse, workspace, num_splits, stream)()
+
+
+def decode_multi(q, k_cache, v_cache, seqlens, scale, num_splits=None, stream=None):
+    """Allocate out / lse / workspace with torch and run fd_decode_multi."""
+    B, q_len, Hq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    S = fd_plan(B, Hq, Hkv, D, Lmax) if num_splits is None else int(num_splits)
+    nbytes = fd_workspace_bytes(B, Hq * q_len, Hkv, D, Lmax, S)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
+    out = torch.empty((B, q_len, Hq, D), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, q_len, Hq), dtype=torch.float32, device=q.device)
+    fd_decode_multi(q, k_cache, v_cache, seqlens, scale, out, lse, ws, S, stream)
+    return out, lse
+
+
 def _paged_shapes(q, k_pages, v_pages, block_table, layout):
     if layout not in LAYOUTS:
         raise ValueError("layout must be 'HND' ([pages, Hkv, page_size, D]) or 'NHD' ([pages, page_size, Hkv, D])")
@@ -292,6 +313,35 @@ def prepare_decode(q, k_cache, v_cache, seqlens, scale, out, lse, workspace=None
         rc = fn(*args)
         if rc != 0:
             raise FdError(rc, "fd_decode_splits")
+
+    call.num_splits = S
+    return call
+
+
+def prepare_decode_multi(q, k_cache, v_cache, seqlens, scale, out, lse, workspace=None, num_splits=None,
+                         stream=None):
+    """prepare_decode for fd_decode_multi: q [B, q_len, Hq, D], out
+    [B, q_len, Hq, D], lse [B, q_len, Hq]."""
+    if q.dim() != 4 or not q.is_contiguous():
+        raise ValueError("q must be a contiguous [B, q_len, Hq, D] tensor")
+    B, q_len, Hq, D = q.shape
+    _, _, Hkv, _, Lmax = _shapes(q.view(B, q_len * Hq, D), k_cache, v_cache)
+    if out.shape != (B, q_len, Hq, D) or lse.shape != (B, q_len, Hq):
+        raise ValueError("out must be [B,q_len,Hq,D] and lse [B,q_len,Hq]")
+    for t, name in ((out, "out"), (lse, "lse")):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor")
+    _seqlens(seqlens, B)
+    S = fd_plan(B, Hq, Hkv, D, Lmax) if num_splits is None else int(num_splits)
+    wp, wb = _ws(workspace)
+    fn = lib().fd_decode_multi
+    args = (B, q_len, Hq, Hkv, D, Lmax, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+            ctypes.c_float(scale), out.data_ptr(), lse.data_ptr(), wp, wb, S, _stream(stream, q.device))
+
+    def call():
+        rc = fn(*args)
+        if rc != 0:
+            raise FdError(rc, "fd_decode_multi")
 
     call.num_splits = S
     return call

@@ -286,8 +286,9 @@ int check_problem(const Problem &pr, bool need_kv) {
     return FD_OK;
 }
 
-void seg_pointers(const Problem &pr, float **so, float **sl, int **tickets) {
-    const WorkspaceLayout w = workspace_layout(pr.B, pr.Hq, pr.Hkv, pr.D, pr.num_splits);
+// `q_len` query positions per sequence: a segment holds q_len * g columns.
+void seg_pointers(const Problem &pr, float **so, float **sl, int **tickets, int q_len = 1) {
+    const WorkspaceLayout w = workspace_layout(pr.B, pr.Hq * q_len, pr.Hkv, pr.D, pr.num_splits);
     if (w.total == 0) {
         *so = *sl = nullptr;
         *tickets = nullptr;
@@ -300,8 +301,9 @@ void seg_pointers(const Problem &pr, float **so, float **sl, int **tickets) {
 }
 
 // The split kernel; `fused` adds the in-kernel combine (fd_decode), without it
-// the segments are left for fd_combine.
-int run_split(const Problem &pr, bool fused) {
+// the segments are left for fd_combine. q_len > 1: several queries per
+// sequence (pr.Hq counts query heads of one query position).
+int run_split(const Problem &pr, bool fused, int q_len = 1) {
     int sms;
     int rc = device_sms(&sms);
     if (rc != FD_OK) return rc;
@@ -320,13 +322,15 @@ int run_split(const Problem &pr, bool fused) {
     p.seqlens = pr.seqlens;
     p.out = pr.out;
     p.lse = pr.lse;
-    seg_pointers(pr, &p.seg_out, &p.seg_lse, &p.row_tickets);
+    seg_pointers(pr, &p.seg_out, &p.seg_lse, &p.row_tickets, q_len);
     p.B = pr.B;
     p.Hq = pr.Hq;
     p.Hkv = pr.Hkv;
     p.g = pr.Hq / pr.Hkv;
     p.Lmax = pr.max_len;
     p.P = pr.num_splits;
+    p.q_len = q_len;
+    p.cols = p.g * q_len;
     p.scale_log2e = pr.scale * kLog2e;
     p.block_table = nullptr;
     p.max_pages = 0;
@@ -334,8 +338,8 @@ int run_split(const Problem &pr, bool fused) {
     p.kv_nhd = 0;
     // with max_len == 0 every block finds zero tiles and only writes empty rows;
     // the (unused) tensor maps stay zeroed
-    return fused ? launch_split<true>(pr.D, p.g, tk, tv, p, pr.stream)
-                 : launch_split<false>(pr.D, p.g, tk, tv, p, pr.stream);
+    return fused ? launch_split<true>(pr.D, p.cols, tk, tv, p, pr.stream)
+                 : launch_split<false>(pr.D, p.cols, tk, tv, p, pr.stream);
 }
 
 struct PagedLayout {
@@ -363,6 +367,8 @@ int run_split_paged(const Problem &pr, const PagedLayout &pl) {
     p.g = pr.Hq / pr.Hkv;
     p.Lmax = pr.max_len;
     p.P = pr.num_splits;
+    p.q_len = 1;
+    p.cols = p.g;
     p.scale_log2e = pr.scale * kLog2e;
     p.block_table = pl.block_table;
     p.max_pages = pl.max_pages;
@@ -584,6 +590,29 @@ int fd_decode_paged(int B, int Hq, int Hkv, int D, int page_size, int num_pages,
     }
     PagedLayout pl{block_table, page_size, num_pages, max_pages_per_seq, kv_layout == FD_KV_NHD};
     return run_split_paged(pr, pl);
+}
+
+int fd_decode_multi(int B, int q_len, int Hq, int Hkv, int D, int max_len, const uint16_t *q,
+                    const uint16_t *k_cache, const uint16_t *v_cache, const int32_t *seqlens, float scale, float *out,
+                    float *lse, void *workspace, size_t workspace_bytes, int num_splits, void *stream) {
+    if (q_len < 1 || q_len > FD_MAX_GROUP) return FD_ERR_SHAPE;
+    int rc = check_shape(B, Hq, Hkv, D, max_len);
+    if (rc != FD_OK) return rc;
+    if (static_cast<long long>(Hq) * q_len / Hkv > FD_MAX_GROUP) return FD_ERR_GROUP;
+    if (num_splits < 0) return FD_ERR_SPLITS;
+    // the workspace and the checks see the (query, head) columns as Hq * q_len query heads
+    const int Hqq = Hq * q_len;
+    Problem pr = make_problem(B, Hqq, Hkv, D, max_len, q, k_cache, v_cache, seqlens, scale, out, lse, workspace,
+                              workspace_bytes, num_splits == 0 ? 1 : num_splits, stream);
+    if ((rc = check_problem(pr, true)) != FD_OK) return rc;
+    if (num_splits == 0) {
+        const int S = fd_plan(B, Hq, Hkv, D, max_len);
+        if (S < 0) return S;
+        pr.num_splits = S;
+        if ((rc = check_problem(pr, true)) != FD_OK) return rc;
+    }
+    pr.Hq = Hq;   // the kernel indexes q / out with the real head count
+    return run_split(pr, true, q_len);
 }
 
 int fd_decode_static(int B, int Hq, int Hkv, int D, int max_len, const uint16_t *q, const uint16_t *k_cache,

@@ -78,6 +78,8 @@ struct SplitParams {
     float *seg_lse;           // [slots, g]
     int *row_tickets;         // [B * Hkv], zero between calls (fused form only)
     int B, Hq, Hkv, g, Lmax, P;
+    int q_len;                // queries per sequence (1: plain decode)
+    int cols;                 // g * q_len: (query, head) columns per (sequence, kv head) row
     float scale_log2e;        // scale * log2(e): logits are kept in base 2
     // paged caches only
     const int32_t *block_table;   // [B, max_pages]: page of each sequence's logical page
@@ -87,6 +89,13 @@ struct SplitParams {
 };
 
 constexpr int kPageWindow = 1024;                 // block-table entries staged in shared memory
+
+// Output row of column `col` of row (b, h): column col = j*g + i is query j,
+// query head h*g + i; out is [B, q_len, Hq, D] and lse [B, q_len, Hq].
+__device__ __forceinline__ size_t out_row(const SplitParams &p, int b, int h, int col) {
+    const int j = col / p.g, i = col - j * p.g;
+    return (static_cast<size_t>(b) * p.q_len + j) * p.Hq + static_cast<size_t>(h) * p.g + i;
+}
 
 template <int D, int G>
 struct SplitConfig {
@@ -246,7 +255,7 @@ __device__ __forceinline__ void merge_warps_and_store(const float *merge, float 
                                                       int nthreads, Bar bar) {
     constexpr int kWarpFloats = G * D + 2 * G;
     float *lse_h = weights + G * kConsumerWarps;   // [G] natural-log lse per head
-    for (int head = tid; head < p.g; head += nthreads) {
+    for (int head = tid; head < p.cols; head += nthreads) {
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge[w * kWarpFloats + G * D + head]);
@@ -268,18 +277,18 @@ __device__ __forceinline__ void merge_warps_and_store(const float *merge, float 
         }
     }
     bar();
-    for (int idx = tid; idx < p.g * D; idx += nthreads) {
+    for (int idx = tid; idx < p.cols * D; idx += nthreads) {
         const int head = idx / D, d = idx - head * D;
         float o = 0.f;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w)
             o = fmaf(weights[head * kConsumerWarps + w], merge[w * kWarpFloats + head * D + d], o);
         if (whole) {
-            const size_t row = static_cast<size_t>(c.b) * p.Hq + static_cast<size_t>(c.h) * p.g + head;
+            const size_t row = out_row(p, c.b, c.h, head);
             p.out[row * D + d] = o;
             if (d == 0) p.lse[row] = lse_h[head];
         } else {
-            const size_t row = slot * p.g + head;
+            const size_t row = slot * p.cols + head;
             p.seg_out[row * D + d] = o;
             if (d == 0) p.seg_lse[row] = lse_h[head];
         }
@@ -296,6 +305,18 @@ struct GroupConsumer {
     uint32_t qf[NT][KS][2];             // Q^T as the B operand, per n-tile
     float m[NT][2], l[NT][2];           // running max (base 2) / partial sum for heads 2c, 2c+1
     float o[NT][MT][4];                 // O^T accumulators
+    int shift[NT][2];                   // causal offset of columns 2c, 2c+1: q_len - 1 - query index
+
+    __device__ __forceinline__ void init(const SplitParams &p) {
+        const int cc = (threadIdx.x & 31) & 3;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int col = nt * 8 + 2 * cc + e;
+                shift[nt][e] = col < p.cols ? p.q_len - 1 - col / p.g : 0;
+            }
+    }
 
     __device__ __forceinline__ void reset() {
 #pragma unroll
@@ -365,8 +386,12 @@ struct GroupConsumer {
         for (int nt = 0; nt < NT; ++nt) {
             float x0 = (s[nt][0] + s2[nt][0]) * scale_log2e, x1 = (s[nt][1] + s2[nt][1]) * scale_log2e;
             float x2 = (s[nt][2] + s2[nt][2]) * scale_log2e, x3 = (s[nt][3] + s2[nt][3]) * scale_log2e;
-            if (r0 >= valid) x0 = x1 = -INFINITY;
-            if (r0 + 8 >= valid) x2 = x3 = -INFINITY;
+            // token r of this warp's slice is inside column e's causal range when r < valid - shift
+            const int va = valid - shift[nt][0], vb = valid - shift[nt][1];
+            if (r0 >= va) x0 = -INFINITY;
+            if (r0 >= vb) x1 = -INFINITY;
+            if (r0 + 8 >= va) x2 = -INFINITY;
+            if (r0 + 8 >= vb) x3 = -INFINITY;
             float ma = fmaxf(x0, x2), mb = fmaxf(x1, x3);
 #pragma unroll
             for (int sh = 4; sh < 32; sh <<= 1) {
@@ -458,6 +483,8 @@ struct HeadConsumer {
     float qv[8];                               // q[d0 .. d0+7] of this lane's 16-byte chunk
     float m, l;                                // running max (base 2, warp-uniform) / lane partial sum
     float acc[8];                              // sum of p * v over this lane's tokens, chunk d0..d0+7
+
+    __device__ __forceinline__ void init(const SplitParams &) {}   // one query, one head: no offsets
 
     __device__ __forceinline__ void reset() {
         m = -INFINITY;
@@ -654,7 +681,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     Cursor c{info->b, info->h, info->tile, info->n, info->first};
     const long long N = info->N;
     volatile int *abort = &info->abort;
-    const uint32_t q_bytes = static_cast<uint32_t>(p.g) * D * 2;
+    const uint32_t q_bytes = static_cast<uint32_t>(p.cols) * D * 2;   // q_len copies of g rows
 
     if (warp == kProducerWarp) {
         // ---------------------------------------------------- producer --
@@ -682,7 +709,10 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         while (remaining > 0) {
             const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
             const int z = c.b * p.Hkv + c.h;
-            const uint16_t *q_row = p.q + (static_cast<size_t>(c.b) * p.Hq + static_cast<size_t>(c.h) * p.g) * D;
+            // query j's g heads: q[b, j, h*g .. h*g+g-1, :], one contiguous run per j
+            const uint16_t *q_row =
+                p.q + (static_cast<size_t>(c.b) * p.q_len * p.Hq + static_cast<size_t>(c.h) * p.g) * D;
+            const uint32_t q_run = static_cast<uint32_t>(p.g) * D * 2;
             const int L = kPaged ? clamp_len(__ldg(p.seqlens + c.b), p.Lmax) : 0;
             for (int k = 0; k < seg; ++k, ++seq) {
                 const int stage = static_cast<int>(seq % kStages);
@@ -729,7 +759,10 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                         }
                     }
                 }
-                if (with_q) bulk_load(vt + Cfg::kTileBytes, q_row, q_bytes, &full[stage]);
+                if (with_q)
+                    for (int j = 0; j < p.q_len; ++j)
+                        bulk_load(vt + Cfg::kTileBytes + j * q_run, q_row + static_cast<size_t>(j) * p.Hq * D, q_run,
+                                  &full[stage]);
             }
             remaining -= seg;
             if (remaining > 0) next_row(c, p);
@@ -743,6 +776,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         // ---------------------------------------------------- consumers --
         const int group = warp / kSliceWarps, slice = warp % kSliceWarps;
         Consumer cons;
+        cons.init(p);
         uint32_t seq = 0, segctr = 0;
         while (remaining > 0) {
             const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
@@ -754,7 +788,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                 const uint32_t phase = (seq / kStages) & 1u;
                 wait_bounded(&full[stage], phase, abort);   // on abort: keep going, outputs are flagged invalid
                 const uint8_t *st = ring + stage * Cfg::kStageBytes;
-                if (k < kGroups) cons.load_q(st + 2 * Cfg::kTileBytes, p.g);
+                if (k < kGroups) cons.load_q(st + 2 * Cfg::kTileBytes, p.cols);
                 const uint32_t kt = smem_addr(st);
                 const int valid = L - ((c.tile + k) * kTileTokens + kWarpTokens * slice);
                 cons.tile(kt, kt + Cfg::kTileBytes, slice, valid, p.scale_log2e);
@@ -844,18 +878,18 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         // all queued rows at once: one float4 output per thread and step
         const int npending = *reinterpret_cast<volatile int *>(&info->npending);
         constexpr int kVec = D / 4;
-        for (int idx = wtid; idx < npending * p.g * kVec; idx += kWorkerThreads) {
-            const int i = idx / (p.g * kVec), rem = idx - i * p.g * kVec;
+        for (int idx = wtid; idx < npending * p.cols * kVec; idx += kWorkerThreads) {
+            const int i = idx / (p.cols * kVec), rem = idx - i * p.cols * kVec;
             const int head = rem / kVec, d4 = rem - head * kVec;
             const PendingRow r = info->pending[i];
             const long long u = static_cast<long long>(r.b) * p.Hkv + r.h;
             const RowRuns rr = row_runs(r.first, r.n, N, p.P);
-            const size_t row0 = static_cast<size_t>(r.b) * p.Hq + static_cast<size_t>(r.h) * p.g;
+            const size_t row = out_row(p, r.b, r.h, head);
             float lse;
-            const float4 v = merge_row_vec<D>(p.seg_out, p.seg_lse, p.g, static_cast<size_t>(rr.i0) + u,
+            const float4 v = merge_row_vec<D>(p.seg_out, p.seg_lse, p.cols, static_cast<size_t>(rr.i0) + u,
                                               rr.i1 - rr.i0 + 1, rr.i0, N, p.P, head, d4, &lse);
-            reinterpret_cast<float4 *>(p.out + (row0 + head) * D)[d4] = v;
-            if (d4 == 0) p.lse[row0 + head] = lse;
+            reinterpret_cast<float4 *>(p.out + row * D)[d4] = v;
+            if (d4 == 0) p.lse[row] = lse;
         }
         if (wtid < npending) {   // every segment of that row has arrived: reset for the next call
             const PendingRow r = info->pending[wtid];
@@ -865,8 +899,12 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         for (long long u = blockIdx.x; u < static_cast<long long>(p.B) * p.Hkv; u += p.P) {
             const int b = static_cast<int>(u / p.Hkv), h = static_cast<int>(u % p.Hkv);
             if (clamp_len(__ldg(p.seqlens + b), p.Lmax) != 0) continue;
-            const size_t row0 = static_cast<size_t>(b) * p.Hq + static_cast<size_t>(h) * p.g;
-            write_empty_row<D>(p.out + row0 * D, p.lse + row0, p.g, wtid, kWorkerThreads);
+            for (int idx = wtid; idx < p.cols * (D / 4); idx += kWorkerThreads) {
+                const int col = idx / (D / 4), d4 = idx - col * (D / 4);
+                const size_t row = out_row(p, b, h, col);
+                reinterpret_cast<float4 *>(p.out + row * D)[d4] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (d4 == 0) p.lse[row] = -INFINITY;
+            }
         }
     }
 }

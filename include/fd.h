@@ -135,6 +135,24 @@ FD_API int fd_decode_splits(int B, int Hq, int Hkv, int D, int max_len,
                      void *workspace, size_t workspace_bytes,
                      int num_splits, void *stream);
 
+/* Several queries per sequence (speculative decoding; the "flash decoding论文"
+ * page: with multi-turn dialogue or speculative decoding several query
+ * vectors are computed in parallel). q [B, q_len, Hq, D] bf16 (16-byte
+ * aligned), out [B, q_len, Hq, D] fp32, lse [B, q_len, Hq] fp32; caches as
+ * for fd_decode. seqlens[b] counts the cached tokens INCLUDING the q_len new
+ * ones, which are the last q_len positions; query j sees the first
+ * seqlens[b] - (q_len - 1 - j) tokens (causal among the new tokens; fewer
+ * than one gives out = 0, lse = -inf). Requires q_len * Hq / Hkv <= 16: the
+ * q_len x (Hq/Hkv) (query, head) pairs of a kv head are one small dense
+ * contraction, so every K/V byte is still read once. Workspace:
+ * fd_workspace_bytes(B, Hq * q_len, Hkv, D, max_len, num_splits);
+ * num_splits = 0 means fd_plan(B, Hq, Hkv, D, max_len). q_len = 1 is
+ * fd_decode_splits. */
+FD_API int fd_decode_multi(int B, int q_len, int Hq, int Hkv, int D, int max_len,
+                           const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                           const int32_t *seqlens, float scale, float *out, float *lse,
+                           void *workspace, size_t workspace_bytes, int num_splits, void *stream);
+
 /* fd_decode_splits over a PAGED key/value cache. The page pools
  * k_pages / v_pages hold num_pages pages of page_size tokens each, laid out
  * head-major (kv_layout = FD_KV_HND: [num_pages][Hkv][page_size][D] bf16) or

@@ -145,6 +145,21 @@ def test_paged_argument_errors_without_a_device():
         assert paged() == -8
 
 
+def test_multi_query_argument_errors_without_a_device():
+    L = fd.lib()
+    buf = (ctypes.c_uint8 * 4096)()
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 15) // 16 * 16)
+
+    def multi(q_len=2, Hq=4, Hkv=2, D=128, S=1, B=1):
+        return L.fd_decode_multi(B, q_len, Hq, Hkv, D, 64, p, p, p, p, 0.1, p, p, p, 4096, S, None)
+
+    assert multi(q_len=0) == -2 and multi(q_len=17) == -2
+    assert multi(q_len=9, Hq=4) == -3          # 9 queries x 2 heads per kv head > 16 columns
+    assert multi(q_len=3, Hq=3) == -3 and multi(D=96) == -4 and multi(S=-1) == -7
+    if not os.path.exists("/dev/nvidia0"):
+        assert multi() == -8 and multi(q_len=8) == -8
+
+
 def segments_rule(B, Hkv, Lmax, seqlens, P):
     """Independent statement of the documented partition: rows u = b*Hkv + j
     in order, ceil(L_b/64) tiles each, run i = flat tiles
