@@ -17,6 +17,16 @@ Recipe (for workload w and seed s):
 The same seed gives the same bytes on the same device type; a CPU draw and a
 CUDA draw of one seed differ (different generators), so each comparison
 draws once and hands the same bytes to both sides.
+
+Quantised caches (make_quant): seqlens and q as above; then per kv head h a
+spread factor f_h = 2^u, u ~ U(-1, 1), from a CPU generator seeded s + 1;
+scales k_scale[h] = 4 sigma_k f_h / R and v_scale[h] = 4 sigma_v f_h / R with
+R = 448 (E4M3) or 127 (int8), so +-4 standard deviations span the code range;
+K then V, one sequence at a time, fp32 randn * sigma * f_h, divided by the
+head's scale and turned into codes by torch's own conversion (E4M3: clamp to
++-448, then torch.float8_e4m3fn; int8: round half to even, clamp to +-127).
+Padding positions hold the NaN code 0x7F (E4M3) or -128 (int8, which has no
+NaN) when the workload pads.
 """
 from dataclasses import dataclass
 
@@ -130,3 +140,64 @@ def make_paged(x: DecodeInputs, page_size: int, layout: str = "HND", seed: int =
             part = part.permute(1, 0, 2, 3) if layout == "HND" else part.permute(1, 2, 0, 3)
             dst[torch.from_numpy(ids.astype(np.int64)).to(dev)] = part.contiguous()
     return PagedInputs(k_pages, v_pages, torch.from_numpy(table).to(dev), table, page_size, layout)
+
+QUANT_RANGE = {"e4m3": 448.0, "int8": 127.0}
+
+
+@dataclass
+class QuantInputs:
+    workload: Workload
+    seed: int
+    kv_type: str             # "e4m3" or "int8"
+    q: torch.Tensor          # [B, Hq, D] bf16
+    k8: torch.Tensor         # [B, Hkv, Lmax, D] uint8 codes
+    v8: torch.Tensor
+    k_scale: torch.Tensor    # [Hkv] float32, same device
+    v_scale: torch.Tensor
+    seqlens: torch.Tensor
+    seqlens_host: np.ndarray
+    scale: float
+
+    def kv_bytes(self) -> int:
+        """Bytes of K and V codes that lie inside the sequences."""
+        w = self.workload
+        return int(self.seqlens_host.astype(np.int64).sum()) * w.Hkv * w.D * 2
+
+
+def _codes(x: torch.Tensor, kv_type: str) -> torch.Tensor:
+    if kv_type == "e4m3":
+        return x.clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    return torch.round(x).clamp(-127.0, 127.0).to(torch.int8).view(torch.uint8)
+
+
+def make_quant(w: Workload, kv_type: str, seed: int = 0, device="cpu", seqlens=None) -> QuantInputs:
+    """Draw a workload with an 8-bit key/value cache (recipe in the module
+    docstring)."""
+    if kv_type not in QUANT_RANGE:
+        raise ValueError("kv_type must be 'e4m3' or 'int8'")
+    device = torch.device(device)
+    lens = draw_seqlens(w, seed) if seqlens is None else np.asarray(seqlens, dtype=np.int32).reshape(w.B)
+    g = torch.Generator(device=device).manual_seed(int(seed))
+    q = (torch.randn((w.B, w.Hq, w.D), generator=g, device=device) * w.sigma_q).to(torch.bfloat16)
+    gh = torch.Generator(device="cpu").manual_seed(int(seed) + 1)
+    f = torch.pow(2.0, torch.rand((w.Hkv,), generator=gh) * 2.0 - 1.0)
+    R = QUANT_RANGE[kv_type]
+    k_scale = (4.0 * w.sigma_k * f / R).to(torch.float32)
+    v_scale = (4.0 * w.sigma_v * f / R).to(torch.float32)
+    k8 = torch.empty((w.B, w.Hkv, w.Lmax, w.D), dtype=torch.uint8, device=device)
+    v8 = torch.empty_like(k8)
+    for dst, sigma, sc in ((k8, w.sigma_k, k_scale), (v8, w.sigma_v, v_scale)):
+        spread = (f * sigma).to(device)[:, None, None]
+        inv = (1.0 / sc).to(device)[:, None, None]
+        for b in range(w.B):
+            x = torch.randn((w.Hkv, w.Lmax, w.D), generator=g, device=device) * spread
+            dst[b] = _codes(x * inv, kv_type)
+    if w.nan_pad:
+        pad = 0x7F if kv_type == "e4m3" else 0x80
+        for b in range(w.B):
+            L = int(lens[b])
+            if L < w.Lmax:
+                k8[b, :, max(L, 0):, :] = pad
+                v8[b, :, max(L, 0):, :] = pad
+    return QuantInputs(w, int(seed), kv_type, q, k8, v8, k_scale.to(device), v_scale.to(device),
+                       torch.from_numpy(lens.copy()).to(device), lens.copy(), w.scale)

@@ -10,7 +10,8 @@ softmax(scale * q K^T) V over the cached tokens of each row, plus the
 log-sum-exp of the logits; section "A faster attention for decoding:
 Flash-Decoding" gives the split / per-split log-sum-exp / rescaled reduction
 steps that reach the same result. Inputs are bf16 bit patterns (numpy uint16);
-outputs are float64.
+outputs are float64. ``attention_quant`` reads a cache of 8-bit codes (OCP
+E4M3 or int8) dequantised with one scale per key/value head.
 """
 import ctypes
 
@@ -22,6 +23,10 @@ _u16p = np.ctypeslib.ndpointer(dtype=np.uint16, flags="C_CONTIGUOUS")
 _i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
 _f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
 _f64p_or_null = ctypes.c_void_p
+_u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
+_f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
+
+KV_TYPES = {"e4m3": 1, "int8": 2}   # codes of fdo_attention_quant's kv_type
 
 
 class Oracle:
@@ -42,6 +47,9 @@ class Oracle:
         lib.fdo_attention_multi.restype = ctypes.c_int
         lib.fdo_attention_multi.argtypes = [ctypes.c_int] * 6 + [_u16p, _u16p, _u16p, _i32p, ctypes.c_double,
                                                                  _f64p, _f64p, ctypes.c_int]
+        lib.fdo_attention_quant.restype = ctypes.c_int
+        lib.fdo_attention_quant.argtypes = ([ctypes.c_int] * 7 + [_u16p, _u8p, _u8p, _f32p, _f32p, _i32p,
+                                                                  ctypes.c_double, _f64p, _f64p, ctypes.c_int])
         lib.fdo_combine.restype = ctypes.c_int
         lib.fdo_combine.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _f64p, _f64p, _f64p, _f64p]
         lib.fdo_mutant.restype = ctypes.c_int
@@ -99,6 +107,33 @@ class Oracle:
             raise RuntimeError(f"fdo_attention_multi failed ({rc})")
         self.threads_used = rc
         return out, lse
+
+    def attention_quant(self, q, k8, v8, k_scale, v_scale, seqlens, scale, kv_type, nthreads=0):
+        """Attention over a quantised cache. q [B,Hq,D] or [B,q_len,Hq,D] bf16
+        bits; k8/v8 [B,Hkv,Lmax,D] uint8 codes; k_scale/v_scale [Hkv] float32;
+        kv_type "e4m3" or "int8". Returns (out, lse) shaped like q (without D
+        for lse), float64."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        single = q.ndim == 3
+        if single:
+            q = q[:, None]
+        k8 = np.ascontiguousarray(k8, dtype=np.uint8)
+        v8 = np.ascontiguousarray(v8, dtype=np.uint8)
+        ks = np.ascontiguousarray(k_scale, dtype=np.float32)
+        vs = np.ascontiguousarray(v_scale, dtype=np.float32)
+        seqlens = np.ascontiguousarray(seqlens, dtype=np.int32)
+        B, q_len, Hq, D = q.shape
+        _, Hkv, Lmax, _ = k8.shape
+        if k8.shape != v8.shape or ks.shape != (Hkv,) or vs.shape != (Hkv,):
+            raise ValueError("cache or scale shapes disagree")
+        out = np.zeros((B, q_len, Hq, D), np.float64)
+        lse = np.zeros((B, q_len, Hq), np.float64)
+        rc = self.lib.fdo_attention_quant(B, q_len, Hq, Hkv, D, Lmax, KV_TYPES[kv_type], q, k8, v8, ks, vs, seqlens,
+                                          float(scale), out, lse, int(nthreads))
+        if rc <= 0:
+            raise RuntimeError(f"fdo_attention_quant failed ({rc})")
+        self.threads_used = rc
+        return (out[:, 0], lse[:, 0]) if single else (out, lse)
 
     def split_attention(self, q, k, v, seqlens, scale, bounds, nthreads=0, want_parts=False):
         """Split-then-reduce form with token boundaries ``bounds`` (nsplit+1
@@ -159,6 +194,10 @@ def attention_multi(q, k, v, seqlens, scale, nthreads=0):
     return default().attention_multi(q, k, v, seqlens, scale, nthreads)
 
 
+def attention_quant(q, k8, v8, k_scale, v_scale, seqlens, scale, kv_type, nthreads=0):
+    return default().attention_quant(q, k8, v8, k_scale, v_scale, seqlens, scale, kv_type, nthreads)
+
+
 LIBRARY = _build.LIBRARY
 SOURCE = _build.SOURCE
-__all__ = ["Oracle", "default", "attention", "attention_multi", "split_attention", "combine", "LIBRARY", "SOURCE"]
+__all__ = ["Oracle", "default", "attention", "attention_multi", "attention_quant", "KV_TYPES", "split_attention", "combine", "LIBRARY", "SOURCE"]

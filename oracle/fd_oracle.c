@@ -45,6 +45,17 @@
  *  - seqlens[b] is clamped to [0, Lmax]; positions t >= seqlens[b] are never
  *    read, so whatever fills them (NaN in the ragged workload) cannot matter.
  *
+ *  - Quantised key/value cache (the "flash decoding论文" page lists INT8/INT4
+ *    quantisation among PaddleNLP's inference techniques). Reading taken:
+ *    each cached byte is a code, dequantised with one scale per key/value
+ *    head, k = k_scale[j] * decode(code), v = v_scale[j] * decode(code);
+ *    the attention is then the definition above over those values.
+ *    decode() is either 8-bit two's complement (int8) or the OCP 8-bit
+ *    floating-point format E4M3 (1 sign bit, 4 exponent bits with bias 7,
+ *    3 mantissa bits; exponent field 0 is subnormal, (m/8) * 2^-6; the one
+ *    code S.1111.111 is NaN; no infinities), written out from its fields.
+ *    fdo_attention_quant() is that, with any number of queries per sequence.
+ *
  * Precision: inputs are bf16 bit patterns decoded exactly to double; all
  * arithmetic is IEEE double with the C library's exp() and log(). Rows are
  * independent, so they are spread over POSIX threads; each row is computed
@@ -72,9 +83,40 @@ static double bf16_to_double(uint16_t h) {
     return (double)f;
 }
 
+/* OCP E4M3 code -> value, from its bit fields. */
+static double e4m3_to_double(uint8_t c) {
+    const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+#if FDO_MUTANT == 9
+    mag = ldexp(1.0 + m / 8.0, e - 7);             /* planted: subnormals read as normals */
+#else
+    if (e == 0)
+        mag = ldexp(m / 8.0, -6);
+    else
+        mag = ldexp(1.0 + m / 8.0, e - 7);
+#endif
+    return s ? -mag : mag;
+}
+
+/* int8 code -> value (two's complement). */
+static double int8_to_double(uint8_t c) {
+#if FDO_MUTANT == 11
+    return (double)c;                              /* planted: read as unsigned */
+#else
+    return c < 128 ? (double)c : (double)c - 256.0;
+#endif
+}
+
+enum { FDO_KV_BF16 = 0, FDO_KV_E4M3 = 1, FDO_KV_INT8 = 2 };
+
 typedef struct {
     int B, Hq, Hkv, D, Lmax;
     const uint16_t *q, *k, *v;
+    /* quantised cache (kv_type != FDO_KV_BF16): codes and per-kv-head scales */
+    int kv_type;
+    const uint8_t *k8, *v8;
+    const float *k_scale, *v_scale;
     const int32_t *seqlens;
     double scale;
     double *out, *lse;
@@ -88,6 +130,30 @@ typedef struct {
     /* thread partition */
     int nthreads, tid;
 } job_t;
+
+static double code_value(int kv_type, uint8_t c) {
+    return kv_type == FDO_KV_E4M3 ? e4m3_to_double(c) : int8_to_double(c);
+}
+
+/* Element idx of the key cache [B,Hkv,Lmax,D], whose kv head is j. */
+static double key_at(const job_t *J, size_t idx, int j) {
+    if (J->kv_type == FDO_KV_BF16) return bf16_to_double(J->k[idx]);
+    return (double)J->k_scale[j] * code_value(J->kv_type, J->k8[idx]);
+}
+
+/* Element idx of the value cache, whose kv head is j. */
+static double value_at(const job_t *J, size_t idx, int j) {
+#if FDO_MUTANT == 5
+    return key_at(J, idx, j);                      /* planted: keys as values */
+#else
+    if (J->kv_type == FDO_KV_BF16) return bf16_to_double(J->v[idx]);
+#if FDO_MUTANT == 10
+    return (double)J->k_scale[j] * code_value(J->kv_type, J->v8[idx]);   /* planted: key scale on values */
+#else
+    return (double)J->v_scale[j] * code_value(J->kv_type, J->v8[idx]);
+#endif
+#endif
+}
 
 static int clamp_len(int L, int Lmax) {
     if (L < 0) return 0;
@@ -104,9 +170,9 @@ static void row_logits(const job_t *J, int b, int i, const uint16_t *qrow, int t
     const int j = i / g;
 #endif
     for (int t = t0; t < t1; ++t) {
-        const uint16_t *krow = J->k + (((size_t)b * J->Hkv + j) * J->Lmax + t) * J->D;
+        const size_t krow = (((size_t)b * J->Hkv + j) * J->Lmax + t) * J->D;
         double dot = 0.0;
-        for (int d = 0; d < J->D; ++d) dot += bf16_to_double(qrow[d]) * bf16_to_double(krow[d]);
+        for (int d = 0; d < J->D; ++d) dot += bf16_to_double(qrow[d]) * key_at(J, krow + d, j);
 #if FDO_MUTANT == 1
         z[t - t0] = dot;                           /* planted: scale dropped */
 #else
@@ -133,12 +199,8 @@ static double row_softmax_sum(const job_t *J, int b, int i, int t0, int t1,
     for (int t = 0; t < t1 - t0; ++t) Z += exp(z[t] - M);
     for (int t = t0; t < t1; ++t) {
         const double w = exp(z[t - t0] - M);
-#if FDO_MUTANT == 5
-        const uint16_t *vrow = J->k + (((size_t)b * J->Hkv + j) * J->Lmax + t) * J->D;  /* planted: keys as values */
-#else
-        const uint16_t *vrow = J->v + (((size_t)b * J->Hkv + j) * J->Lmax + t) * J->D;
-#endif
-        for (int d = 0; d < J->D; ++d) o[d] += w * bf16_to_double(vrow[d]);
+        const size_t vrow = (((size_t)b * J->Hkv + j) * J->Lmax + t) * J->D;
+        for (int d = 0; d < J->D; ++d) o[d] += w * value_at(J, vrow + d, j);
     }
 #if FDO_MUTANT != 6
     for (int d = 0; d < J->D; ++d) o[d] /= Z;       /* mutant 6 plants: no normalisation */
@@ -321,6 +383,27 @@ int fdo_attention_multi(int B, int q_len, int Hq, int Hkv, int D, int Lmax,
     memset(&J, 0, sizeof J);
     J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.Lmax = Lmax;
     J.q = q; J.k = k; J.v = v; J.seqlens = seqlens; J.scale = scale;
+    J.out = out; J.lse = lse; J.q_len = q_len;
+    return run_threads_rows(&J, multi_worker, nthreads, B * q_len * Hq);
+}
+
+/* Quantised cache: k8/v8 [B,Hkv,Lmax,D] codes (kv_type 1 = E4M3, 2 = int8),
+ * k_scale/v_scale [Hkv]; q [B,q_len,Hq,D] bf16 bits; out [B,q_len,Hq,D],
+ * lse [B,q_len,Hq]. Query j sees t < seqlens[b] - (q_len - 1 - j), as in
+ * fdo_attention_multi. Returns threads used or a negative value. */
+int fdo_attention_quant(int B, int q_len, int Hq, int Hkv, int D, int Lmax, int kv_type,
+                        const uint16_t *q, const uint8_t *k8, const uint8_t *v8,
+                        const float *k_scale, const float *v_scale,
+                        const int32_t *seqlens, double scale,
+                        double *out, double *lse, int nthreads) {
+    if (check_shape(B, Hq, Hkv, D, Lmax) || q_len < 1) return -1;
+    if (kv_type != FDO_KV_E4M3 && kv_type != FDO_KV_INT8) return -1;
+    if (B == 0) return 1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.Lmax = Lmax;
+    J.q = q; J.kv_type = kv_type; J.k8 = k8; J.v8 = v8; J.k_scale = k_scale; J.v_scale = v_scale;
+    J.seqlens = seqlens; J.scale = scale;
     J.out = out; J.lse = lse; J.q_len = q_len;
     return run_threads_rows(&J, multi_worker, nthreads, B * q_len * Hq);
 }

@@ -331,6 +331,119 @@ def pin_multi_query_library_mask(orc):
         close(out[b], ref[0].permute(1, 0, 2).numpy(), 1e-12, "multi-query sdpa out")
 
 
+# ----------------------------------------------- quantised key/value cache --
+
+def one_key_codes(orc, kv_type, codes, v_scale):
+    """A row with one cached token whose value holds `codes`: the softmax
+    weight is 1, so out = v_scale * decode(code) for each element."""
+    D = len(codes)
+    q = to_bits(np.full((1, 1, D), 0.5))
+    k8 = np.full((1, 1, 1, D), 0x38 if kv_type == "e4m3" else 1, np.uint8)
+    v8 = np.asarray(codes, np.uint8).reshape(1, 1, 1, D)
+    out, lse = orc.attention_quant(q, k8, v8, np.array([0.25], np.float32), np.array([v_scale], np.float32),
+                                   np.array([1], np.int32), 0.5, kv_type)
+    return out[0, 0], lse[0, 0]
+
+
+def pin_e4m3_codes(orc):
+    """Every E4M3 code against torch's float8_e4m3fn conversion (library),
+    plus values fixed by the format's definition: 0x38 = 1, 0x7E = 448 (the
+    largest), 0x08 = 2^-6 (smallest normal), 0x01 = 2^-9 (smallest
+    subnormal), 0x80 = -0, 0x7F = NaN."""
+    codes = np.arange(256, dtype=np.uint8)
+    out, lse = one_key_codes(orc, "e4m3", codes, 1.0)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    if not np.array_equal(np.isnan(out), np.isnan(ref)):
+        raise AssertionError("e4m3: NaN codes differ from torch")
+    close(out[~np.isnan(ref)], ref[~np.isnan(ref)], 0.0, "e4m3 code values vs torch")
+    for c, val in ((0x38, 1.0), (0x7E, 448.0), (0x08, 2.0 ** -6), (0x01, 2.0 ** -9), (0xB8, -1.0), (0x80, 0.0)):
+        close(out[c], val, 0.0, f"e4m3 code {c:#04x}")
+    if not (np.isnan(out[0x7F]) and np.isnan(out[0xFF])):
+        raise AssertionError("e4m3: 0x7F / 0xFF must be NaN")
+    # one key of all-ones codes (k = 0.25 each): lse = 0.5 * 0.25 * 0.5 * D
+    close(lse, 0.5 * 0.25 * 0.5 * 256, 1e-12, "e4m3 one-key lse")
+
+
+def pin_int8_codes(orc):
+    """Every int8 code is its two's-complement value times the head's scale."""
+    codes = np.arange(256, dtype=np.uint8)
+    out, _ = one_key_codes(orc, "int8", codes, 0.5)
+    close(out, codes.view(np.int8).astype(np.float64) * 0.5, 0.0, "int8 codes")
+
+
+def quant_case(rng, kv_type, B, q_len, Hq, Hkv, D, Lmax):
+    """Random codes (no NaN codes) and distinct per-head scales."""
+    q = to_bits(rng.standard_normal((B, q_len, Hq, D)))
+    if kv_type == "e4m3":
+        pool = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+        k8, v8 = (rng.choice(pool, (B, Hkv, Lmax, D)) for _ in range(2))
+    else:
+        k8, v8 = (rng.integers(0, 256, (B, Hkv, Lmax, D)).astype(np.uint8) for _ in range(2))
+    ks = (rng.uniform(0.5, 2.0, Hkv) * (0.02 if kv_type == "e4m3" else 0.03)).astype(np.float32)
+    vs = (rng.uniform(0.5, 2.0, Hkv) * (0.05 if kv_type == "e4m3" else 0.04)).astype(np.float32)
+    return q, k8, v8, ks, vs
+
+
+def dequant_torch(codes, scales, kv_type):
+    t = torch.from_numpy(np.ascontiguousarray(codes))
+    vals = t.view(torch.float8_e4m3fn).to(torch.float64) if kv_type == "e4m3" else t.view(torch.int8).to(torch.float64)
+    return vals * torch.from_numpy(scales.astype(np.float64))[None, :, None, None]
+
+
+def pin_quant_library_sdpa(orc):
+    """Quantised cache against torch scaled_dot_product_attention (float64)
+    over the cache dequantised by torch's own conversions, with grouped heads,
+    ragged lengths and several queries (causal-offset mask)."""
+    rng = np.random.default_rng(91)
+    for kv_type in ("e4m3", "int8"):
+        B, q_len, Hq, Hkv, D, Lmax = 3, 2, 6, 2, 16, 40
+        q, k8, v8, ks, vs = quant_case(rng, kv_type, B, q_len, Hq, Hkv, D, Lmax)
+        seq = np.array([40, 17, 1], np.int32)
+        out, lse = orc.attention_quant(q, k8, v8, ks, vs, seq, 0.25, kv_type)
+        qf = torch.from_numpy(bits_to_f64(q))
+        kf, vf = dequant_torch(k8, ks, kv_type), dequant_torch(v8, vs, kv_type)
+        for b in range(B):
+            L = int(seq[b])
+            mask = torch.zeros((q_len, L), dtype=torch.bool)
+            for j in range(q_len):
+                mask[j, :max(0, L - (q_len - 1 - j))] = True
+            qb = qf[b].permute(1, 0, 2)                                   # [Hq, q_len, D]
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                qb[None], kf[b, :, :L][None], vf[b, :, :L][None], attn_mask=mask, scale=0.25, enable_gqa=True)
+            z = 0.25 * torch.einsum("hqd,htd->hqt", qb, kf[b, :, :L].repeat_interleave(Hq // Hkv, 0))
+            ref_lse = torch.logsumexp(z.masked_fill(~mask[None], -math.inf), dim=-1)   # [Hq, q_len]
+            for j in range(q_len):
+                if mask[j].any():
+                    close(out[b, j], ref[0, :, j].numpy(), 1e-12, f"{kv_type} sdpa out b={b} j={j}")
+                    close(lse[b, j], ref_lse[:, j].numpy(), 1e-12, f"{kv_type} lse b={b} j={j}")
+                else:
+                    close(out[b, j], 0.0, 0.0, f"{kv_type} empty query out")
+                    if not np.all(np.isneginf(lse[b, j])):
+                        raise AssertionError(f"{kv_type}: a query that sees no token must have lse = -inf")
+
+
+def pin_quant_scales(orc):
+    """Scale laws: multiplying every k_scale by c is multiplying the softmax
+    scale by c; multiplying v_scale[h] by c multiplies the outputs of that
+    head's group by c and leaves every lse and the other heads unchanged."""
+    rng = np.random.default_rng(92)
+    for kv_type in ("e4m3", "int8"):
+        B, Hq, Hkv, D, Lmax = 2, 4, 2, 8, 25
+        q, k8, v8, ks, vs = quant_case(rng, kv_type, B, 1, Hq, Hkv, D, Lmax)
+        seq = np.array([25, 9], np.int32)
+        o1, l1 = orc.attention_quant(q, k8, v8, ks * np.float32(2.0), vs, seq, 0.3, kv_type)
+        o2, l2 = orc.attention_quant(q, k8, v8, ks, vs, seq, 0.6, kv_type)
+        close(o1, o2, 1e-13, f"{kv_type}: k_scale*2 vs scale*2 out")
+        close(l1, l2, 1e-12, f"{kv_type}: k_scale*2 vs scale*2 lse")
+        vs2 = vs.copy()
+        vs2[1] *= np.float32(4.0)
+        o3, l3 = orc.attention_quant(q, k8, v8, ks, vs, seq, 0.3, kv_type)
+        o4, l4 = orc.attention_quant(q, k8, v8, ks, vs2, seq, 0.3, kv_type)
+        close(l3, l4, 0.0, f"{kv_type}: v_scale must not move lse")
+        close(o4[:, :, :2], o3[:, :, :2], 0.0, f"{kv_type}: v_scale of head 1 moved head 0's group")
+        close(o4[:, :, 2:], 4.0 * o3[:, :, 2:], 1e-13, f"{kv_type}: v_scale of head 1")
+
+
 ALL_PINS = [
     pin_brute_force_decimal,
     pin_worked_examples,
@@ -343,4 +456,8 @@ ALL_PINS = [
     pin_group_mapping,
     pin_multi_query_decimal,
     pin_multi_query_library_mask,
+    pin_e4m3_codes,
+    pin_int8_codes,
+    pin_quant_library_sdpa,
+    pin_quant_scales,
 ]

@@ -1,6 +1,7 @@
 """The seeded input generator: determinism, the ragged-length recipe, NaN
 padding and bf16 rounding (CPU only)."""
 import numpy as np
+import pytest
 import torch
 
 from decode_attention_07_b200.configs import WORKLOADS, ORDER
@@ -47,3 +48,33 @@ def test_sigma_and_rounding():
     g = torch.Generator().manual_seed(1)
     q32 = torch.randn((w.B, w.Hq, w.D), generator=g)
     assert torch.equal(q32.to(torch.bfloat16), x.q)
+
+
+# ------------------------------------------------------ quantised caches --
+
+from decode_attention_07_b200.inputs import QUANT_RANGE, make_quant  # noqa: E402
+
+
+@pytest.mark.parametrize("kv_type", ["e4m3", "int8"])
+def test_quant_inputs_recipe(kv_type):
+    w = WORKLOADS["ragged_64k"].with_(B=3, Lmax=200)
+    a = make_quant(w, kv_type, seed=5)
+    b = make_quant(w, kv_type, seed=5)
+    assert torch.equal(a.k8, b.k8) and torch.equal(a.v8, b.v8) and torch.equal(a.q, b.q)
+    assert a.k8.dtype == torch.uint8 and a.k8.shape == (w.B, w.Hkv, w.Lmax, w.D)
+    assert a.k_scale.shape == (w.Hkv,) and a.k_scale.dtype == torch.float32
+    # per-head spread f_h in [1/2, 2]: k_scale / (4 sigma_k / R) is that factor, the same for v
+    f_k = a.k_scale.double() / (4 * w.sigma_k / QUANT_RANGE[kv_type])
+    f_v = a.v_scale.double() / (4 * w.sigma_v / QUANT_RANGE[kv_type])
+    assert torch.allclose(f_k, f_v, rtol=1e-6) and bool((f_k >= 0.5).all() and (f_k <= 2.0).all())
+    pad = 0x7F if kv_type == "e4m3" else 0x80
+    for bb in range(w.B):
+        L = int(a.seqlens_host[bb])
+        assert bool((a.k8[bb, :, L:] == pad).all() and (a.v8[bb, :, L:] == pad).all())
+        # inside the sequence: dequantised values have the head's sigma * f_h spread
+        vals = (a.k8[bb, :, :L].view(torch.float8_e4m3fn).float() if kv_type == "e4m3"
+                else a.k8[bb, :, :L].view(torch.int8).float())
+        if L >= 100:
+            sd = (vals * a.k_scale[:, None, None]).std(dim=(1, 2)) / (w.sigma_k * f_k.float())
+            assert bool(((sd > 0.8) & (sd < 1.2)).all())
+    assert make_quant(w, kv_type, seed=6).k8.ne(a.k8).any()

@@ -1,7 +1,7 @@
 """Each planted mistake in the oracle (FDO_MUTANT in fd_oracle.c) must be
 caught by at least one pin: this shows the pins constrain every step of the
 oracle (scale, group mapping, sequence length, log base, value operand,
-normalisation, split reduction)."""
+normalisation, split reduction, causal offset, dequantisation)."""
 import pytest
 
 import oracle
@@ -17,6 +17,9 @@ MUTANTS = {
     6: "softmax weights not normalised",
     7: "split weights not rescaled by the total log-sum-exp",
     8: "each of several queries sees one token too few",
+    9: "E4M3 subnormal codes decoded as normals",
+    10: "values dequantised with the key scale",
+    11: "int8 codes read as unsigned",
 }
 
 
