@@ -133,12 +133,12 @@ class ClockSampler:
 
 # ------------------------------------------------------------ byte counts --
 
-def byte_counts(w, lens, S, q_len=1):
+def byte_counts(w, lens, S, q_len=1, elem_bytes=2):
     """Algorithmic bytes of one call: K/V inside the sequences, q, and the
     outputs / workspace segments each stage writes and reads (q_len queries
     per sequence: q_len times the query and output bytes)."""
     lens = np.clip(lens.astype(np.int64), 0, w.Lmax)
-    kv = int(lens.sum()) * w.Hkv * w.D * 2 * 2
+    kv = int(lens.sum()) * w.Hkv * w.D * elem_bytes * 2
     q = w.B * q_len * w.Hq * w.D * 2
     seg = fd.fd_segments(w.B, w.Hkv, w.Lmax, lens.astype(np.int32), S)
     used = seg["row"] >= 0
@@ -164,6 +164,8 @@ def oracle_sample(x, budget_s=12.0, nthreads=0):
     import oracle
     w = x.workload
     orc = oracle.default()
+    quant = hasattr(x, "k8")
+    elem = 1 if quant else 2
     order = np.argsort(-x.seqlens_host, kind="stable")
     done_bytes, spent, rows, threads = 0, 0.0, 0, 0
     for b in order:
@@ -175,20 +177,28 @@ def oracle_sample(x, budget_s=12.0, nthreads=0):
         for j0 in range(0, w.Hkv, step):
             j1 = min(w.Hkv, j0 + step)
             qh = bf16_bits(x.q[b:b + 1, j0 * w.g:j1 * w.g])
-            kh = bf16_bits(x.k[b:b + 1, j0:j1, :L])
-            vh = bf16_bits(x.v[b:b + 1, j0:j1, :L])
-            t0 = time.perf_counter()
-            orc.attention(qh, kh, vh, np.array([L], np.int32), x.scale, nthreads)
+            if quant:
+                kh = x.k8[b:b + 1, j0:j1, :L].cpu().numpy()
+                vh = x.v8[b:b + 1, j0:j1, :L].cpu().numpy()
+                ks, vs = x.k_scale[j0:j1].cpu().numpy(), x.v_scale[j0:j1].cpu().numpy()
+                t0 = time.perf_counter()
+                orc.attention_quant(qh, kh, vh, ks, vs, np.array([L], np.int32), x.scale, x.kv_type, nthreads)
+            else:
+                kh = bf16_bits(x.k[b:b + 1, j0:j1, :L])
+                vh = bf16_bits(x.v[b:b + 1, j0:j1, :L])
+                t0 = time.perf_counter()
+                orc.attention(qh, kh, vh, np.array([L], np.int32), x.scale, nthreads)
             spent += time.perf_counter() - t0
             threads = max(threads, orc.threads_used)
-            done_bytes += (j1 - j0) * L * w.D * 2 * 2
+            done_bytes += (j1 - j0) * L * w.D * elem * 2
             rows += j1 - j0
             if spent >= budget_s:
                 break
         if spent >= budget_s:
             break
-    desc = (f"{rows} (sequence, kv-head) rows x {w.g} query heads of {w.name} seed {x.seed}, "
-            f"longest sequences first; KV bytes of the sample / oracle seconds")
+    desc = (f"{rows} (sequence, kv-head) rows x {w.g} query heads of {w.name} seed {x.seed}"
+            f"{' (' + x.kv_type + ' cache)' if quant else ''}, longest sequences first; "
+            f"KV bytes of the sample / oracle seconds")
     return done_bytes, spent, threads, desc
 
 
@@ -252,7 +262,15 @@ def run_fd(args, w, rank, world):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.Lmax)
-    xs = [make_inputs(w, rank_seed(args.seed, rank), device=dev)]
+    quant = args.kv != "bf16"
+
+    def draw(seed):
+        if quant:
+            from decode_attention_07_b200.inputs import make_quant
+            return make_quant(w, args.kv, seed, device=dev)
+        return make_inputs(w, seed, device=dev)
+
+    xs = [draw(rank_seed(args.seed, rank))]
     kv_per_copy = xs[0].kv_bytes()
     if kv_per_copy >= L2_BYTES:
         # rotate input copies so every call streams bytes that are not in L2
@@ -262,7 +280,7 @@ def run_fd(args, w, rank, world):
         n_copies = 1
         l2_note = "L2 flushed before every timed call (256 MiB write outside the timed events)"
     for c in range(1, n_copies):
-        xs.append(make_inputs(w, rank_seed(args.seed, rank) + 1000 * c, device=dev))
+        xs.append(draw(rank_seed(args.seed, rank) + 1000 * c))
     Q = args.q_len
     nbytes = fd.fd_workspace_bytes(w.B, w.Hq * Q, w.Hkv, w.D, w.Lmax, S)
     ws = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=dev)      # row counters start at zero
@@ -275,7 +293,7 @@ def run_fd(args, w, rank, world):
             g = torch.Generator(device=dev).manual_seed(rank_seed(args.seed, rank) + 77 + i)
             x.q = (torch.randn((w.B, Q, w.Hq, w.D), generator=g, device=dev) * w.sigma_q).to(torch.bfloat16)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if n_copies == 1 else None
-    counts = byte_counts(w, xs[0].seqlens_host, S, Q)
+    counts = byte_counts(w, xs[0].seqlens_host, S, Q, 1 if quant else 2)
     kv_bytes = sum(x.kv_bytes() for x in xs) / n_copies
     if args.paged:
         # the same logical caches, scattered into shuffled page pools
@@ -286,6 +304,9 @@ def run_fd(args, w, rank, world):
         torch.cuda.empty_cache()
         calls = [fd.prepare_decode_paged(x.q, pg.k_pages, pg.v_pages, pg.block_table, x.seqlens, x.scale, out, lse,
                                          ws, args.layout, S, stream) for x, pg in zip(xs, pgs)]
+    elif quant:
+        calls = [fd.prepare_decode_quant(x.q, x.k8, x.v8, x.k_scale, x.v_scale, args.kv, x.seqlens, x.scale, out, lse,
+                                         ws, S, stream) for x in xs]
     elif Q > 1:
         calls = [fd.prepare_decode_multi(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream) for x in xs]
     else:
@@ -336,7 +357,8 @@ def run_fd(args, w, rank, world):
 
     # ---- the two stages as separate kernels (for the per-stage split) ------
     ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-             torch.cuda.Event(enable_timing=True)) for _ in range(args.steps if not args.paged and Q == 1 else 0)]
+             torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps if not args.paged and Q == 1 and not quant else 0)]
     for i in range(len(ev_s)):
         x = xs[i % n_copies]
         if flush is not None:
@@ -354,12 +376,16 @@ def run_fd(args, w, rank, world):
     e2e = None
     if not args.no_e2e and not args.paged:
         x = xs[0]
-        hq, hk, hv = x.q.cpu().pin_memory(), x.k.cpu().pin_memory(), x.v.cpu().pin_memory()
+        kc, vc = (x.k8, x.v8) if quant else (x.k, x.v)
+        hq, hk, hv = x.q.cpu().pin_memory(), kc.cpu().pin_memory(), vc.cpu().pin_memory()
         hs = x.seqlens.cpu().pin_memory()
-        dq, dk, dv, dsq = (torch.empty_like(t) for t in (x.q, x.k, x.v, x.seqlens))
+        dq, dk, dv, dsq = (torch.empty_like(t) for t in (x.q, kc, vc, x.seqlens))
+        if quant:   # the per-head scales travel with the cache
+            hks, hvs = x.k_scale.cpu().pin_memory(), x.v_scale.cpu().pin_memory()
+            dks, dvs = torch.empty_like(x.k_scale), torch.empty_like(x.v_scale)
         ho = torch.empty(tuple(out.shape), dtype=torch.float32).pin_memory()
         hl = torch.empty(tuple(lse.shape), dtype=torch.float32).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs))
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs) + ((hks, hvs) if quant else ()))
         d2h = ho.numel() * 4 + hl.numel() * 4
         e_steps = max(3, min(args.steps, 20))
 
@@ -368,7 +394,11 @@ def run_fd(args, w, rank, world):
             dk.copy_(hk, non_blocking=True)
             dv.copy_(hv, non_blocking=True)
             dsq.copy_(hs, non_blocking=True)
-            if Q > 1:
+            if quant:
+                dks.copy_(hks, non_blocking=True)
+                dvs.copy_(hvs, non_blocking=True)
+                fd.fd_decode_quant(dq, dk, dv, dks, dvs, args.kv, dsq, x.scale, out, lse, ws, S, stream)
+            elif Q > 1:
                 fd.fd_decode_multi(dq, dk, dv, dsq, x.scale, out, lse, ws, S, stream)
             else:
                 fd.fd_decode_splits(dq, dk, dv, dsq, x.scale, out, lse, ws, S, stream)
@@ -400,15 +430,17 @@ def run_fd(args, w, rank, world):
     line = {
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_max / args.steps, "us_per_call": us_per_call,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(config_dict(w, S, l2_note), **({"paged": {"page_size": args.paged, "layout": args.layout}}
-                                                      if args.paged else {}), **({"q_len": Q} if Q > 1 else {})),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": args.kv, "data": "synthetic",
+        "config": dict(config_dict(w, S, l2_note), **({"kv_cache": args.kv} if quant else {}),
+                       **({"paged": {"page_size": args.paged, "layout": args.layout}} if args.paged else {}),
+                       **({"q_len": Q} if Q > 1 else {})),
         "pct_of_nominal_hbm": 100.0 * gbs / world / NOMINAL_HBM_GBS,
         "pct_of_measured_copy": 100.0 * gbs / world / peak,
         "call_bytes_gbs": world * counts["total"] * args.steps / (ms_max * 1e-3) / 1e9,
-        "roofline": {"kernel": "fd_split_kernel (fused combine)", "bound": "hbm", "achieved": kernel_gbs,
+        "roofline": {"kernel": "fd_split_kernel (fused combine)" + (f", {args.kv} cache" if quant else ""), "bound": "hbm", "achieved": kernel_gbs,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": kernel_gbs / peak,
-                     "traffic": None if args.paged or Q > 1 else measured_traffic(w.name), "bytes_per_launch": counts["total"],
+                     "traffic": None if args.paged or Q > 1 or quant else measured_traffic(w.name),
+                     "bytes_per_launch": counts["total"],
                      "us_per_launch": us_per_call,
                      "frac_of_nominal_8tbs": kernel_gbs / NOMINAL_HBM_GBS},
         "stages_alone": {"split_us": split_us, "combine_us": combine_us},
@@ -417,7 +449,7 @@ def run_fd(args, w, rank, world):
         "e2e": e2e,
         "wall_s": wall,
     }
-    if world == 1 and not args.no_cpu_baseline and not args.paged and Q == 1:
+    if world == 1 and not args.no_cpu_baseline and not args.paged and Q == 1:   # bf16 or 8-bit cache
         b, s, t, desc = oracle_sample(xs[0], budget_s=args.cpu_seconds)
         line["cpu_baseline"] = {"value": b / s / 1e9, "unit": "GB/s", "cores": t, "kind": "oracle",
                                 "sample": desc, "seconds": s}
@@ -439,11 +471,15 @@ def main():
     ap.add_argument("--paged", type=int, default=0, metavar="PAGE_SIZE",
                     help="read the caches from a shuffled page pool with this page size (fd_decode_paged)")
     ap.add_argument("--layout", choices=["HND", "NHD"], default="HND", help="page layout for --paged")
+    ap.add_argument("--kv", choices=["bf16", "e4m3", "int8"], default="bf16",
+                    help="key/value cache element type; e4m3 / int8 use fd_decode_quant with per-head scales")
     ap.add_argument("--q-len", type=int, default=1,
                     help="new tokens per sequence, each a query seeing the cache up to itself (fd_decode_multi)")
     ap.add_argument("--no-clock-window", action="store_true",
                     help="do not extend clock sampling past the timed region (for profiler runs)")
     args = ap.parse_args()
+    if args.paged and (args.kv != "bf16" or args.q_len != 1):
+        ap.error("--paged reads a bf16 cache with one query per sequence")
     w = WORKLOADS[args.config]
     world = int(os.environ.get("WORLD_SIZE", 1))
     rank = int(os.environ.get("RANK", 0))

@@ -57,12 +57,13 @@ def lib() -> ctypes.CDLL:
         L.fd_decode_static.argtypes = [_i] * 5 + [_p, _p, _p, _p, _f, _p, _p, _p]
         L.fd_decode_paged.argtypes = [_i] * 8 + [_p, _p, _p, _p, _p, _f, _p, _p, _p, _sz, _i, _p]
         L.fd_decode_multi.argtypes = [_i] * 6 + [_p, _p, _p, _p, _f, _p, _p, _p, _sz, _i, _p]
+        L.fd_decode_quant.argtypes = [_i] * 7 + [_p, _p, _p, _p, _p, _p, _f, _p, _p, _p, _sz, _i, _p]
         L.fd_strerror.argtypes = [_i]
         L.fd_strerror.restype = ctypes.c_char_p
         L.fd_version.argtypes = []
         for name in ("fd_plan", "fd_plan_for_sms", "fd_decode", "fd_decode_splits", "fd_split", "fd_combine",
                      "fd_segments", "fd_device_status", "fd_version", "fd_workspace_init", "fd_decode_static",
-                     "fd_decode_paged", "fd_decode_multi"):
+                     "fd_decode_paged", "fd_decode_multi", "fd_decode_quant"):
             getattr(L, name).restype = _i
         _lib = L
     return _lib
@@ -345,6 +346,87 @@ def prepare_decode_multi(q, k_cache, v_cache, seqlens, scale, out, lse, workspac
 
     call.num_splits = S
     return call
+
+
+FD_KV_E4M3, FD_KV_INT8 = 1, 2
+KV_CODES = {"e4m3": FD_KV_E4M3, "int8": FD_KV_INT8}
+
+
+def prepare_decode_quant(q, k_codes, v_codes, k_scale, v_scale, kv_type, seqlens, scale, out, lse, workspace=None,
+                         num_splits=None, stream=None):
+    """prepare_decode for fd_decode_quant: an 8-bit cache (k_codes / v_codes
+    uint8 [B, Hkv, Lmax, D], k_scale / v_scale float32 [Hkv], kv_type "e4m3"
+    or "int8"); q [B, Hq, D] (one query) or [B, q_len, Hq, D], out / lse
+    shaped to match."""
+    if kv_type not in KV_CODES:
+        raise ValueError("kv_type must be 'e4m3' or 'int8'")
+    if q.dim() == 3:
+        B, Hq, D = q.shape
+        q_len = 1
+    elif q.dim() == 4:
+        B, q_len, Hq, D = q.shape
+    else:
+        raise ValueError("q must be [B, Hq, D] or [B, q_len, Hq, D]")
+    if q.dtype != torch.bfloat16 or not q.is_cuda or not q.is_contiguous():
+        raise ValueError("q must be a contiguous bf16 CUDA tensor")
+    if k_codes.dim() != 4 or v_codes.shape != k_codes.shape or k_codes.shape[0] != B or k_codes.shape[3] != D:
+        raise ValueError("k_codes, v_codes must be [B, Hkv, Lmax, D]")
+    _, Hkv, Lmax, _ = k_codes.shape
+    for t, name in ((k_codes, "k_codes"), (v_codes, "v_codes")):
+        if t.dtype != torch.uint8 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous uint8 CUDA tensor")
+    for t, name in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        if t.shape != (Hkv,) or t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor of shape [Hkv]")
+    oshape = q.shape[:-1]
+    if out.shape != q.shape or lse.shape != oshape:
+        raise ValueError("out must be shaped like q and lse like q without D")
+    for t, name in ((out, "out"), (lse, "lse")):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor")
+    _seqlens(seqlens, B)
+    S = fd_plan(B, Hq, Hkv, D, Lmax) if num_splits is None else int(num_splits)
+    wp, wb = _ws(workspace)
+    fn = lib().fd_decode_quant
+    args = (B, q_len, Hq, Hkv, D, Lmax, KV_CODES[kv_type], q.data_ptr(), k_codes.data_ptr(), v_codes.data_ptr(),
+            k_scale.data_ptr(), v_scale.data_ptr(), seqlens.data_ptr(), ctypes.c_float(scale), out.data_ptr(),
+            lse.data_ptr(), wp, wb, S, _stream(stream, q.device))
+
+    def call():
+        rc = fn(*args)
+        if rc != 0:
+            raise FdError(rc, "fd_decode_quant")
+
+    call.num_splits = S
+    return call
+
+
+def fd_decode_quant(q, k_codes, v_codes, k_scale, v_scale, kv_type, seqlens, scale, out, lse, workspace=None,
+                    num_splits=0, stream=None):
+    """Attention over an 8-bit key/value cache (see prepare_decode_quant);
+    num_splits 0 lets the library plan the split count."""
+    prepare_decode_quant(q, k_codes, v_codes, k_scale, v_scale, kv_type, seqlens, scale, out, lse, workspace,
+                         num_splits, stream)()
+
+
+def quant_workspace_bytes(q, k_codes, num_splits):
+    """Workspace bytes fd_decode_quant needs for these shapes."""
+    q_len = 1 if q.dim() == 3 else q.shape[1]
+    B, Hq, D = q.shape[0], q.shape[-2], q.shape[-1]
+    return fd_workspace_bytes(B, Hq * q_len, k_codes.shape[1], D, k_codes.shape[2], num_splits)
+
+
+def decode_quant(q, k_codes, v_codes, k_scale, v_scale, kv_type, seqlens, scale, num_splits=None, stream=None):
+    """Allocate out / lse / workspace with torch and run fd_decode_quant."""
+    B, Hq, D = q.shape[0], q.shape[-2], q.shape[-1]
+    Hkv, Lmax = k_codes.shape[1], k_codes.shape[2]
+    S = fd_plan(B, Hq, Hkv, D, Lmax) if num_splits is None else int(num_splits)
+    nbytes = quant_workspace_bytes(q, k_codes, S)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
+    out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    fd_decode_quant(q, k_codes, v_codes, k_scale, v_scale, kv_type, seqlens, scale, out, lse, ws, S, stream)
+    return out, lse
 
 
 def workspace_layout(B, Hq, Hkv, D, num_splits):

@@ -12,6 +12,7 @@
 #include "fd.h"
 #include "fd_combine.cuh"
 #include "fd_partition.cuh"
+#include "fd_quant.cuh"
 #include "fd_split.cuh"
 
 namespace {
@@ -124,18 +125,22 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// K or V cache [B*Hkv rows][Lmax][D] bf16 as a 3-D tensor (D innermost);
-// box = 64 head-dim elements (128 bytes, 128-byte swizzle) x 64 tokens x 1 row.
-int encode_cache_map(CUtensorMap *map, const void *base, int D, int Lmax, long long rows) {
+// K or V cache [B*Hkv rows][Lmax][D] as a 3-D tensor (D innermost). bf16:
+// box = 64 head-dim elements (128 bytes, 128-byte swizzle) x 64 tokens x 1
+// row. 8-bit codes (one_byte): box = all D codes of a token (128 bytes with
+// the 128-byte swizzle for D = 128, 64 bytes with the 64-byte one for D = 64).
+int encode_cache_map(CUtensorMap *map, const void *base, int D, int Lmax, long long rows, bool one_byte = false) {
     auto fn = encode_fn();
     if (!fn) return FD_ERR_LAUNCH;
+    const cuuint64_t e = one_byte ? 1 : 2;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Lmax), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Lmax) * D * 2};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(fd::kTileTokens), 1};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * e, static_cast<cuuint64_t>(Lmax) * D * e};
+    cuuint32_t box[3] = {one_byte ? static_cast<cuuint32_t>(D) : 64u, static_cast<cuuint32_t>(fd::kTileTokens), 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUtensorMapSwizzle swz = one_byte && D == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    CUresult r = fn(map, one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FD_OK : FD_ERR_LAUNCH;
 }
 
@@ -182,7 +187,7 @@ int encode_paged_map(CUtensorMap *map, const void *base, int D, int page_size, i
 // ---------------------------------------------------------------- launches --
 template <int D, class Consumer, bool kFused, bool kPaged>
 int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p, cudaStream_t st) {
-    constexpr int smem = fd::SplitConfig<D, Consumer::G>::kSmemBytes;
+    constexpr int smem = fd::SplitConfig<D, Consumer::G, Consumer::kElemBytes>::kSmemBytes;
     auto kern = fd::fd_split_kernel<D, Consumer, kFused, kPaged>;
     // the attribute is per function and device; set it once per device
     static std::once_flag once[kMaxDevices];
@@ -230,6 +235,18 @@ int launch_split(int D, int g, const CUtensorMap &tk, const CUtensorMap &tv, con
     if (g == 1) return launch_split_t<64, fd::HeadConsumer<64>, kFused, kPaged>(tk, tv, p, st);
     if (g <= 8) return launch_split_t<64, fd::GroupConsumer<64, 1>, kFused, kPaged>(tk, tv, p, st);
     return launch_split_t<64, fd::GroupConsumer<64, 2>, kFused, kPaged>(tk, tv, p, st);
+}
+
+// 8-bit caches: the tensor-core consumer for every column count (fused form).
+template <bool kE4M3>
+int launch_split_quant(int D, int cols, const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p,
+                       cudaStream_t st) {
+    if (D == 128) {
+        if (cols <= 8) return launch_split_t<128, fd::QuantConsumer<128, 1, kE4M3>, true, false>(tk, tv, p, st);
+        return launch_split_t<128, fd::QuantConsumer<128, 2, kE4M3>, true, false>(tk, tv, p, st);
+    }
+    if (cols <= 8) return launch_split_t<64, fd::QuantConsumer<64, 1, kE4M3>, true, false>(tk, tv, p, st);
+    return launch_split_t<64, fd::QuantConsumer<64, 2, kE4M3>, true, false>(tk, tv, p, st);
 }
 
 int launch_combine(int D, const fd::CombineParams &p, cudaStream_t st, bool after_split) {
@@ -336,6 +353,7 @@ int run_split(const Problem &pr, bool fused, int q_len = 1) {
     p.max_pages = 0;
     p.page_shift = 0;
     p.kv_nhd = 0;
+    p.k_scale = p.v_scale = nullptr;
     // with max_len == 0 every block finds zero tiles and only writes empty rows;
     // the (unused) tensor maps stay zeroed
     return fused ? launch_split<true>(pr.D, p.cols, tk, tv, p, pr.stream)
@@ -375,7 +393,46 @@ int run_split_paged(const Problem &pr, const PagedLayout &pl) {
     p.page_shift = 0;
     while ((1 << p.page_shift) < pl.page_size) ++p.page_shift;
     p.kv_nhd = pl.nhd ? 1 : 0;
+    p.k_scale = p.v_scale = nullptr;
     return launch_split<true, true>(pr.D, p.g, tk, tv, p, pr.stream);
+}
+
+// Fused split kernel over an 8-bit cache (pr.k / pr.v point at the codes).
+int run_split_quant(const Problem &pr, int q_len, int kv_type, const float *k_scale, const float *v_scale) {
+    int sms;
+    int rc = device_sms(&sms);
+    if (rc != FD_OK) return rc;
+    CUtensorMap tk, tv;
+    std::memset(&tk, 0, sizeof tk);
+    std::memset(&tv, 0, sizeof tv);
+    const long long rows = static_cast<long long>(pr.B) * pr.Hkv;
+    if (pr.max_len > 0) {
+        if ((rc = encode_cache_map(&tk, pr.k, pr.D, pr.max_len, rows, true)) != FD_OK) return rc;
+        if ((rc = encode_cache_map(&tv, pr.v, pr.D, pr.max_len, rows, true)) != FD_OK) return rc;
+    }
+    fd::SplitParams p;
+    p.q = pr.q;
+    p.seqlens = pr.seqlens;
+    p.out = pr.out;
+    p.lse = pr.lse;
+    seg_pointers(pr, &p.seg_out, &p.seg_lse, &p.row_tickets, q_len);
+    p.B = pr.B;
+    p.Hq = pr.Hq;
+    p.Hkv = pr.Hkv;
+    p.g = pr.Hq / pr.Hkv;
+    p.Lmax = pr.max_len;
+    p.P = pr.num_splits;
+    p.q_len = q_len;
+    p.cols = p.g * q_len;
+    p.scale_log2e = pr.scale * kLog2e;
+    p.block_table = nullptr;
+    p.max_pages = 0;
+    p.page_shift = 0;
+    p.kv_nhd = 0;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    return kv_type == FD_KV_E4M3 ? launch_split_quant<true>(pr.D, p.cols, tk, tv, p, pr.stream)
+                                 : launch_split_quant<false>(pr.D, p.cols, tk, tv, p, pr.stream);
 }
 
 int run_combine(const Problem &pr, bool after_split) {
@@ -613,6 +670,36 @@ int fd_decode_multi(int B, int q_len, int Hq, int Hkv, int D, int max_len, const
     }
     pr.Hq = Hq;   // the kernel indexes q / out with the real head count
     return run_split(pr, true, q_len);
+}
+
+int fd_decode_quant(int B, int q_len, int Hq, int Hkv, int D, int max_len, int kv_type, const uint16_t *q,
+                    const uint8_t *k_codes, const uint8_t *v_codes, const float *k_scale, const float *v_scale,
+                    const int32_t *seqlens, float scale, float *out, float *lse, void *workspace,
+                    size_t workspace_bytes, int num_splits, void *stream) {
+    if (q_len < 1 || q_len > FD_MAX_GROUP) return FD_ERR_SHAPE;
+    if (kv_type != FD_KV_E4M3 && kv_type != FD_KV_INT8) return FD_ERR_SHAPE;
+    int rc = check_shape(B, Hq, Hkv, D, max_len);
+    if (rc != FD_OK) return rc;
+    if (static_cast<long long>(Hq) * q_len / Hkv > FD_MAX_GROUP) return FD_ERR_GROUP;
+    if (num_splits < 0) return FD_ERR_SPLITS;
+    if (max_len > 0) {
+        if (!k_scale || !v_scale) return FD_ERR_NULL_POINTER;
+        if (!aligned(k_scale, 4) || !aligned(v_scale, 4)) return FD_ERR_ALIGNMENT;
+    }
+    // the checks and the workspace see the (query, head) columns as Hq * q_len heads
+    const int Hqq = Hq * q_len;
+    Problem pr = make_problem(B, Hqq, Hkv, D, max_len, q, reinterpret_cast<const uint16_t *>(k_codes),
+                              reinterpret_cast<const uint16_t *>(v_codes), seqlens, scale, out, lse, workspace,
+                              workspace_bytes, num_splits == 0 ? 1 : num_splits, stream);
+    if ((rc = check_problem(pr, true)) != FD_OK) return rc;
+    if (num_splits == 0) {
+        const int S = fd_plan(B, Hq, Hkv, D, max_len);
+        if (S < 0) return S;
+        pr.num_splits = S;
+        if ((rc = check_problem(pr, true)) != FD_OK) return rc;
+    }
+    pr.Hq = Hq;
+    return run_split_quant(pr, q_len, kv_type, k_scale, v_scale);
 }
 
 int fd_decode_static(int B, int Hq, int Hkv, int D, int max_len, const uint16_t *q, const uint16_t *k_cache,

@@ -86,6 +86,9 @@ struct SplitParams {
     int max_pages;            // block-table row length (a multiple of 4)
     int page_shift;           // log2(page_size)
     int kv_nhd;               // 0: pages [num_pages, Hkv, page_size, D]; 1: [num_pages, page_size, Hkv, D]
+    // 8-bit caches only: value of a cached element = scale[kv head] * decode(code)
+    const float *k_scale;     // [Hkv]
+    const float *v_scale;     // [Hkv]
 };
 
 constexpr int kPageWindow = 1024;                 // block-table entries staged in shared memory
@@ -97,22 +100,31 @@ __device__ __forceinline__ size_t out_row(const SplitParams &p, int b, int h, in
     return (static_cast<size_t>(b) * p.q_len + j) * p.Hq + static_cast<size_t>(h) * p.g + i;
 }
 
-template <int D, int G>
+// E = bytes per cached element: 2 (bf16) or 1 (8-bit codes).
+template <int D, int G, int E = 2>
 struct SplitConfig {
-    static constexpr int kBoxes = D / 64;                                  // 128-byte boxes per row
-    static constexpr int kTileBytes = kTileTokens * D * 2;                 // one K (or V) tile
-    static constexpr int kQSlotBytes = (G * D * 2 + 1023) / 1024 * 1024;   // query heads of a row
+    static constexpr int kRowBytes = D * E;                                // one token of one head
+    static constexpr int kBoxRowBytes = kRowBytes < 128 ? kRowBytes : 128; // a box row = one swizzle span
+    static constexpr int kBoxCols = kBoxRowBytes / E;                      // head-dim elements per box
+    static constexpr int kBoxes = D / kBoxCols;                            // boxes per tile
+    static constexpr int kBoxBytes = kTileTokens * kBoxRowBytes;
+    static constexpr int kTileBytes = kTileTokens * kRowBytes;             // one K (or V) tile
+    static constexpr int kQSlotBytes = (G * D * 2 + 1023) / 1024 * 1024;   // query heads of a row (bf16)
     static constexpr int kStageBytes = 2 * kTileBytes + kQSlotBytes;       // multiple of 1024 (swizzle)
-    static constexpr int kStages = D == 128 ? 4 : 8;                       // 128 KiB of K/V: measured best
-    static constexpr int kRingBytes = kStages * kStageBytes;
     static constexpr int kWarpFloats = G * D + 2 * G;                      // o, m, l of one warp
     static constexpr int kMergeFloats = kConsumerWarps * kWarpFloats;      // one merge buffer
     static constexpr int kCtrlBytes = 2048;                                // barriers, start info, queue, weights
     static constexpr int kPageBytes = kPageWindow * 4;                     // block-table window (paged)
-    static constexpr int kMergeBufs =
-        1024 + kRingBytes + 2 * kMergeFloats * 4 + kCtrlBytes + kPageBytes <= kSmemLimit ? 2 : 1;
-    static constexpr int kSmemBytes =
-        1024 + kRingBytes + kMergeBufs * kMergeFloats * 4 + kCtrlBytes + kPageBytes;
+    static constexpr int kFixedBytes = 1024 + kCtrlBytes + kPageBytes;
+    // 128 KiB of K/V tiles in flight (measured best for bf16: 4 stages at
+    // D = 128), as many as fit next to one merge buffer, in whole pairs
+    static constexpr int fit_stages(int s) {
+        return s > 2 && kFixedBytes + s * kStageBytes + kMergeFloats * 4 > kSmemLimit ? fit_stages(s - 2) : s;
+    }
+    static constexpr int kStages = fit_stages(1024 / kRowBytes);
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kMergeBufs = kFixedBytes + kRingBytes + 2 * kMergeFloats * 4 <= kSmemLimit ? 2 : 1;
+    static constexpr int kSmemBytes = kFixedBytes + kRingBytes + kMergeBufs * kMergeFloats * 4;
     // Each consumer group owns whole stages: a stage shared by both groups
     // could be waited on two phases ahead of a tile still in flight, where a
     // parity wait would pass on the older phase.
@@ -301,6 +313,7 @@ struct GroupConsumer {
     static constexpr int KS = D / 16;   // k-steps of the logit contraction
     static constexpr int MT = D / 16;   // m-tiles of the P V contraction
     static constexpr int G = 8 * NT;    // heads held (padded)
+    static constexpr int kElemBytes = 2;
 
     uint32_t qf[NT][KS][2];             // Q^T as the B operand, per n-tile
     float m[NT][2], l[NT][2];           // running max (base 2) / partial sum for heads 2c, 2c+1
@@ -317,6 +330,8 @@ struct GroupConsumer {
                 shift[nt][e] = col < p.cols ? p.q_len - 1 - col / p.g : 0;
             }
     }
+
+    __device__ __forceinline__ void set_row(const SplitParams &, int) {}   // bf16 cache: no per-head scales
 
     __device__ __forceinline__ void reset() {
 #pragma unroll
@@ -476,6 +491,7 @@ struct GroupConsumer {
 template <int D>
 struct HeadConsumer {
     static constexpr int G = 1;
+    static constexpr int kElemBytes = 2;
     static constexpr int LPT = D / 8;          // lanes per token (16 bytes = 8 bf16 each)
     static constexpr int TPI = 32 / LPT;       // tokens per warp-wide load
     static constexpr int ITER = kWarpTokens / TPI;
@@ -485,6 +501,7 @@ struct HeadConsumer {
     float acc[8];                              // sum of p * v over this lane's tokens, chunk d0..d0+7
 
     __device__ __forceinline__ void init(const SplitParams &) {}   // one query, one head: no offsets
+    __device__ __forceinline__ void set_row(const SplitParams &, int) {}
 
     __device__ __forceinline__ void reset() {
         m = -INFINITY;
@@ -613,7 +630,8 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     fd_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const SplitParams p) {
     constexpr int G = Consumer::G;
-    using Cfg = SplitConfig<D, G>;
+    using Cfg = SplitConfig<D, G, Consumer::kElemBytes>;
+    static_assert(!kPaged || Consumer::kElemBytes == 2, "paged caches are bf16");
     constexpr int kStages = Cfg::kStages;
     constexpr int kBufs = Cfg::kMergeBufs;
 
@@ -666,7 +684,8 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             if (t < info->count && tile < info->n) {
                 const CUtensorMap *map = (lane & 1) ? &tm_v : &tm_k;
                 const int z = info->b * p.Hkv + info->h;
-                for (int bx = 0; bx < D / 64; ++bx) tma_prefetch_l2_3d(map, 64 * bx, tile * kTileTokens, z);
+                for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+                    tma_prefetch_l2_3d(map, Cfg::kBoxCols * bx, tile * kTileTokens, z);
             }
         }
         __syncwarp();
@@ -727,8 +746,8 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                     mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kTileBytes + qb);
 #pragma unroll
                     for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-                        tma_load_3d(kt + bx * kBoxBytes, &tm_k, &full[stage], 64 * bx, y, z, policy);
-                        tma_load_3d(vt + bx * kBoxBytes, &tm_v, &full[stage], 64 * bx, y, z, policy);
+                        tma_load_3d(kt + bx * Cfg::kBoxBytes, &tm_k, &full[stage], Cfg::kBoxCols * bx, y, z, policy);
+                        tma_load_3d(vt + bx * Cfg::kBoxBytes, &tm_v, &full[stage], Cfg::kBoxCols * bx, y, z, policy);
                     }
                 } else {
                     // the tile's tokens [y, y + 64) span one page (page_size >= 64) or
@@ -782,6 +801,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
             const int L = clamp_len(__ldg(p.seqlens + c.b), p.Lmax);
             cons.reset();
+            cons.set_row(p, c.h);
             for (int k = 0; k < seg; ++k, ++seq) {
                 if (static_cast<int>(seq % kGroups) != group) continue;
                 const int stage = static_cast<int>(seq % kStages);

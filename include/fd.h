@@ -90,6 +90,8 @@ extern "C" {
 #define FD_STATIC_SCRATCH_BYTES (8u << 20)   /* fixed device scratch behind fd_decode_static */
 #define FD_KV_HND           0     /* paged pool [num_pages][Hkv][page_size][D] */
 #define FD_KV_NHD           1     /* paged pool [num_pages][page_size][Hkv][D] */
+#define FD_KV_E4M3          1     /* 8-bit cache codes: OCP FP8 E4M3 (fd_decode_quant) */
+#define FD_KV_INT8          2     /* 8-bit cache codes: int8, two's complement (fd_decode_quant) */
 
 /* Number of splits (thread blocks of the split stage) for a problem shape,
  * sized to the current device's SM count: one block per SM while the batch
@@ -152,6 +154,31 @@ FD_API int fd_decode_multi(int B, int q_len, int Hq, int Hkv, int D, int max_len
                            const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
                            const int32_t *seqlens, float scale, float *out, float *lse,
                            void *workspace, size_t workspace_bytes, int num_splits, void *stream);
+
+/* fd_decode_multi over an 8-bit key/value cache with one scale per kv head.
+ * The "flash decoding论文" page lists INT8/INT4 quantisation among PaddleNLP's
+ * inference techniques; one byte per cached element halves the bytes a
+ * decode step streams. k_codes / v_codes: [B][Hkv][max_len][D] bytes, device,
+ * 16-byte aligned; kv_type FD_KV_E4M3 (OCP 8-bit floating point E4M3: sign,
+ * 4 exponent bits with bias 7, 3 mantissa bits, exponent field 0
+ * subnormal, S.1111.111 NaN, no infinities) or FD_KV_INT8. k_scale /
+ * v_scale: [Hkv] float32, device, 4-byte aligned. The cached key of token t
+ * is k_scale[h] * decode(k_codes[b][h][t][:]), the value likewise with
+ * v_scale, and the attention is that of fd_decode_multi over those values
+ * (q [B][q_len][Hq][D] bf16, out [B][q_len][Hq][D] and lse [B][q_len][Hq]
+ * fp32; q_len = 1 is single-query decode; q_len * Hq/Hkv <= 16). Codes past
+ * seqlens[b] are never used, whatever they hold. The query must be finite;
+ * it enters the tensor-core contraction as f16 after an exact power-of-two
+ * prescale per (query, head), so only its elements smaller than 2^-25 of
+ * that query head's largest are rounded. Workspace as fd_decode_multi;
+ * num_splits = 0 means fd_plan(B, Hq, Hkv, D, max_len).
+ * Errors: FD_ERR_SHAPE also for kv_type or q_len out of range;
+ * FD_ERR_NULL_POINTER / FD_ERR_ALIGNMENT also for the scales. */
+FD_API int fd_decode_quant(int B, int q_len, int Hq, int Hkv, int D, int max_len, int kv_type,
+                           const uint16_t *q, const uint8_t *k_codes, const uint8_t *v_codes,
+                           const float *k_scale, const float *v_scale, const int32_t *seqlens, float scale,
+                           float *out, float *lse, void *workspace, size_t workspace_bytes, int num_splits,
+                           void *stream);
 
 /* fd_decode_splits over a PAGED key/value cache. The page pools
  * k_pages / v_pages hold num_pages pages of page_size tokens each, laid out

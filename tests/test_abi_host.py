@@ -38,6 +38,8 @@ def test_constants_match_header():
     assert int(consts["FD_TILE_TOKENS"]) == _lib.FD_TILE_TOKENS
     assert int(consts["FD_MAX_SPLITS"]) == _lib.FD_MAX_SPLITS
     assert int(consts["FD_MAX_GROUP"]) == _lib.FD_MAX_GROUP
+    assert int(consts["FD_KV_E4M3"]) == _lib.FD_KV_E4M3 and int(consts["FD_KV_INT8"]) == _lib.FD_KV_INT8
+    assert int(consts["FD_KV_HND"]) == _lib.FD_KV_HND and int(consts["FD_KV_NHD"]) == _lib.FD_KV_NHD
     for code, name in _lib.ERRORS.items():
         assert int(consts[name]) == code
 
@@ -158,6 +160,24 @@ def test_multi_query_argument_errors_without_a_device():
     assert multi(q_len=3, Hq=3) == -3 and multi(D=96) == -4 and multi(S=-1) == -7
     if not os.path.exists("/dev/nvidia0"):
         assert multi() == -8 and multi(q_len=8) == -8
+
+
+def test_quant_argument_errors_without_a_device():
+    L = fd.lib()
+    buf = (ctypes.c_uint8 * 4096)()
+    a16 = (ctypes.addressof(buf) + 15) // 16 * 16
+    p = ctypes.c_void_p(a16)
+
+    def quant(kv_type=1, q_len=1, Hq=4, Hkv=2, D=128, S=1, ks=p, vs=p, kc=p):
+        return L.fd_decode_quant(1, q_len, Hq, Hkv, D, 64, kv_type, p, kc, p, ks, vs, p, 0.1, p, p, p, 4096, S,
+                                 None)
+
+    assert quant(kv_type=0) == -2 and quant(kv_type=3) == -2 and quant(q_len=0) == -2
+    assert quant(q_len=9) == -3 and quant(Hq=3) == -3 and quant(D=96) == -4 and quant(S=-1) == -7
+    assert quant(ks=None) == -1 and quant(vs=None) == -1
+    assert quant(ks=ctypes.c_void_p(a16 + 2)) == -5 and quant(kc=ctypes.c_void_p(a16 + 8)) == -5
+    if not os.path.exists("/dev/nvidia0"):
+        assert quant() == -8 and quant(kv_type=2, q_len=2) == -8
 
 
 def segments_rule(B, Hkv, Lmax, seqlens, P):
