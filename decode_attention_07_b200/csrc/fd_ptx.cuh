@@ -195,6 +195,25 @@ __device__ __forceinline__ void int8x4_to_f16(uint32_t w, uint32_t &lo, uint32_t
     asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(bias));
 }
 
+// The same widening for a register that ldmatrix.trans filled from an 8-bit
+// tile read as 16-bit elements: bytes (t, d), (t, d+1), (t+1, d), (t+1, d+1)
+// of tokens t, t+1 and head dims d, d+1. lo gets the pair (t, t+1) at d,
+// hi the pair at d + 1 (token t in bits 0..15).
+__device__ __forceinline__ void e4m3x4t_to_f16(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    uint32_t g;
+    asm("prmt.b32 %0, %1, %2, 0x3120;" : "=r"(g) : "r"(w), "r"(0u));
+    e4m3x4_to_f16(g, lo, hi);
+}
+__device__ __forceinline__ void int8x4t_to_f16(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    uint32_t a, b;
+    asm("prmt.b32 %0, %1, %2, 0x7270;" : "=r"(a) : "r"(u), "r"(0x64646464u));
+    asm("prmt.b32 %0, %1, %2, 0x7371;" : "=r"(b) : "r"(u), "r"(0x64646464u));
+    const uint32_t bias = 0x64806480u;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(bias));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(bias));
+}
+
 // Hardware base-2 exponential and logarithm (MUFU), flushing denormals.
 __device__ __forceinline__ float ex2(float x) {
     float y;

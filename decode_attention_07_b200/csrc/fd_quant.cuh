@@ -27,14 +27,24 @@
 //     16-element k-step once the query's B fragment is loaded in the same
 //     order (q[4c .. 4c+3] per thread): the contraction index is only
 //     permuted, identically on both sides.
-//   * P V, O^T += V^T P^T: V must be transposed (tokens along k). The codes of
-//     one token are widened, then movmatrix transposes each 8x8 f16 block in
-//     registers; the head-dim rows come out permuted within each 16-element
-//     chunk (d = 4(r/2) + r%2, then +2), which the store at the end undoes.
-//   * P enters as f16 high part + f16 remainder, scaled by 2^14 so that small
-//     probabilities stay normal f16 numbers; the running sum carries the same
-//     factor, so the normalised output is unchanged and only the log-sum-exp
-//     is corrected (m - 14).
+//   * P V, O^T += V^T P^T: V must be transposed (tokens along k). ldmatrix
+//     .trans of the 8-bit tile, read as 16-bit elements, hands each thread
+//     two tokens x two head dims; one byte permute regroups them into token
+//     pairs per head dim before widening. The accumulator rows then hold the
+//     even head dims of a chunk (rows 0-7) and the odd ones (rows 8-15),
+//     which the store at the end puts back in order.
+//   * Softmax with a lazy reference maximum, after FlashDecoding++'s
+//     asynchronous softmax with a unified max value (the "flash decoding论文"
+//     page names the synchronised partial-softmax update as the problem it
+//     removes): each column keeps a reference m and only a tile with a logit
+//     above m + kLazy triggers the rescale of the running sum and the
+//     accumulators; otherwise its p = 2^(x - m) is summed as is. The result
+//     is the same softmax (m cancels in o / l and in the log-sum-exp); the
+//     common tile skips the cross-lane max and the accumulator rescale.
+//   * P enters as f16 high part + f16 remainder, scaled by 2^kPScale so that
+//     small probabilities stay normal f16 numbers; the running sum carries
+//     the same factor, so the normalised output is unchanged and only the
+//     log-sum-exp is corrected (m - kPScale).
 #pragma once
 
 #include "fd_split.cuh"
@@ -47,11 +57,15 @@ struct QuantConsumer {
     static constexpr int kElemBytes = 1;
     static constexpr int KC = D / 16;       // 16-byte chunks of a token = k-steps of S = m-tiles of O^T
     static constexpr int kRowBytes = D;
-    static constexpr float kPScale = 14.f;  // p enters the P V product as p * 2^14
+    // The reference max lags the running max by at most kLazy (base 2), so
+    // p = 2^(x - m) <= 2^kLazy; P enters the P V product as p * 2^kPScale,
+    // at most 2^15 (f16 tops out near 2^16) and a normal f16 down to p = 2^-21.
+    static constexpr float kLazy = 8.f;
+    static constexpr float kPScale = 7.f;
 
     uint32_t qf[NT][KC][2];                 // Q^T as the B operand (f16), per n-tile
-    float m[NT][2], l[NT][2];               // running max (base 2) / partial sum (x 2^14) for columns 2c, 2c+1
-    float o[NT][KC][4];                     // O^T accumulators (x 2^14, head dims permuted within chunks)
+    float m[NT][2], l[NT][2];               // reference max (base 2) / partial sum (x 2^kPScale), columns 2c, 2c+1
+    float o[NT][KC][4];                     // O^T accumulators (x 2^kPScale, head dims even | odd per chunk)
     int shift[NT][2];                       // causal offset of columns 2c, 2c+1
     float colmul[NT][2];                    // logit multiplier (base 2) of columns 2c, 2c+1
     float kmul, vmul;                       // scale * log2(e) * k_scale[h], and v_scale[h]
@@ -97,6 +111,12 @@ struct QuantConsumer {
             e4m3x4_to_f16(w, lo, hi);
         else
             int8x4_to_f16(w, lo, hi);
+    }
+    static __device__ __forceinline__ void widen_t(uint32_t w, uint32_t &lo, uint32_t &hi) {
+        if constexpr (kE4M3)
+            e4m3x4t_to_f16(w, lo, hi);
+        else
+            int8x4t_to_f16(w, lo, hi);
     }
 
     // Q^T fragments from the stage's bf16 copy of the row's columns ([cols][D]).
@@ -175,39 +195,61 @@ struct QuantConsumer {
             }
         }
 
-        // online softmax per column; P^T fragments (f16 high + remainder, x 2^14)
+        // Online softmax per column with a lazy reference maximum: m moves
+        // (and the accumulators are rescaled) only when a logit of the tile
+        // exceeds it by more than kLazy; otherwise p = 2^(x - m) directly.
+        float x[NT][4];
+        bool grow = false;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            x[nt][0] = (s[nt][0] + s2[nt][0]) * colmul[nt][0];
+            x[nt][1] = (s[nt][1] + s2[nt][1]) * colmul[nt][1];
+            x[nt][2] = (s[nt][2] + s2[nt][2]) * colmul[nt][0];
+            x[nt][3] = (s[nt][3] + s2[nt][3]) * colmul[nt][1];
+            const int va = valid - shift[nt][0], vb = valid - shift[nt][1];
+            if (r0 >= va) x[nt][0] = -INFINITY;
+            if (r0 >= vb) x[nt][1] = -INFINITY;
+            if (r0 + 8 >= va) x[nt][2] = -INFINITY;
+            if (r0 + 8 >= vb) x[nt][3] = -INFINITY;
+            const float ta = m[nt][0] + kLazy, tb = m[nt][1] + kLazy;
+            grow |= x[nt][0] > ta || x[nt][2] > ta || x[nt][1] > tb || x[nt][3] > tb;
+        }
+        if (__any_sync(0xffffffffu, grow)) {   // the fallback: a synchronised rescale
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float ma = fmaxf(x[nt][0], x[nt][2]), mb = fmaxf(x[nt][1], x[nt][3]);
+#pragma unroll
+                for (int sh = 4; sh < 32; sh <<= 1) {
+                    ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, sh));
+                    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, sh));
+                }
+                const float na = fmaxf(m[nt][0], ma), nb = fmaxf(m[nt][1], mb);
+                const float ua = na == -INFINITY ? 0.f : na, ub = nb == -INFINITY ? 0.f : nb;
+                const float alpha_a = ex2(m[nt][0] - ua), alpha_b = ex2(m[nt][1] - ub);
+                l[nt][0] *= alpha_a;
+                l[nt][1] *= alpha_b;
+                m[nt][0] = na;
+                m[nt][1] = nb;
+#pragma unroll
+                for (int c = 0; c < KC; ++c) {
+                    o[nt][c][0] *= alpha_a;
+                    o[nt][c][1] *= alpha_b;
+                    o[nt][c][2] *= alpha_a;
+                    o[nt][c][3] *= alpha_b;
+                }
+            }
+        }
+
+        // P^T fragments (f16 high part + remainder, x 2^kPScale)
         uint32_t bh[NT][2], bl[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            float x0 = (s[nt][0] + s2[nt][0]) * colmul[nt][0], x1 = (s[nt][1] + s2[nt][1]) * colmul[nt][1];
-            float x2 = (s[nt][2] + s2[nt][2]) * colmul[nt][0], x3 = (s[nt][3] + s2[nt][3]) * colmul[nt][1];
-            const int va = valid - shift[nt][0], vb = valid - shift[nt][1];
-            if (r0 >= va) x0 = -INFINITY;
-            if (r0 >= vb) x1 = -INFINITY;
-            if (r0 + 8 >= va) x2 = -INFINITY;
-            if (r0 + 8 >= vb) x3 = -INFINITY;
-            float ma = fmaxf(x0, x2), mb = fmaxf(x1, x3);
-#pragma unroll
-            for (int sh = 4; sh < 32; sh <<= 1) {
-                ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, sh));
-                mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, sh));
-            }
-            const float na = fmaxf(m[nt][0], ma), nb = fmaxf(m[nt][1], mb);
-            const float ua = na == -INFINITY ? 0.f : na, ub = nb == -INFINITY ? 0.f : nb;
-            const float alpha_a = ex2(m[nt][0] - ua), alpha_b = ex2(m[nt][1] - ub);
-            const float ta = kPScale - ua, tb = kPScale - ub;
-            const float p0 = ex2(x0 + ta), p2 = ex2(x2 + ta), p1 = ex2(x1 + tb), p3 = ex2(x3 + tb);
-            l[nt][0] = fmaf(l[nt][0], alpha_a, p0 + p2);
-            l[nt][1] = fmaf(l[nt][1], alpha_b, p1 + p3);
-            m[nt][0] = na;
-            m[nt][1] = nb;
-#pragma unroll
-            for (int c = 0; c < KC; ++c) {
-                o[nt][c][0] *= alpha_a;
-                o[nt][c][1] *= alpha_b;
-                o[nt][c][2] *= alpha_a;
-                o[nt][c][3] *= alpha_b;
-            }
+            const float ta = kPScale - (m[nt][0] == -INFINITY ? 0.f : m[nt][0]);
+            const float tb = kPScale - (m[nt][1] == -INFINITY ? 0.f : m[nt][1]);
+            const float p0 = ex2(x[nt][0] + ta), p2 = ex2(x[nt][2] + ta);
+            const float p1 = ex2(x[nt][1] + tb), p3 = ex2(x[nt][3] + tb);
+            l[nt][0] += p0 + p2;
+            l[nt][1] += p1 + p3;
             const uint32_t h01 = pack_f16x2(p0, p1), h23 = pack_f16x2(p2, p3);
             const uint32_t l01 = pack_f16x2(p0 - f16lo_to_f32(h01), p1 - f16hi_to_f32(h01));
             const uint32_t l23 = pack_f16x2(p2 - f16lo_to_f32(h23), p3 - f16hi_to_f32(h23));
@@ -217,20 +259,22 @@ struct QuantConsumer {
             bl[nt][1] = movmatrix_trans(l23);
         }
 
-        // O^T += V^T P^T, one 16-element chunk of head dims per m-tile
+        // O^T += V^T P^T, one 16-element chunk of head dims per m-tile.
+        // ldmatrix.trans of the 8-bit tile read as 16-bit elements gives each
+        // thread tokens (2cc, 2cc+1) x head dims (2r0, 2r0+1) of a chunk; the
+        // widening regroups them into token pairs at head dims 2r0 (accumulator
+        // row r0) and 2r0 + 1 (row r0 + 8).
 #pragma unroll
         for (int pc = 0; pc < KC / 2; ++pc) {
             const int chunk = 2 * pc + (mi >> 1);
             uint32_t a[4];
-            ldsm_x4(v_smem + lrow * kRowBytes + (swz(chunk, lrow) << 4), a[0], a[1], a[2], a[3]);
+            ldsm_x4_trans(v_smem + lrow * kRowBytes + (swz(chunk, lrow) << 4), a[0], a[1], a[2], a[3]);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                // tokens r0 (x) and r0 + 8 (y), chunk 2pc + half, four codes each
-                uint32_t xl, xh, yl, yh;
-                widen(a[2 * half], xl, xh);
-                widen(a[2 * half + 1], yl, yh);
-                uint32_t A0 = movmatrix_trans(xl), A1 = movmatrix_trans(xh);
-                uint32_t A2 = movmatrix_trans(yl), A3 = movmatrix_trans(yh);
+                // tokens 0..7 (x) and 8..15 (y) of the slice, chunk 2pc + half
+                uint32_t A0, A1, A2, A3;
+                widen_t(a[2 * half], A0, A1);
+                widen_t(a[2 * half + 1], A2, A3);
                 if (valid < kWarpTokens) {   // rows past the end may hold anything (NaN codes): zero them
                     A0 = keep_tokens(A0, 2 * cc, valid);
                     A1 = keep_tokens(A1, 2 * cc, valid);
@@ -248,11 +292,11 @@ struct QuantConsumer {
 
     // This warp's (o, m, l) into a merge buffer slot: o[G][D] with the head
     // dims back in order and the value scale applied, then m[G] (base 2,
-    // without the 2^14 factor), l[G].
+    // without the 2^kPScale factor), l[G].
     __device__ __forceinline__ void to_smem(float *wb) {
         const int lane = threadIdx.x & 31;
         const int r0 = lane >> 2, cc = lane & 3;
-        const int dlo = 4 * (r0 >> 1) + (r0 & 1);   // head dim of accumulator row r0 within its chunk
+        const int dlo = 2 * r0;   // head dim of accumulator row r0 within its chunk (row r0 + 8: dlo + 1)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -262,7 +306,7 @@ struct QuantConsumer {
             const int ha = nt * 8 + 2 * cc, hb = ha + 1;
 #pragma unroll
             for (int c = 0; c < KC; ++c) {
-                const int d0 = 16 * c + dlo, d1 = d0 + 2;
+                const int d0 = 16 * c + dlo, d1 = d0 + 1;
                 wb[ha * D + d0] = o[nt][c][0] * vmul;
                 wb[hb * D + d0] = o[nt][c][1] * vmul;
                 wb[ha * D + d1] = o[nt][c][2] * vmul;

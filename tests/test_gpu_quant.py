@@ -123,3 +123,34 @@ def test_full_size(name, kv_type):
     bs = list(range(w.B)) if w.B <= 4 else [0, w.B // 2, w.B - 1]
     ref_o, ref_l = oracle_quant(x, bs=bs)
     compare(out[bs], lse[bs], ref_o, ref_l, f"{name} {kv_type}")
+
+
+def codes_with_profile(x, prof_k):
+    """Replace x's key codes by fresh ones whose magnitude follows prof_k[t]
+    along the sequence (scales re-derived so the largest value uses the code
+    range); value codes are kept."""
+    from decode_attention_07_b200.inputs import QUANT_RANGE, _codes
+    w = x.workload
+    g = torch.Generator(device="cuda").manual_seed(11)
+    k = torch.randn((w.B, w.Hkv, w.Lmax, w.D), generator=g, device="cuda") * prof_k[None, None, :, None]
+    ks = (k.abs().amax(dim=(0, 2, 3)) / QUANT_RANGE[x.kv_type]).float()
+    x.k8 = _codes(k / ks[None, :, None, None], x.kv_type).contiguous()
+    x.k_scale = ks.contiguous()
+    return x
+
+
+@pytest.mark.parametrize("kv_type", KV)
+@pytest.mark.parametrize("profile", ["rising", "falling"])
+def test_lazy_max_fallback(kv_type, profile):
+    """Rising logits exceed the reference maximum again and again (the
+    rescale fallback runs on many tiles); falling logits put the maximum in
+    the first tile (no fallback after it). Both against the oracle."""
+    w = Workload("q8", B=2, Hq=8, Hkv=2, D=128, Lmax=4096, ragged=False, nan_pad=False, sigma_q=1.0)
+    x = make_quant(w, kv_type, seed=8, device="cuda")
+    t = torch.arange(w.Lmax, device="cuda", dtype=torch.float32) / w.Lmax
+    prof = 0.2 + 6.0 * t if profile == "rising" else 6.2 - 6.0 * t
+    x = codes_with_profile(x, prof)
+    ref_o, ref_l = oracle_quant(x)
+    for S in (1, 9, 148):
+        out, lse = run(x, S=S)
+        compare(out, lse, ref_o, ref_l, f"{kv_type} {profile} S={S}")
