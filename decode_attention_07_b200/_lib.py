@@ -58,12 +58,13 @@ def lib() -> ctypes.CDLL:
         L.fd_decode_paged.argtypes = [_i] * 8 + [_p, _p, _p, _p, _p, _f, _p, _p, _p, _sz, _i, _p]
         L.fd_decode_multi.argtypes = [_i] * 6 + [_p, _p, _p, _p, _f, _p, _p, _p, _sz, _i, _p]
         L.fd_decode_quant.argtypes = [_i] * 7 + [_p, _p, _p, _p, _p, _p, _f, _p, _p, _p, _sz, _i, _p]
+        L.fd_merge_partials.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p]
         L.fd_strerror.argtypes = [_i]
         L.fd_strerror.restype = ctypes.c_char_p
         L.fd_version.argtypes = []
         for name in ("fd_plan", "fd_plan_for_sms", "fd_decode", "fd_decode_splits", "fd_split", "fd_combine",
                      "fd_segments", "fd_device_status", "fd_version", "fd_workspace_init", "fd_decode_static",
-                     "fd_decode_paged", "fd_decode_multi", "fd_decode_quant"):
+                     "fd_decode_paged", "fd_decode_multi", "fd_decode_quant", "fd_merge_partials"):
             getattr(L, name).restype = _i
         _lib = L
     return _lib
@@ -427,6 +428,22 @@ def decode_quant(q, k_codes, v_codes, k_scale, v_scale, kv_type, seqlens, scale,
     lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
     fd_decode_quant(q, k_codes, v_codes, k_scale, v_scale, kv_type, seqlens, scale, out, lse, ws, S, stream)
     return out, lse
+
+
+def fd_merge_partials(part_out, part_lse, out, lse, stream=None):
+    """Merge R partial results per row: part_out [R, ..., D] and part_lse
+    [R, ...] (fp32, contiguous, CUDA) into out [..., D] and lse [...]."""
+    if part_out.dim() < 2 or part_lse.shape != part_out.shape[:-1]:
+        raise ValueError("part_out must be [R, ..., D] and part_lse [R, ...]")
+    R, D = part_out.shape[0], part_out.shape[-1]
+    rows = part_lse[0].numel()
+    if out.shape != part_out.shape[1:] or lse.shape != part_lse.shape[1:]:
+        raise ValueError("out / lse must be shaped like one part")
+    for t, name in ((part_out, "part_out"), (part_lse, "part_lse"), (out, "out"), (lse, "lse")):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor")
+    _check(lib().fd_merge_partials(R, rows, D, part_out.data_ptr(), part_lse.data_ptr(), out.data_ptr(),
+                                   lse.data_ptr(), _stream(stream, out.device)), "fd_merge_partials")
 
 
 def workspace_layout(B, Hq, Hkv, D, num_splits):

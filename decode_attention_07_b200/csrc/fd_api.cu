@@ -11,6 +11,7 @@
 
 #include "fd.h"
 #include "fd_combine.cuh"
+#include "fd_partials.cuh"
 #include "fd_partition.cuh"
 #include "fd_quant.cuh"
 #include "fd_split.cuh"
@@ -700,6 +701,24 @@ int fd_decode_quant(int B, int q_len, int Hq, int Hkv, int D, int max_len, int k
     }
     pr.Hq = Hq;
     return run_split_quant(pr, q_len, kv_type, k_scale, v_scale);
+}
+
+int fd_merge_partials(int R, int rows, int D, const float *part_out, const float *part_lse, float *out, float *lse,
+                      void *stream) {
+    if (R < 1 || rows < 0) return FD_ERR_SHAPE;
+    if (D < 4 || D > 4096 || D % 4 != 0) return FD_ERR_HEAD_DIM;
+    if (rows == 0) return FD_OK;
+    if (!part_out || !part_lse || !out || !lse) return FD_ERR_NULL_POINTER;
+    if (!aligned(part_out, 16) || !aligned(out, 16) || !aligned(part_lse, 4) || !aligned(lse, 4))
+        return FD_ERR_ALIGNMENT;
+    int dev;
+    if (current_device(&dev) != FD_OK) return FD_ERR_DEVICE;
+    const long long items = static_cast<long long>(rows) * (D / 4);
+    const long long blocks = (items + fd::kPartialsThreads - 1) / fd::kPartialsThreads;
+    fd::fd_merge_partials_kernel<<<static_cast<unsigned>(blocks), fd::kPartialsThreads, 0,
+                                   static_cast<cudaStream_t>(stream)>>>(part_out, part_lse, R, rows, D, out, lse);
+    if (cudaGetLastError() != cudaSuccess) return FD_ERR_LAUNCH;
+    return FD_OK;
 }
 
 int fd_decode_static(int B, int Hq, int Hkv, int D, int max_len, const uint16_t *q, const uint16_t *k_cache,

@@ -180,6 +180,25 @@ FD_API int fd_decode_quant(int B, int q_len, int Hq, int Hkv, int D, int max_len
                            float *out, float *lse, void *workspace, size_t workspace_bytes, int num_splits,
                            void *stream);
 
+/* The final reduction over R partial results per row computed elsewhere,
+ * e.g. one per GPU when a long sequence is sharded along its tokens across
+ * GPUs (context parallelism; the DISTFLASHATTN abstract on the "Related
+ * papers: Glinthawk" page distributes attention over GPUs along the
+ * sequence). Part r of row i is (part_out[r][i][0..D), part_lse[r][i]), the
+ * normalised output and natural-log log-sum-exp of the row's attention over
+ * that part's tokens, as fd_decode writes them. Writes
+ *     lse[i] = log sum_r exp(part_lse[r][i]),
+ *     out[i] = sum_r exp(part_lse[r][i] - lse[i]) * part_out[r][i]
+ * ("Flash-Decoding for long-context inference", section "A faster attention
+ * for decoding: Flash-Decoding", the final reduction), parts in increasing r
+ * (deterministic). Parts with lse = -inf weigh 0; a row with no non-empty part
+ * gets out = 0, lse = -inf. part_out / out: fp32, device, 16-byte aligned;
+ * part_lse / lse: fp32, device, 4-byte aligned; out may not overlap the
+ * parts. R >= 1, rows >= 0 (0: nothing to do, no CUDA call), D a multiple
+ * of 4 in [4, 4096]. Asynchronous on `stream`. */
+FD_API int fd_merge_partials(int R, int rows, int D, const float *part_out, const float *part_lse,
+                             float *out, float *lse, void *stream);
+
 /* fd_decode_splits over a PAGED key/value cache. The page pools
  * k_pages / v_pages hold num_pages pages of page_size tokens each, laid out
  * head-major (kv_layout = FD_KV_HND: [num_pages][Hkv][page_size][D] bf16) or

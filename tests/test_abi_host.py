@@ -180,6 +180,24 @@ def test_quant_argument_errors_without_a_device():
         assert quant() == -8 and quant(kv_type=2, q_len=2) == -8
 
 
+def test_merge_partials_argument_errors_without_a_device():
+    L = fd.lib()
+    buf = (ctypes.c_uint8 * 4096)()
+    a16 = (ctypes.addressof(buf) + 15) // 16 * 16
+    p = ctypes.c_void_p(a16)
+
+    def merge(R=2, rows=3, D=128, po=p, out=p, pl=p):
+        return L.fd_merge_partials(R, rows, D, po, pl, out, p, None)
+
+    assert merge(R=0) == -2 and merge(rows=-1) == -2
+    assert merge(D=6) == -4 and merge(D=0) == -4 and merge(D=8192) == -4
+    assert merge(rows=0, po=None) == 0                      # nothing to merge: no pointer read, no CUDA call
+    assert merge(po=None) == -1 and merge(pl=None) == -1
+    assert merge(out=ctypes.c_void_p(a16 + 4)) == -5 and merge(pl=ctypes.c_void_p(a16 + 2)) == -5
+    if not os.path.exists("/dev/nvidia0"):
+        assert merge() == -8
+
+
 def segments_rule(B, Hkv, Lmax, seqlens, P):
     """Independent statement of the documented partition: rows u = b*Hkv + j
     in order, ceil(L_b/64) tiles each, run i = flat tiles
