@@ -457,6 +457,98 @@ def run_fd(args, w, rank, world):
     return 0
 
 
+def run_cp(args, w, rank, world):
+    """Context parallelism: one batch whose cache is sharded along its token
+    positions over the `world` ranks. A step is the local split-kernel decode
+    of this rank's range, the all-gather of the (out, lse) partials and their
+    merge; total work is fixed as ranks are added (strong scaling)."""
+    from decode_attention_07_b200 import context
+    from decode_attention_07_b200.inputs import draw_seqlens
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    lo, hi = context.token_range(w.Lmax, rank, world)
+    ws_ = w.with_(Lmax=hi - lo)
+    lens = draw_seqlens(w, args.seed)                                     # the same batch on every rank
+    local = np.clip(lens.astype(np.int64) - lo, 0, hi - lo).astype(np.int32)
+    gq = torch.Generator(device=dev).manual_seed(args.seed)              # the same query on every rank
+    q = (torch.randn((w.B, w.Hq, w.D), generator=gq, device=dev) * w.sigma_q).to(torch.bfloat16)
+    xs = [make_inputs(ws_, args.seed + 1000 * c + rank, device=dev, seqlens=local) for c in range(2)]
+    for x in xs:
+        x.q = q
+    n_copies = 2 if xs[0].kv_bytes() >= L2_BYTES else 1
+    S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, ws_.Lmax)
+    nbytes = fd.fd_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, ws_.Lmax, S)
+    wsb = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    part_o = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
+    part_l = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    all_o = torch.empty((world, w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
+    all_l = torch.empty((world, w.B, w.Hq), dtype=torch.float32, device=dev)
+    out = torch.empty_like(part_o)
+    lse = torch.empty_like(part_l)
+    calls = [fd.prepare_decode(x.q, x.k, x.v, x.seqlens, x.scale, part_o, part_l, wsb, S, stream)
+             for x in xs[:n_copies]]
+    flush = None if n_copies == 2 else torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step(i):
+        calls[i % n_copies]()
+        if world > 1:
+            torch.distributed.all_gather_into_tensor(all_o, part_o)
+            torch.distributed.all_gather_into_tensor(all_l, part_l)
+            fd.fd_merge_partials(all_o, all_l, out, lse, stream)
+        else:
+            fd.fd_merge_partials(part_o[None], part_l[None], out, lse, stream)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps if flush is not None else 1)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        if flush is None:
+            ev[0][0].record(stream)
+            for i in range(args.steps):
+                step(i)
+            ev[0][1].record(stream)
+        else:
+            for i in range(args.steps):
+                flush.fill_(i & 255)
+                ev[i][0].record(stream)
+                step(i)
+                ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    ms_max = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev)
+    status = fd.fd_device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {fd.fd_strerror(status)}")
+    if rank != 0:
+        return 0
+    total_kv = int(np.clip(lens, 0, w.Lmax).astype(np.int64).sum()) * w.Hkv * w.D * 2 * 2
+    gbs = total_kv * args.steps / (ms_max * 1e-3) / 1e9
+    peak, peak_kind = peaks()
+    line = {
+        "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_max / args.steps, "us_per_call": ms_max * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_dict(w, S, "inputs larger than L2: 2 shard copies rotated" if n_copies == 2
+                                   else "L2 flushed before every timed step (256 MiB write outside the events)"),
+                       parallelism=f"cp{world}", shard_tokens=hi - lo),
+        "roofline": {"kernel": "whole step per rank (split kernel + all-gather + merge)", "bound": "hbm",
+                     "achieved": gbs / world, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": gbs / world / peak, "traffic": None},
+        "gpu_launches": args.steps * 2,
+        "clocks": clocks.summary(),
+        "e2e": None,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -471,6 +563,8 @@ def main():
     ap.add_argument("--paged", type=int, default=0, metavar="PAGE_SIZE",
                     help="read the caches from a shuffled page pool with this page size (fd_decode_paged)")
     ap.add_argument("--layout", choices=["HND", "NHD"], default="HND", help="page layout for --paged")
+    ap.add_argument("--cp", action="store_true",
+                    help="context parallelism: shard the cache's tokens over the ranks (strong scaling)")
     ap.add_argument("--kv", choices=["bf16", "e4m3", "int8"], default="bf16",
                     help="key/value cache element type; e4m3 / int8 use fd_decode_quant with per-head scales")
     ap.add_argument("--q-len", type=int, default=1,
@@ -480,6 +574,8 @@ def main():
     args = ap.parse_args()
     if args.paged and (args.kv != "bf16" or args.q_len != 1):
         ap.error("--paged reads a bf16 cache with one query per sequence")
+    if args.cp and (args.paged or args.kv != "bf16" or args.q_len != 1):
+        ap.error("--cp shards a contiguous bf16 cache with one query per sequence")
     w = WORKLOADS[args.config]
     world = int(os.environ.get("WORLD_SIZE", 1))
     rank = int(os.environ.get("RANK", 0))
@@ -490,6 +586,8 @@ def main():
     try:
         if args.impl == "reference":
             return run_reference(args, w, rank, world)
+        if args.cp:
+            return run_cp(args, w, rank, world)
         return run_fd(args, w, rank, world)
     finally:
         if world > 1 and torch.distributed.is_initialized():
