@@ -185,6 +185,47 @@ int encode_paged_map(CUtensorMap *map, const void *base, int D, int page_size, i
     return r == CUDA_SUCCESS ? FD_OK : FD_ERR_LAUNCH;
 }
 
+// Small pages at D = 128 (page_size < 64): each 256-byte token row viewed as
+// two 128-byte halves, so one box brings a whole page of one kv head,
+// [token][half][128 B] with the 128-byte swizzle. Head-major pages:
+// {64, 2, page_size, Hkv, num_pages}, box {64, 2, page_size, 1, 1}; token-major:
+// {64, 2, Hkv, page_size, num_pages}, box {64, 2, 1, page_size, 1}.
+int encode_paged_map_rows(CUtensorMap *map, const void *base, int page_size, int Hkv, long long num_pages, bool nhd) {
+    auto fn = encode_fn();
+    if (!fn) return FD_ERR_LAUNCH;
+    const cuuint64_t row = 256;   // bytes of one token of one head (D = 128, bf16)
+    cuuint64_t dims[5], strides[4];
+    cuuint32_t box[5];
+    dims[0] = 64;
+    dims[1] = 2;
+    dims[4] = static_cast<cuuint64_t>(num_pages);
+    strides[0] = 128;
+    box[0] = 64;
+    box[1] = 2;
+    box[4] = 1;
+    if (nhd) {
+        dims[2] = static_cast<cuuint64_t>(Hkv);
+        dims[3] = static_cast<cuuint64_t>(page_size);
+        strides[1] = row;
+        strides[2] = static_cast<cuuint64_t>(Hkv) * row;
+        box[2] = 1;
+        box[3] = static_cast<cuuint32_t>(page_size);
+    } else {
+        dims[2] = static_cast<cuuint64_t>(page_size);
+        dims[3] = static_cast<cuuint64_t>(Hkv);
+        strides[1] = row;
+        strides[2] = static_cast<cuuint64_t>(page_size) * row;
+        box[2] = static_cast<cuuint32_t>(page_size);
+        box[3] = 1;
+    }
+    strides[3] = static_cast<cuuint64_t>(page_size) * Hkv * row;
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FD_OK : FD_ERR_LAUNCH;
+}
+
 // ---------------------------------------------------------------- launches --
 template <int D, class Consumer, bool kFused, bool kPaged>
 int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p, cudaStream_t st) {
@@ -372,8 +413,14 @@ int run_split_paged(const Problem &pr, const PagedLayout &pl) {
     int rc = device_sms(&sms);
     if (rc != FD_OK) return rc;
     CUtensorMap tk, tv;
-    if ((rc = encode_paged_map(&tk, pr.k, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
-    if ((rc = encode_paged_map(&tv, pr.v, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
+    const bool rows_map = pr.D == 128 && pl.page_size < fd::kTileTokens;   // one box per small page
+    if (rows_map) {
+        if ((rc = encode_paged_map_rows(&tk, pr.k, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
+        if ((rc = encode_paged_map_rows(&tv, pr.v, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
+    } else {
+        if ((rc = encode_paged_map(&tk, pr.k, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
+        if ((rc = encode_paged_map(&tv, pr.v, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
+    }
     fd::SplitParams p;
     p.q = pr.q;
     p.seqlens = pr.seqlens;
@@ -395,6 +442,11 @@ int run_split_paged(const Problem &pr, const PagedLayout &pl) {
     while ((1 << p.page_shift) < pl.page_size) ++p.page_shift;
     p.kv_nhd = pl.nhd ? 1 : 0;
     p.k_scale = p.v_scale = nullptr;
+    if (rows_map) {
+        if (p.g == 1) return launch_split_t<128, fd::HeadConsumer<128, true>, true, true>(tk, tv, p, pr.stream);
+        if (p.g <= 8) return launch_split_t<128, fd::GroupConsumer<128, 1, true>, true, true>(tk, tv, p, pr.stream);
+        return launch_split_t<128, fd::GroupConsumer<128, 2, true>, true, true>(tk, tv, p, pr.stream);
+    }
     return launch_split<true, true>(pr.D, p.g, tk, tv, p, pr.stream);
 }
 

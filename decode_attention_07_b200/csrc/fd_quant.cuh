@@ -55,6 +55,7 @@ template <int D, int NT, bool kE4M3>
 struct QuantConsumer {
     static constexpr int G = 8 * NT;        // columns held (padded)
     static constexpr int kElemBytes = 1;
+    static constexpr bool kInterleaved = false;
     static constexpr int KC = D / 16;       // 16-byte chunks of a token = k-steps of S = m-tiles of O^T
     static constexpr int kRowBytes = D;
     // The reference max lags the running max by at most kLazy (base 2), so

@@ -93,6 +93,22 @@ struct SplitParams {
 
 constexpr int kPageWindow = 1024;                 // block-table entries staged in shared memory
 
+// Byte offset, inside a K or V tile, of 16-byte chunk j (0..7) of the
+// 64-element half `half` of token t. Default layout (one TMA box per half):
+// [half][64 tokens][128 B]. Interleaved layout (one box covers both halves
+// of a token, used for small pages at D = 128): [64 tokens][half][128 B].
+// Either way a 128-byte row R keeps the 128-byte swizzle: chunk j sits at
+// position j ^ (R & 7).
+template <bool kInter>
+__device__ __forceinline__ uint32_t tile_offset(int t, int half, int j) {
+    if constexpr (kInter) {
+        const int R = 2 * t + half;
+        return static_cast<uint32_t>(R * 128 + ((j ^ (R & 7)) << 4));
+    } else {
+        return static_cast<uint32_t>(half * kBoxBytes + t * 128 + ((j ^ (t & 7)) << 4));
+    }
+}
+
 // Output row of column `col` of row (b, h): column col = j*g + i is query j,
 // query head h*g + i; out is [B, q_len, Hq, D] and lse [B, q_len, Hq].
 __device__ __forceinline__ size_t out_row(const SplitParams &p, int b, int h, int col) {
@@ -308,12 +324,13 @@ __device__ __forceinline__ void merge_warps_and_store(const float *merge, float 
 }
 
 // ------------------------------------------------- grouped-head consumer --
-template <int D, int NT>
+template <int D, int NT, bool kInter = false>
 struct GroupConsumer {
     static constexpr int KS = D / 16;   // k-steps of the logit contraction
     static constexpr int MT = D / 16;   // m-tiles of the P V contraction
     static constexpr int G = 8 * NT;    // heads held (padded)
     static constexpr int kElemBytes = 2;
+    static constexpr bool kInterleaved = kInter;
 
     uint32_t qf[NT][KS][2];             // Q^T as the B operand, per n-tile
     float m[NT][2], l[NT][2];           // running max (base 2) / partial sum for heads 2c, 2c+1
@@ -383,7 +400,7 @@ struct GroupConsumer {
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
             const int d = 16 * ks + 8 * (mi >> 1);
-            const uint32_t addr = k_smem + (d >> 6) * kBoxBytes + krow * 128 + ((((d & 63) >> 3) ^ rr) << 4);
+            const uint32_t addr = k_smem + tile_offset<kInter>(krow, d >> 6, (d & 63) >> 3);
             uint32_t a0, a1, a2, a3;
             ldsm_x4(addr, a0, a1, a2, a3);
 #pragma unroll
@@ -442,7 +459,7 @@ struct GroupConsumer {
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
             const int d = 16 * mt + 8 * (mi & 1);
-            const uint32_t addr = v_smem + (d >> 6) * kBoxBytes + vrow * 128 + ((((d & 63) >> 3) ^ rr) << 4);
+            const uint32_t addr = v_smem + tile_offset<kInter>(vrow, d >> 6, (d & 63) >> 3);
             uint32_t a0, a1, a2, a3;
             ldsm_x4_trans(addr, a0, a1, a2, a3);
             if (valid < kWarpTokens) {   // rows past the end may hold anything (NaN): zero them
@@ -488,10 +505,11 @@ struct GroupConsumer {
 };
 
 // ------------------------------------------------ one-head (MHA) consumer --
-template <int D>
+template <int D, bool kInter = false>
 struct HeadConsumer {
     static constexpr int G = 1;
     static constexpr int kElemBytes = 2;
+    static constexpr bool kInterleaved = kInter;
     static constexpr int LPT = D / 8;          // lanes per token (16 bytes = 8 bf16 each)
     static constexpr int TPI = 32 / LPT;       // tokens per warp-wide load
     static constexpr int ITER = kWarpTokens / TPI;
@@ -535,15 +553,14 @@ struct HeadConsumer {
         const int lane = threadIdx.x & 31;
         const int half = lane / LPT, chunk = lane % LPT;
         const int d0 = 8 * chunk;
-        const uint32_t col = (d0 >> 6) * kBoxBytes;
-        const int j = (d0 & 63) >> 3;
+        const int dhalf = d0 >> 6, j = (d0 & 63) >> 3;   // 64-element half of the head dims, chunk in it
 
         // partial dots over this lane's 8 dims for tokens TPI*it + half
         float pd[ITER];
 #pragma unroll
         for (int it = 0; it < ITER; ++it) {
             const int r = kWarpTokens * slice + TPI * it + half;
-            const uint4 w = lds128(k_smem + col + r * 128 + ((j ^ (r & 7)) << 4));
+            const uint4 w = lds128(k_smem + tile_offset<kInter>(r, dhalf, j));
             float a = qv[0] * bf16lo_to_f32(w.x);
             a = fmaf(qv[1], bf16hi_to_f32(w.x), a);
             a = fmaf(qv[2], bf16lo_to_f32(w.y), a);
@@ -591,7 +608,7 @@ struct HeadConsumer {
             const int t = TPI * it + half;
             if (t < valid) {
                 const int r = kWarpTokens * slice + t;
-                const uint4 w = lds128(v_smem + col + r * 128 + ((j ^ (r & 7)) << 4));
+                const uint4 w = lds128(v_smem + tile_offset<kInter>(r, dhalf, j));
                 acc[0] = fmaf(pt, bf16lo_to_f32(w.x), acc[0]);
                 acc[1] = fmaf(pt, bf16hi_to_f32(w.x), acc[1]);
                 acc[2] = fmaf(pt, bf16lo_to_f32(w.y), acc[2]);
@@ -762,18 +779,31 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                     int page[kTileTokens / 8];
                     for (int j = 0; j < nsub; ++j)
                         if (!page_of(c.b, lp0 + j, &page[j])) return;
-                    const uint32_t sub_bytes = static_cast<uint32_t>(rows) * 128u;
-                    mbar_arrive_expect_tx(&full[stage], 2u * nsub * sub_bytes * Cfg::kBoxes + qb);
-                    for (int j = 0; j < nsub; ++j) {
+                    if constexpr (Consumer::kInterleaved) {
+                        // one 5-D box per page, both halves of its tokens: [token][half][128 B].
+                        // Coordinates {element, half, token, head, page} (head-major pages)
+                        // or {element, half, head, token, page} (token-major pages).
+                        const uint32_t page_bytes = static_cast<uint32_t>(rows) * D * 2;
+                        mbar_arrive_expect_tx(&full[stage], 2u * nsub * page_bytes + qb);
+                        const int cz = p.kv_nhd ? c.h : off, cw = p.kv_nhd ? off : c.h;
+                        for (int j = 0; j < nsub; ++j) {
+                            tma_load_5d(kt + j * page_bytes, &tm_k, &full[stage], 0, 0, cz, cw, page[j], policy);
+                            tma_load_5d(vt + j * page_bytes, &tm_v, &full[stage], 0, 0, cz, cw, page[j], policy);
+                        }
+                    } else {
+                        const uint32_t sub_bytes = static_cast<uint32_t>(rows) * 128u;
+                        mbar_arrive_expect_tx(&full[stage], 2u * nsub * sub_bytes * Cfg::kBoxes + qb);
+                        for (int j = 0; j < nsub; ++j) {
 #pragma unroll
-                        for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-                            const int dst = bx * kBoxBytes + j * rows * 128;
-                            if (p.kv_nhd) {
-                                tma_load_4d(kt + dst, &tm_k, &full[stage], 64 * bx, c.h, off, page[j], policy);
-                                tma_load_4d(vt + dst, &tm_v, &full[stage], 64 * bx, c.h, off, page[j], policy);
-                            } else {
-                                tma_load_4d(kt + dst, &tm_k, &full[stage], 64 * bx, off, c.h, page[j], policy);
-                                tma_load_4d(vt + dst, &tm_v, &full[stage], 64 * bx, off, c.h, page[j], policy);
+                            for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+                                const int dst = bx * kBoxBytes + j * rows * 128;
+                                if (p.kv_nhd) {
+                                    tma_load_4d(kt + dst, &tm_k, &full[stage], 64 * bx, c.h, off, page[j], policy);
+                                    tma_load_4d(vt + dst, &tm_v, &full[stage], 64 * bx, c.h, off, page[j], policy);
+                                } else {
+                                    tma_load_4d(kt + dst, &tm_k, &full[stage], 64 * bx, off, c.h, page[j], policy);
+                                    tma_load_4d(vt + dst, &tm_v, &full[stage], 64 * bx, off, c.h, page[j], policy);
+                                }
                             }
                         }
                     }
