@@ -439,7 +439,7 @@ def run_fd(args, w, rank, world):
         "call_bytes_gbs": world * counts["total"] * args.steps / (ms_max * 1e-3) / 1e9,
         "roofline": {"kernel": "fd_split_kernel (fused combine)" + (f", {args.kv} cache" if quant else ""), "bound": "hbm", "achieved": kernel_gbs,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": kernel_gbs / peak,
-                     "traffic": None if args.paged or Q > 1 or quant else measured_traffic(w.name),
+                     "traffic": None if args.paged or Q > 1 else measured_traffic(w.name + (f":{args.kv}" if quant else "")),
                      "bytes_per_launch": counts["total"],
                      "us_per_launch": us_per_call,
                      "frac_of_nominal_8tbs": kernel_gbs / NOMINAL_HBM_GBS},
