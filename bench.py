@@ -36,14 +36,19 @@ NOMINAL_HBM_GBS = 8000.0
 L2_BYTES = 126 * 1024 * 1024
 
 
+# The sources that define the split kernel and its launch (tile sizes, ring,
+# consumers, grid): DRAM traffic recorded for one hash is valid while they
+# are unchanged.
+SPLIT_KERNEL_SOURCES = ("fd_api.cu", "fd_merge.cuh", "fd_partition.cuh", "fd_ptx.cuh", "fd_quant.cuh",
+                        "fd_split.cuh")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources (decode_attention_07_b200/csrc/*, include/fd.h)."""
-    import glob
+    """Hash of the split kernel's CUDA sources (SPLIT_KERNEL_SOURCES)."""
     import hashlib
     h = hashlib.sha256()
-    files = sorted(glob.glob(os.path.join(ROOT, "decode_attention_07_b200", "csrc", "*")))
-    for f in files + [os.path.join(ROOT, "include", "fd.h")]:
-        with open(f, "rb") as fh:
+    for name in SPLIT_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "decode_attention_07_b200", "csrc", name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
@@ -257,6 +262,43 @@ def config_dict(w, S, l2):
 
 # ------------------------------------------------------------- the GPU arm --
 
+def read_probe_gbs(dev, stream, nbytes=2 << 30, reps=10):
+    """HBM read ceiling on this GPU: fd_read_probe over a buffer far larger
+    than L2, CUDA events around `reps` back-to-back passes."""
+    buf = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    sink = torch.zeros(1, dtype=torch.int64, device=dev)
+    for _ in range(2):
+        fd.fd_read_probe(buf, sink, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fd.fd_read_probe(buf, sink, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    gbs = nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    del buf
+    torch.cuda.empty_cache()
+    return gbs
+
+
+def per_call_stats(call_at, dev, stream, steps):
+    """Each call timed alone with CUDA events, L2 flushed before it by a
+    write of twice its size (outside the events): median, p10, p90 in us."""
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 255)
+        ev[i][0].record(stream)
+        call_at(i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    t = np.array([a.elapsed_time(b) * 1e3 for a, b in ev])
+    del flush
+    return {"median_us": float(np.median(t)), "p10_us": float(np.percentile(t, 10)),
+            "p90_us": float(np.percentile(t, 90)), "calls": steps,
+            "l2": "flushed before every call (write of 2x L2, outside the events)"}
+
+
 def run_fd(args, w, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
@@ -316,6 +358,7 @@ def run_fd(args, w, rank, world):
         if world > 1:
             torch.distributed.barrier()
 
+    probe = read_probe_gbs(dev, stream) if rank == 0 else None
     for i in range(max(3, args.warmup)):
         calls[i % n_copies]()
     torch.cuda.synchronize(dev)
@@ -354,6 +397,8 @@ def run_fd(args, w, rank, world):
     ms_max = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev)
     us_per_call = ms_max * 1e3 / args.steps
     gbs = whole_job_gbs(world, kv_bytes, args.steps, ms_max)
+
+    per_call = per_call_stats(lambda i: calls[i % n_copies](), dev, stream, max(10, min(args.steps, 50)))
 
     # ---- the two stages as separate kernels (for the per-stage split) ------
     ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -436,6 +481,9 @@ def run_fd(args, w, rank, world):
                        **({"q_len": Q} if Q > 1 else {})),
         "pct_of_nominal_hbm": 100.0 * gbs / world / NOMINAL_HBM_GBS,
         "pct_of_measured_copy": 100.0 * gbs / world / peak,
+        "read_probe": {"gbs": probe, "bytes": 2 << 30, "kernel": "fd_read_probe (bulk copies, 1 block per SM, 128 KiB in flight)"},
+        "pct_of_read_probe": 100.0 * gbs / world / probe if probe else None,
+        "per_call": per_call,
         "call_bytes_gbs": world * counts["total"] * args.steps / (ms_max * 1e-3) / 1e9,
         "roofline": {"kernel": "fd_split_kernel (fused combine)" + (f", {args.kv} cache" if quant else ""), "bound": "hbm", "achieved": kernel_gbs,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": kernel_gbs / peak,
@@ -451,8 +499,11 @@ def run_fd(args, w, rank, world):
     }
     if world == 1 and not args.no_cpu_baseline and not args.paged and Q == 1:   # bf16 or 8-bit cache
         b, s, t, desc = oracle_sample(xs[0], budget_s=args.cpu_seconds)
+        b1, s1, _, desc1 = oracle_sample(xs[0], budget_s=max(1.0, args.cpu_seconds / 4), nthreads=1)
         line["cpu_baseline"] = {"value": b / s / 1e9, "unit": "GB/s", "cores": t, "kind": "oracle",
-                                "sample": desc, "seconds": s}
+                                "sample": desc, "seconds": s,
+                                "single_thread": {"value": b1 / s1 / 1e9, "unit": "GB/s", "cores": 1,
+                                                  "sample": desc1, "seconds": s1}}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -59,12 +59,13 @@ def lib() -> ctypes.CDLL:
         L.fd_decode_multi.argtypes = [_i] * 6 + [_p, _p, _p, _p, _f, _p, _p, _p, _sz, _i, _p]
         L.fd_decode_quant.argtypes = [_i] * 7 + [_p, _p, _p, _p, _p, _p, _f, _p, _p, _p, _sz, _i, _p]
         L.fd_merge_partials.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p]
+        L.fd_read_probe.argtypes = [_p, _sz, _p, _p]
         L.fd_strerror.argtypes = [_i]
         L.fd_strerror.restype = ctypes.c_char_p
         L.fd_version.argtypes = []
         for name in ("fd_plan", "fd_plan_for_sms", "fd_decode", "fd_decode_splits", "fd_split", "fd_combine",
                      "fd_segments", "fd_device_status", "fd_version", "fd_workspace_init", "fd_decode_static",
-                     "fd_decode_paged", "fd_decode_multi", "fd_decode_quant", "fd_merge_partials"):
+                     "fd_decode_paged", "fd_decode_multi", "fd_decode_quant", "fd_merge_partials", "fd_read_probe"):
             getattr(L, name).restype = _i
         _lib = L
     return _lib
@@ -444,6 +445,16 @@ def fd_merge_partials(part_out, part_lse, out, lse, stream=None):
             raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor")
     _check(lib().fd_merge_partials(R, rows, D, part_out.data_ptr(), part_lse.data_ptr(), out.data_ptr(),
                                    lse.data_ptr(), _stream(stream, out.device)), "fd_merge_partials")
+
+
+def fd_read_probe(buf, sink, stream=None):
+    """Read every byte of the CUDA tensor `buf` once (HBM read-bandwidth
+    probe); `sink` is a one-element int64 CUDA tensor."""
+    if not buf.is_cuda or not buf.is_contiguous() or sink.dtype != torch.int64 or not sink.is_cuda:
+        raise ValueError("buf must be a contiguous CUDA tensor and sink an int64 CUDA tensor")
+    nbytes = buf.numel() * buf.element_size()
+    _check(lib().fd_read_probe(buf.data_ptr(), nbytes, sink.data_ptr(), _stream(stream, buf.device)),
+           "fd_read_probe")
 
 
 def workspace_layout(B, Hq, Hkv, D, num_splits):

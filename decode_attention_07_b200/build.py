@@ -8,7 +8,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libfdecode.so")
-SOURCES = [os.path.join(CSRC, "fd_api.cu")]
+SOURCES = [os.path.join(CSRC, "fd_api.cu"), os.path.join(CSRC, "fd_probe.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + \
     [os.path.join(INCLUDE, "fd.h")]
 

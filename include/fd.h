@@ -199,6 +199,18 @@ FD_API int fd_decode_quant(int B, int q_len, int Hq, int Hkv, int D, int max_len
 FD_API int fd_merge_partials(int R, int rows, int D, const float *part_out, const float *part_lse,
                              float *out, float *lse, void *stream);
 
+/* Measurement utility, not part of the attention (the pages have no
+ * counterpart): reads `bytes` of device memory at `buf` once, streaming it
+ * the way the split kernel does (one block per SM, 32 KiB bulk copies into a
+ * 4-stage shared-memory ring, chunks round-robin over the blocks) with no
+ * compute. Timing it over a buffer larger than L2 gives the HBM read ceiling
+ * the decode kernels are compared with. The first 32-bit word of every
+ * 32 KiB chunk is xor-folded into the low half of *sink (device, 8-byte
+ * aligned, zero on entry) so the copies cannot be elided; the high half is
+ * set to 1 if a bounded wait gave up (2 s). buf 16-byte aligned, bytes a
+ * multiple of 16 (0: nothing). Asynchronous on `stream`. */
+FD_API int fd_read_probe(const void *buf, size_t bytes, unsigned long long *sink, void *stream);
+
 /* fd_decode_splits over a PAGED key/value cache. The page pools
  * k_pages / v_pages hold num_pages pages of page_size tokens each, laid out
  * head-major (kv_layout = FD_KV_HND: [num_pages][Hkv][page_size][D] bf16) or

@@ -198,6 +198,19 @@ def test_merge_partials_argument_errors_without_a_device():
         assert merge() == -8
 
 
+def test_read_probe_argument_errors_without_a_device():
+    L = fd.lib()
+    buf = (ctypes.c_uint8 * 4096)()
+    a16 = (ctypes.addressof(buf) + 15) // 16 * 16
+    p = ctypes.c_void_p(a16)
+    assert L.fd_read_probe(p, 0, None, None) == 0          # nothing to read: no pointer used, no CUDA call
+    assert L.fd_read_probe(None, 64, p, None) == -1 and L.fd_read_probe(p, 64, None, None) == -1
+    assert L.fd_read_probe(ctypes.c_void_p(a16 + 4), 64, p, None) == -5
+    assert L.fd_read_probe(p, 24, p, None) == -5 and L.fd_read_probe(p, 64, ctypes.c_void_p(a16 + 4), None) == -5
+    if not os.path.exists("/dev/nvidia0"):
+        assert L.fd_read_probe(p, 64, p, None) == -8
+
+
 def segments_rule(B, Hkv, Lmax, seqlens, P):
     """Independent statement of the documented partition: rows u = b*Hkv + j
     in order, ceil(L_b/64) tiles each, run i = flat tiles

@@ -87,3 +87,21 @@ def test_sharded_headline_workload():
     out, lse = sharded_decode(x, 8)
     ref_o, ref_l = oracle_rows(x)
     compare(out, lse, ref_o, ref_l, "mha_16k over 8 token ranges")
+
+
+def test_read_probe_reads_every_chunk():
+    """The bandwidth probe folds the first 32-bit word of every 32 KiB chunk
+    with xor: its result must equal that fold computed on the host (sizes
+    with a short last chunk, fewer chunks than SMs, many per SM)."""
+    import numpy as np
+    for n_words in (4, 1000 * 4, (1 << 22) + 12, (1 << 25) + 4):
+        g = torch.Generator(device="cpu").manual_seed(n_words)
+        host = torch.randint(-2**31, 2**31 - 1, (n_words,), generator=g, dtype=torch.int64).to(torch.int32)
+        sink = torch.zeros(1, dtype=torch.int64, device="cuda")
+        fd.fd_read_probe(host.cuda(), sink)
+        torch.cuda.synchronize()
+        words = host.numpy().view(np.uint32)[::32768 // 4]
+        want = int(np.bitwise_xor.reduce(words))
+        got = int(sink.item())
+        assert got >> 32 == 0, "a bounded wait gave up"
+        assert got & 0xFFFFFFFF == want
