@@ -160,12 +160,13 @@ def byte_counts(w, lens, S, q_len=1, elem_bytes=2):
 
 # ------------------------------------------------------------- the CPU arm --
 
-def oracle_sample(x, budget_s=12.0, nthreads=0):
+def oracle_sample(x, budget_s=12.0, nthreads=0, collect=None):
     """Time the CPU oracle on a bounded sample of the workload: whole
     sequences (all kv heads and query heads; the oracle spreads the rows over
     the host cores), longest first, until about `budget_s` seconds of work;
     a sequence too long for the budget is cut to its first kv heads.
-    Returns (kv_bytes_processed, seconds, threads, description)."""
+    Returns (kv_bytes_processed, seconds, threads, description); with a list
+    `collect`, appends (b, first query head, oracle out, oracle lse) per call."""
     import oracle
     w = x.workload
     orc = oracle.default()
@@ -187,13 +188,16 @@ def oracle_sample(x, budget_s=12.0, nthreads=0):
                 vh = x.v8[b:b + 1, j0:j1, :L].cpu().numpy()
                 ks, vs = x.k_scale[j0:j1].cpu().numpy(), x.v_scale[j0:j1].cpu().numpy()
                 t0 = time.perf_counter()
-                orc.attention_quant(qh, kh, vh, ks, vs, np.array([L], np.int32), x.scale, x.kv_type, nthreads)
+                o, lo = orc.attention_quant(qh, kh, vh, ks, vs, np.array([L], np.int32), x.scale, x.kv_type,
+                                            nthreads)
             else:
                 kh = bf16_bits(x.k[b:b + 1, j0:j1, :L])
                 vh = bf16_bits(x.v[b:b + 1, j0:j1, :L])
                 t0 = time.perf_counter()
-                orc.attention(qh, kh, vh, np.array([L], np.int32), x.scale, nthreads)
+                o, lo = orc.attention(qh, kh, vh, np.array([L], np.int32), x.scale, nthreads)
             spent += time.perf_counter() - t0
+            if collect is not None:
+                collect.append((int(b), j0 * w.g, o[0], lo[0]))
             threads = max(threads, orc.threads_used)
             done_bytes += (j1 - j0) * L * w.D * elem * 2
             rows += j1 - j0
@@ -498,7 +502,22 @@ def run_fd(args, w, rank, world):
         "wall_s": wall,
     }
     if world == 1 and not args.no_cpu_baseline and not args.paged and Q == 1:   # bf16 or 8-bit cache
-        b, s, t, desc = oracle_sample(xs[0], budget_s=args.cpu_seconds)
+        rows = []
+        b, s, t, desc = oracle_sample(xs[0], budget_s=args.cpu_seconds, collect=rows)
+        # parity of the timed path on the same sample: one more call on the first input copy
+        calls[0]()
+        torch.cuda.synchronize(dev)
+        o_gpu, l_gpu = out.double().cpu().numpy(), lse.double().cpu().numpy()
+        err_o, err_l = 0.0, 0.0
+        for bb, h0, o_ref, l_ref in rows:
+            og, lg = o_gpu[bb, h0:h0 + o_ref.shape[0]], l_gpu[bb, h0:h0 + l_ref.shape[0]]
+            err_o = max(err_o, float(np.abs(og - o_ref).max()))
+            fin = np.isfinite(l_ref)
+            if fin.any():
+                err_l = max(err_l, float((np.abs(lg[fin] - l_ref[fin]) / np.maximum(1.0, np.abs(l_ref[fin]))).max()))
+        line["parity"] = {"max_abs_err_out": err_o, "max_rel_err_lse": err_l,
+                          "rows": sum(r[2].shape[0] for r in rows), "tolerance": {"out_abs": 2e-3, "lse_rel": 1e-4},
+                          "against": "oracle (fp64) on the cpu_baseline sample"}
         b1, s1, _, desc1 = oracle_sample(xs[0], budget_s=max(1.0, args.cpu_seconds / 4), nthreads=1)
         line["cpu_baseline"] = {"value": b / s / 1e9, "unit": "GB/s", "cores": t, "kind": "oracle",
                                 "sample": desc, "seconds": s,

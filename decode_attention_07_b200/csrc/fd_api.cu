@@ -226,6 +226,18 @@ int encode_paged_map_rows(CUtensorMap *map, const void *base, int page_size, int
     return r == CUDA_SUCCESS ? FD_OK : FD_ERR_LAUNCH;
 }
 
+// Host-side failure injection for tests: with FD_TEST_FAIL_LAUNCH set in the
+// environment (to anything but "0"), every kernel launch of the library is
+// skipped and reported as FD_ERR_LAUNCH, as a failed launch would be. Read
+// once per process.
+bool inject_launch_failure() {
+    static const bool fail = [] {
+        const char *v = std::getenv("FD_TEST_FAIL_LAUNCH");
+        return v != nullptr && v[0] != '\0' && !(v[0] == '0' && v[1] == '\0');
+    }();
+    return fail;
+}
+
 // ---------------------------------------------------------------- launches --
 template <int D, class Consumer, bool kFused, bool kPaged>
 int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p, cudaStream_t st) {
@@ -259,6 +271,7 @@ int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::Split
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (inject_launch_failure()) return FD_ERR_LAUNCH;
     if (cudaLaunchKernelEx(&cfg, kern, tk, tv, p) != cudaSuccess) {
         cudaGetLastError();
         return FD_ERR_LAUNCH;
@@ -303,6 +316,7 @@ int launch_combine(int D, const fd::CombineParams &p, cudaStream_t st, bool afte
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = after_split ? 1 : 0;
+    if (inject_launch_failure()) return FD_ERR_LAUNCH;
     cudaError_t e = D == 128 ? cudaLaunchKernelEx(&cfg, fd::fd_combine_kernel<128>, p)
                              : cudaLaunchKernelEx(&cfg, fd::fd_combine_kernel<64>, p);
     if (e != cudaSuccess) {
@@ -767,6 +781,7 @@ int fd_merge_partials(int R, int rows, int D, const float *part_out, const float
     if (current_device(&dev) != FD_OK) return FD_ERR_DEVICE;
     const long long items = static_cast<long long>(rows) * (D / 4);
     const long long blocks = (items + fd::kPartialsThreads - 1) / fd::kPartialsThreads;
+    if (inject_launch_failure()) return FD_ERR_LAUNCH;
     fd::fd_merge_partials_kernel<<<static_cast<unsigned>(blocks), fd::kPartialsThreads, 0,
                                    static_cast<cudaStream_t>(stream)>>>(part_out, part_lse, R, rows, D, out, lse);
     if (cudaGetLastError() != cudaSuccess) return FD_ERR_LAUNCH;
