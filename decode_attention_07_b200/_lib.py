@@ -10,6 +10,7 @@ import torch
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIBRARY = os.path.join(PKG, "libfdecode.so")
+DEBUG_LIBRARY = os.path.join(PKG, "libfdecode_debug.so")   # built with -DFD_DEBUG (device-side bounds checks)
 
 FD_OK = 0
 FD_TILE_TOKENS = 64
@@ -18,7 +19,7 @@ FD_MAX_GROUP = 16
 ERRORS = {
     -1: "FD_ERR_NULL_POINTER", -2: "FD_ERR_SHAPE", -3: "FD_ERR_GROUP", -4: "FD_ERR_HEAD_DIM",
     -5: "FD_ERR_ALIGNMENT", -6: "FD_ERR_WORKSPACE", -7: "FD_ERR_SPLITS", -8: "FD_ERR_DEVICE",
-    -9: "FD_ERR_LAUNCH", -10: "FD_ERR_TIMEOUT", -11: "FD_ERR_CAPACITY", -12: "FD_ERR_STATIC_LIMIT",
+    -9: "FD_ERR_LAUNCH", -10: "FD_ERR_TIMEOUT", -11: "FD_ERR_CAPACITY", -12: "FD_ERR_STATIC_LIMIT", -13: "FD_ERR_BOUNDS",
 }
 FD_STATIC_SCRATCH_BYTES = 8 << 20
 FD_KV_HND, FD_KV_NHD = 0, 1
@@ -36,12 +37,14 @@ _i, _p, _sz, _f = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
 
 
 def lib() -> ctypes.CDLL:
-    """Load libfdecode.so (built in-tree by decode_attention_07_b200.build)."""
+    """Load libfdecode.so (built in-tree by decode_attention_07_b200.build);
+    with FD_DEBUG=1 in the environment, the debug build libfdecode_debug.so."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIBRARY):
-            raise RuntimeError(f"{LIBRARY} is not built: run `python -c 'import __graft_entry__ as g; g.build()'`")
-        L = ctypes.CDLL(LIBRARY)
+        path = DEBUG_LIBRARY if os.environ.get("FD_DEBUG", "0") not in ("", "0") else LIBRARY
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is not built: run `python -c 'import __graft_entry__ as g; g.build()'`")
+        L = ctypes.CDLL(path)
         L.fd_plan.argtypes = [_i] * 5
         L.fd_plan_for_sms.argtypes = [_i] * 6
         L.fd_workspace_bytes.argtypes = [_i] * 6

@@ -8,6 +8,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libfdecode.so")
+DEBUG_LIBRARY = os.path.join(PKG, "libfdecode_debug.so")   # -DFD_DEBUG: device-side bounds checks
 SOURCES = [os.path.join(CSRC, "fd_api.cu"), os.path.join(CSRC, "fd_probe.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + \
     [os.path.join(INCLUDE, "fd.h")]
@@ -34,10 +35,11 @@ def up_to_date(out: str) -> bool:
     return all(os.path.getmtime(d) <= t for d in DEPS)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False, out: str = LIBRARY) -> str:
+def build(force: bool = False, verbose_ptxas: bool = False, out: str = None, debug: bool = False) -> str:
+    out = out or (DEBUG_LIBRARY if debug else LIBRARY)
     if not force and up_to_date(out):
         return out
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", out, *SOURCES]
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-DFD_DEBUG"] if debug else []), "-I", INCLUDE, "-I", CSRC, "-o", out, *SOURCES]
     if verbose_ptxas:
         cmd[1:1] = ["-Xptxas", "-v"]
     subprocess.run(cmd, check=True)
@@ -45,4 +47,4 @@ def build(force: bool = False, verbose_ptxas: bool = False, out: str = LIBRARY) 
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose_ptxas="-v" in sys.argv))
+    print(build(force=True, verbose_ptxas="-v" in sys.argv, debug="--debug" in sys.argv))

@@ -238,6 +238,18 @@ bool inject_launch_failure() {
     return fail;
 }
 
+// Debug builds: FD_DEBUG_WITHHOLD=<n> makes block 0 of the split kernel arm
+// the barrier of its n-th tile without issuing the copy, so a consumer's
+// bounded wait runs out (tests of the timeout path). Release builds: off.
+int debug_withhold() {
+#ifdef FD_DEBUG
+    const char *v = std::getenv("FD_DEBUG_WITHHOLD");
+    return v != nullptr ? std::atoi(v) : -1;
+#else
+    return -1;
+#endif
+}
+
 // ---------------------------------------------------------------- launches --
 template <int D, class Consumer, bool kFused, bool kPaged>
 int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p, cudaStream_t st) {
@@ -410,6 +422,7 @@ int run_split(const Problem &pr, bool fused, int q_len = 1) {
     p.page_shift = 0;
     p.kv_nhd = 0;
     p.k_scale = p.v_scale = nullptr;
+    p.debug_withhold = debug_withhold();
     // with max_len == 0 every block finds zero tiles and only writes empty rows;
     // the (unused) tensor maps stay zeroed
     return fused ? launch_split<true>(pr.D, p.cols, tk, tv, p, pr.stream)
@@ -456,6 +469,7 @@ int run_split_paged(const Problem &pr, const PagedLayout &pl) {
     while ((1 << p.page_shift) < pl.page_size) ++p.page_shift;
     p.kv_nhd = pl.nhd ? 1 : 0;
     p.k_scale = p.v_scale = nullptr;
+    p.debug_withhold = debug_withhold();
     if (rows_map) {
         if (p.g == 1) return launch_split_t<128, fd::HeadConsumer<128, true>, true, true>(tk, tv, p, pr.stream);
         if (p.g <= 8) return launch_split_t<128, fd::GroupConsumer<128, 1, true>, true, true>(tk, tv, p, pr.stream);
@@ -498,6 +512,7 @@ int run_split_quant(const Problem &pr, int q_len, int kv_type, const float *k_sc
     p.kv_nhd = 0;
     p.k_scale = k_scale;
     p.v_scale = v_scale;
+    p.debug_withhold = debug_withhold();
     return kv_type == FD_KV_E4M3 ? launch_split_quant<true>(pr.D, p.cols, tk, tv, p, pr.stream)
                                  : launch_split_quant<false>(pr.D, p.cols, tk, tv, p, pr.stream);
 }
@@ -861,6 +876,7 @@ const char *fd_strerror(int code) {
         case FD_ERR_CAPACITY: return "output arrays too small";
         case FD_ERR_STATIC_LIMIT:
             return "problem needs more scratch than fd_decode_static's fixed 8 MiB buffer; use fd_decode with a workspace";
+        case FD_ERR_BOUNDS: return "a debug build's device-side bounds check failed; outputs of that call are invalid";
         default: return "unknown error code";
     }
 }

@@ -54,6 +54,7 @@ __global__ void __launch_bounds__(kCombineThreads) fd_combine_kernel(const Combi
 
     // Everything below reads what the split grid wrote, or writes next to it.
     grid_dependency_wait();
+    if (!FD_DCHECK(row0 + p.g <= static_cast<size_t>(p.B) * p.Hq)) return;
 
     if (n_b == 0) {
         write_empty_row<D>(p.out + row0 * D, p.lse + row0, p.g, tid, kCombineThreads);
@@ -63,6 +64,9 @@ __global__ void __launch_bounds__(kCombineThreads) fd_combine_kernel(const Combi
     const long long first = before * p.Hkv + static_cast<long long>(h) * n_b;
     const RowRuns rr = row_runs(first, n_b, N, p.P);
     if (rr.i0 == rr.i1) return;   // one segment: the split stage wrote this row
+    if (!FD_DCHECK(static_cast<size_t>(rr.i1) + static_cast<size_t>(u) <
+                   static_cast<size_t>(p.P) + static_cast<size_t>(p.B) * p.Hkv - 1))
+        return;
     merge_row<D>(p.seg_out, p.seg_lse, p.g, u, rr, N, p.P, p.out + row0 * D, p.lse + row0, tid, kCombineThreads);
 }
 

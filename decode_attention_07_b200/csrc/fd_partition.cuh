@@ -22,6 +22,24 @@
 
 namespace fd {
 
+// Sticky per-device error word (FD_ERR_TIMEOUT when a wait gave up,
+// FD_ERR_BOUNDS when a debug build's bounds check failed).
+__device__ int g_fd_error_word;
+
+// Debug builds (-DFD_DEBUG) check the global accesses whose indices come
+// from the partition arithmetic; a failed check records FD_ERR_BOUNDS and
+// the access is skipped. Release builds compile the checks away.
+__device__ __forceinline__ bool debug_check(bool ok) {
+    if (!ok) atomicExch(&g_fd_error_word, -13 /* FD_ERR_BOUNDS */);
+    return ok;
+}
+#ifdef FD_DEBUG
+#define FD_DCHECK(cond) ::fd::debug_check(cond)
+#else
+#define FD_DCHECK(cond) true
+#endif
+
+
 constexpr int kTileTokens = 64;
 
 __host__ __device__ __forceinline__ int clamp_len(int L, int Lmax) {

@@ -64,10 +64,13 @@ constexpr int kPrefetchTiles = 8;                 // tiles guessed into L2 befor
 constexpr int kWarpTokens = 16;                   // tokens of a tile owned by one consumer warp
 constexpr int kBoxBytes = kTileTokens * 128;      // one TMA box: 64 rows x 128 bytes (64 bf16)
 constexpr int kSmemLimit = 232448;                // 227 KiB opt-in shared memory per block
+#ifdef FD_DEBUG
+constexpr uint64_t kWaitLimitNs = 50000000ull;    // debug builds: a bounded wait gives up after 50 ms
+#else
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a bounded wait gives up after 2 s
+#endif
 
-// Sticky per-device error word (FD_ERR_TIMEOUT when a wait gave up).
-__device__ int g_fd_error_word;
+
 
 struct SplitParams {
     const uint16_t *q;        // [B, Hq, D]
@@ -89,7 +92,16 @@ struct SplitParams {
     // 8-bit caches only: value of a cached element = scale[kv head] * decode(code)
     const float *k_scale;     // [Hkv]
     const float *v_scale;     // [Hkv]
+    int debug_withhold;       // debug builds: block 0 issues no copy for this tile (a wait then runs out); -1: off
 };
+
+// Sizes the debug checks compare with.
+__device__ __forceinline__ size_t out_rows(const SplitParams &p) {
+    return static_cast<size_t>(p.B) * p.q_len * p.Hq;
+}
+__device__ __forceinline__ size_t seg_rows(const SplitParams &p) {
+    return (static_cast<size_t>(p.P) + static_cast<size_t>(p.B) * p.Hkv - 1) * p.cols;
+}
 
 constexpr int kPageWindow = 1024;                 // block-table entries staged in shared memory
 
@@ -185,6 +197,28 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
             return false;
         }
     }
+}
+
+// After a wait gave up: wait once more, bounded and regardless of the abort
+// flag, for a phase whose copies were issued, so that no copy still lands in
+// this block's shared memory after it exits.
+__device__ __forceinline__ void drain_phase(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_timer_ns() - t0 > kWaitLimitNs) return;
+}
+
+// The producer's copies still possibly in flight when it gives up: the last
+// load issued into each stage (`issued` tiles so far, stage = tile % stages)
+// and the block-table window (when `window_pending`).
+template <int kStages>
+__device__ __forceinline__ void drain_copies(uint64_t *full, uint32_t issued, uint64_t *pbar, bool window_pending,
+                                             uint32_t win_phase) {
+    for (uint32_t s = 0; s < static_cast<uint32_t>(kStages) && s < issued; ++s) {
+        const uint32_t n = (issued - 1 - s) / kStages + 1;   // loads issued into stage s
+        drain_phase(&full[s], (n - 1) & 1u);
+    }
+    if (window_pending) drain_phase(pbar, win_phase);
 }
 
 __device__ __forceinline__ int row_tiles(const int32_t *seqlens, int b, int Lmax) {
@@ -313,10 +347,12 @@ __device__ __forceinline__ void merge_warps_and_store(const float *merge, float 
             o = fmaf(weights[head * kConsumerWarps + w], merge[w * kWarpFloats + head * D + d], o);
         if (whole) {
             const size_t row = out_row(p, c.b, c.h, head);
+            if (!FD_DCHECK(row < out_rows(p))) continue;
             p.out[row * D + d] = o;
             if (d == 0) p.lse[row] = lse_h[head];
         } else {
             const size_t row = slot * p.cols + head;
+            if (!FD_DCHECK(row < seg_rows(p))) continue;
             p.seg_out[row * D + d] = o;
             if (d == 0) p.seg_lse[row] = lse_h[head];
         }
@@ -727,6 +763,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         // shared memory, fetched with a 1-D bulk copy when a page falls outside it
         int win_b = -1, win_lo = 0, win_hi = 0;
         uint32_t win_phase = 0;
+        bool win_pending = false;   // a window copy issued and not yet seen complete
         auto page_of = [&](int b, int lp, int *page) -> bool {
             if (b != win_b || lp < win_lo || lp >= win_hi) {
                 win_b = b;
@@ -734,8 +771,11 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                 win_hi = min(win_lo + kPageWindow, p.max_pages);
                 const uint32_t bytes = static_cast<uint32_t>(win_hi - win_lo) * 4u;
                 mbar_arrive_expect_tx(pbar, bytes);
-                bulk_load(page_win, p.block_table + static_cast<size_t>(b) * p.max_pages + win_lo, bytes, pbar);
+                if (FD_DCHECK(b < p.B && win_lo >= 0 && win_lo < win_hi))
+                    bulk_load(page_win, p.block_table + static_cast<size_t>(b) * p.max_pages + win_lo, bytes, pbar);
+                win_pending = true;
                 if (!wait_bounded(pbar, win_phase, abort)) return false;
+                win_pending = false;
                 win_phase ^= 1u;
             }
             *page = page_win[lp - win_lo];
@@ -753,11 +793,22 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             for (int k = 0; k < seg; ++k, ++seq) {
                 const int stage = static_cast<int>(seq % kStages);
                 const uint32_t phase = (seq / kStages) & 1u;
-                if (!wait_bounded(&empty[stage], phase ^ 1u, abort)) return;
+                // once a wait anywhere in the block gave up, issue nothing more (a
+                // stage whose copy never completed must not be armed again)
+                if (*abort || !wait_bounded(&empty[stage], phase ^ 1u, abort)) {
+                    drain_copies<kStages>(full, seq, pbar, win_pending, win_phase);
+                    return;
+                }
                 uint8_t *kt = ring + stage * Cfg::kStageBytes;
                 uint8_t *vt = kt + Cfg::kTileBytes;
                 const bool with_q = k < kGroups;   // each group's first tile of the segment
                 const uint32_t qb = with_q ? q_bytes : 0u;
+#ifdef FD_DEBUG
+                if (blockIdx.x == 0 && static_cast<int>(seq) == p.debug_withhold) {
+                    mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kTileBytes + qb);   // armed, never filled
+                    continue;
+                }
+#endif
                 const int y = (c.tile + k) * kTileTokens;
                 if (!kPaged) {
                     mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kTileBytes + qb);
@@ -778,7 +829,10 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                     const int off = psize >= kTileTokens ? (y & (psize - 1)) : 0;
                     int page[kTileTokens / 8];
                     for (int j = 0; j < nsub; ++j)
-                        if (!page_of(c.b, lp0 + j, &page[j])) return;
+                        if (!page_of(c.b, lp0 + j, &page[j])) {
+                            drain_copies<kStages>(full, seq, pbar, win_pending, win_phase);
+                            return;
+                        }
                     if constexpr (Consumer::kInterleaved) {
                         // one 5-D box per page, both halves of its tokens: [token][half][128 B].
                         // Coordinates {element, half, token, head, page} (head-major pages)
@@ -809,13 +863,18 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                     }
                 }
                 if (with_q)
-                    for (int j = 0; j < p.q_len; ++j)
-                        bulk_load(vt + Cfg::kTileBytes + j * q_run, q_row + static_cast<size_t>(j) * p.Hq * D, q_run,
-                                  &full[stage]);
+                    for (int j = 0; j < p.q_len; ++j) {
+                        const uint16_t *src = q_row + static_cast<size_t>(j) * p.Hq * D;
+                        if (FD_DCHECK(src >= p.q && src + q_run / 2 <= p.q + out_rows(p) * D))
+                            bulk_load(vt + Cfg::kTileBytes + j * q_run, src, q_run, &full[stage]);
+                    }
             }
             remaining -= seg;
             if (remaining > 0) next_row(c, p);
         }
+        // after an abort the consumers no longer wait for the last stages: the
+        // producer keeps the block alive until its copies have landed
+        if (*abort) drain_copies<kStages>(full, seq, pbar, win_pending, win_phase);
         return;
     }
 
@@ -884,7 +943,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                 named_barrier_sync(kBarFinishers, kFinisherThreads);
                 if (ftid == 0) {
                     const RowRuns rr = row_runs(c.first, c.n, N, p.P);
-                    const int prev = atomicAdd(p.row_tickets + u, 1);
+                    const int prev = FD_DCHECK(u < static_cast<long long>(p.B) * p.Hkv) ? atomicAdd(p.row_tickets + u, 1) : -1;
                     if (prev == rr.count - 1 && info->npending < kPendingMax)
                         info->pending[info->npending++] = PendingRow{c.first, c.b, c.h, c.n};
                     __threadfence();   // acquire: the row's other segments are read after this
@@ -916,7 +975,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             if (wtid == 0) {
                 __threadfence();
                 const RowRuns rr = row_runs(last_c.first, last_c.n, N, p.P);
-                const int prev = atomicAdd(p.row_tickets + u, 1);
+                const int prev = FD_DCHECK(u < static_cast<long long>(p.B) * p.Hkv) ? atomicAdd(p.row_tickets + u, 1) : -1;
                 if (prev == rr.count - 1 && info->npending < kPendingMax)
                     info->pending[info->npending++] = PendingRow{last_c.first, last_c.b, last_c.h, last_c.n};
                 __threadfence();
@@ -935,6 +994,9 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             const long long u = static_cast<long long>(r.b) * p.Hkv + r.h;
             const RowRuns rr = row_runs(r.first, r.n, N, p.P);
             const size_t row = out_row(p, r.b, r.h, head);
+            if (!FD_DCHECK(row < out_rows(p) &&
+                           (static_cast<size_t>(rr.i1) + u + 1) * p.cols <= seg_rows(p)))
+                continue;
             float lse;
             const float4 v = merge_row_vec<D>(p.seg_out, p.seg_lse, p.cols, static_cast<size_t>(rr.i0) + u,
                                               rr.i1 - rr.i0 + 1, rr.i0, N, p.P, head, d4, &lse);
@@ -952,6 +1014,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             for (int idx = wtid; idx < p.cols * (D / 4); idx += kWorkerThreads) {
                 const int col = idx / (D / 4), d4 = idx - col * (D / 4);
                 const size_t row = out_row(p, b, h, col);
+                if (!FD_DCHECK(row < out_rows(p))) continue;
                 reinterpret_cast<float4 *>(p.out + row * D)[d4] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (d4 == 0) p.lse[row] = -INFINITY;
             }

@@ -83,6 +83,8 @@ extern "C" {
 #define FD_ERR_TIMEOUT      -10   /* a device-side wait gave up (reported by fd_device_status) */
 #define FD_ERR_CAPACITY     -11   /* an output array passed to fd_segments is too small */
 #define FD_ERR_STATIC_LIMIT -12   /* fd_decode_static: the problem needs more scratch than its fixed buffer */
+#define FD_ERR_BOUNDS       -13   /* debug builds only (-DFD_DEBUG): a device-side bounds check failed; the
+                                     access was skipped and the call's outputs are invalid */
 
 #define FD_TILE_TOKENS     64     /* tokens per tile; split boundaries are multiples of this */
 #define FD_MAX_SPLITS      65535
