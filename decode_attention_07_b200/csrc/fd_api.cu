@@ -308,12 +308,14 @@ int launch_split(int D, int g, const CUtensorMap &tk, const CUtensorMap &tv, con
 template <bool kE4M3>
 int launch_split_quant(int D, int cols, const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p,
                        cudaStream_t st) {
+    // up to 8 columns: four groups of two warps, 32 tokens per warp (more work
+    // in flight per warp); 16 columns: the default two groups of four
     if (D == 128) {
-        if (cols <= 8) return launch_split_t<128, fd::QuantConsumer<128, 1, kE4M3>, true, false>(tk, tv, p, st);
-        return launch_split_t<128, fd::QuantConsumer<128, 2, kE4M3>, true, false>(tk, tv, p, st);
+        if (cols <= 8) return launch_split_t<128, fd::QuantConsumer<128, 1, kE4M3, 32>, true, false>(tk, tv, p, st);
+        return launch_split_t<128, fd::QuantConsumer<128, 2, kE4M3, 16>, true, false>(tk, tv, p, st);
     }
-    if (cols <= 8) return launch_split_t<64, fd::QuantConsumer<64, 1, kE4M3>, true, false>(tk, tv, p, st);
-    return launch_split_t<64, fd::QuantConsumer<64, 2, kE4M3>, true, false>(tk, tv, p, st);
+    if (cols <= 8) return launch_split_t<64, fd::QuantConsumer<64, 1, kE4M3, 32>, true, false>(tk, tv, p, st);
+    return launch_split_t<64, fd::QuantConsumer<64, 2, kE4M3, 16>, true, false>(tk, tv, p, st);
 }
 
 int launch_combine(int D, const fd::CombineParams &p, cudaStream_t st, bool after_split) {

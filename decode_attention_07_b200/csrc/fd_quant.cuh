@@ -51,10 +51,13 @@
 
 namespace fd {
 
-template <int D, int NT, bool kE4M3>
+template <int D, int NT, bool kE4M3, int kTok = 16>
 struct QuantConsumer {
     static constexpr int G = 8 * NT;        // columns held (padded)
     static constexpr int kElemBytes = 1;
+    static constexpr int kWarpTokens = kTok;          // tokens of each tile per warp (16 or 32)
+    static constexpr int MB = kTok / 16;              // 16-token blocks per warp
+    static constexpr int KACC = MB == 1 ? 2 : 1;      // logit accumulators per block
     static constexpr bool kInterleaved = false;
     static constexpr int KC = D / 16;       // 16-byte chunks of a token = k-steps of S = m-tiles of O^T
     static constexpr int kRowBytes = D;
@@ -165,66 +168,87 @@ struct QuantConsumer {
         return w & ((t < valid ? 0x0000ffffu : 0u) | (t + 1 < valid ? 0xffff0000u : 0u));
     }
 
-    // One tile: `slice` = this warp's 16-token slice, `valid` = how many of
-    // those 16 tokens are inside the row.
+    // One tile: `slice` = this warp's slice of kWarpTokens tokens (MB blocks
+    // of 16), `valid` = how many of those tokens are inside the row.
     __device__ __forceinline__ void tile(uint32_t k_smem, uint32_t v_smem, int slice, int valid, float) {
         const int lane = threadIdx.x & 31;
         const int mi = lane >> 3, rr = lane & 7;
         const int r0 = lane >> 2, cc = lane & 3;
-        // ldmatrix x4 over two chunks: matrices (tokens 0-7 | 8-15) x (chunk 2pc | 2pc+1)
-        const int lrow = kWarpTokens * slice + rr + 8 * (mi & 1);
+        const int base = kWarpTokens * slice;
 
-        float s[NT][4], s2[NT][4];
+        // logits S^T = K Q^T per 16-token block; ldmatrix x4 over two chunks:
+        // matrices (tokens 0-7 | 8-15) x (chunk 2pc | 2pc+1). One block keeps
+        // two accumulators (even / odd chunks) for two independent mma
+        // chains; two blocks already give two.
+        float s[MB][KACC][NT][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
+            for (int a = 0; a < KACC; ++a)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) s[mb][a][nt][e] = 0.f;
 #pragma unroll
         for (int pc = 0; pc < KC / 2; ++pc) {
             const int chunk = 2 * pc + (mi >> 1);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(k_smem + lrow * kRowBytes + (swz(chunk, lrow) << 4), a0, a1, a2, a3);
-            uint32_t l0, h0, l1, h1, l2, h2, l3, h3;
-            widen(a0, l0, h0);
-            widen(a1, l1, h1);
-            widen(a2, l2, h2);
-            widen(a3, l3, h3);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                mma_f16_16816(s[nt], l0, l1, h0, h1, qf[nt][2 * pc][0], qf[nt][2 * pc][1]);
-                mma_f16_16816(s2[nt], l2, l3, h2, h3, qf[nt][2 * pc + 1][0], qf[nt][2 * pc + 1][1]);
+            for (int mb = 0; mb < MB; ++mb) {
+                const int lrow = base + 16 * mb + rr + 8 * (mi & 1);
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(k_smem + lrow * kRowBytes + (swz(chunk, lrow) << 4), a0, a1, a2, a3);
+                uint32_t l0, h0, l1, h1, l2, h2, l3, h3;
+                widen(a0, l0, h0);
+                widen(a1, l1, h1);
+                widen(a2, l2, h2);
+                widen(a3, l3, h3);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    mma_f16_16816(s[mb][0][nt], l0, l1, h0, h1, qf[nt][2 * pc][0], qf[nt][2 * pc][1]);
+                    mma_f16_16816(s[mb][KACC - 1][nt], l2, l3, h2, h3, qf[nt][2 * pc + 1][0], qf[nt][2 * pc + 1][1]);
+                }
             }
         }
 
         // Online softmax per column with a lazy reference maximum: m moves
         // (and the accumulators are rescaled) only when a logit of the tile
         // exceeds it by more than kLazy; otherwise p = 2^(x - m) directly.
-        float x[NT][4];
+        float x[MB][NT][4];
         bool grow = false;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            x[nt][0] = (s[nt][0] + s2[nt][0]) * colmul[nt][0];
-            x[nt][1] = (s[nt][1] + s2[nt][1]) * colmul[nt][1];
-            x[nt][2] = (s[nt][2] + s2[nt][2]) * colmul[nt][0];
-            x[nt][3] = (s[nt][3] + s2[nt][3]) * colmul[nt][1];
-            const int va = valid - shift[nt][0], vb = valid - shift[nt][1];
-            if (r0 >= va) x[nt][0] = -INFINITY;
-            if (r0 >= vb) x[nt][1] = -INFINITY;
-            if (r0 + 8 >= va) x[nt][2] = -INFINITY;
-            if (r0 + 8 >= vb) x[nt][3] = -INFINITY;
-            const float ta = m[nt][0] + kLazy, tb = m[nt][1] + kLazy;
-            grow |= x[nt][0] > ta || x[nt][2] > ta || x[nt][1] > tb || x[nt][3] > tb;
-        }
+        for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float acc = s[mb][0][nt][e];
+                    if (KACC == 2) acc += s[mb][KACC - 1][nt][e];
+                    x[mb][nt][e] = acc * colmul[nt][e & 1];
+                }
+                // token r of this block is inside column e's causal range when r < valid - 16 mb - shift
+                const int va = valid - 16 * mb - shift[nt][0], vb = valid - 16 * mb - shift[nt][1];
+                if (r0 >= va) x[mb][nt][0] = -INFINITY;
+                if (r0 >= vb) x[mb][nt][1] = -INFINITY;
+                if (r0 + 8 >= va) x[mb][nt][2] = -INFINITY;
+                if (r0 + 8 >= vb) x[mb][nt][3] = -INFINITY;
+                const float ta = m[nt][0] + kLazy, tb = m[nt][1] + kLazy;
+                grow |= x[mb][nt][0] > ta || x[mb][nt][2] > ta || x[mb][nt][1] > tb || x[mb][nt][3] > tb;
+            }
         if (__any_sync(0xffffffffu, grow)) {   // the fallback: a synchronised rescale
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                float ma = fmaxf(x[nt][0], x[nt][2]), mb = fmaxf(x[nt][1], x[nt][3]);
+                float ma = -INFINITY, mbx = -INFINITY;
+#pragma unroll
+                for (int mb = 0; mb < MB; ++mb) {
+                    ma = fmaxf(ma, fmaxf(x[mb][nt][0], x[mb][nt][2]));
+                    mbx = fmaxf(mbx, fmaxf(x[mb][nt][1], x[mb][nt][3]));
+                }
 #pragma unroll
                 for (int sh = 4; sh < 32; sh <<= 1) {
                     ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, sh));
-                    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, sh));
+                    mbx = fmaxf(mbx, __shfl_xor_sync(0xffffffffu, mbx, sh));
                 }
-                const float na = fmaxf(m[nt][0], ma), nb = fmaxf(m[nt][1], mb);
+                const float na = fmaxf(m[nt][0], ma), nb = fmaxf(m[nt][1], mbx);
                 const float ua = na == -INFINITY ? 0.f : na, ub = nb == -INFINITY ? 0.f : nb;
                 const float alpha_a = ex2(m[nt][0] - ua), alpha_b = ex2(m[nt][1] - ub);
                 l[nt][0] *= alpha_a;
@@ -241,51 +265,59 @@ struct QuantConsumer {
             }
         }
 
-        // P^T fragments (f16 high part + remainder, x 2^kPScale)
-        uint32_t bh[NT][2], bl[NT][2];
+        // P^T fragments per block (f16 high part + remainder, x 2^kPScale)
+        uint32_t bh[MB][NT][2], bl[MB][NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const float ta = kPScale - (m[nt][0] == -INFINITY ? 0.f : m[nt][0]);
             const float tb = kPScale - (m[nt][1] == -INFINITY ? 0.f : m[nt][1]);
-            const float p0 = ex2(x[nt][0] + ta), p2 = ex2(x[nt][2] + ta);
-            const float p1 = ex2(x[nt][1] + tb), p3 = ex2(x[nt][3] + tb);
-            l[nt][0] += p0 + p2;
-            l[nt][1] += p1 + p3;
-            const uint32_t h01 = pack_f16x2(p0, p1), h23 = pack_f16x2(p2, p3);
-            const uint32_t l01 = pack_f16x2(p0 - f16lo_to_f32(h01), p1 - f16hi_to_f32(h01));
-            const uint32_t l23 = pack_f16x2(p2 - f16lo_to_f32(h23), p3 - f16hi_to_f32(h23));
-            bh[nt][0] = movmatrix_trans(h01);
-            bh[nt][1] = movmatrix_trans(h23);
-            bl[nt][0] = movmatrix_trans(l01);
-            bl[nt][1] = movmatrix_trans(l23);
+#pragma unroll
+            for (int mb = 0; mb < MB; ++mb) {
+                const float p0 = ex2(x[mb][nt][0] + ta), p2 = ex2(x[mb][nt][2] + ta);
+                const float p1 = ex2(x[mb][nt][1] + tb), p3 = ex2(x[mb][nt][3] + tb);
+                l[nt][0] += p0 + p2;
+                l[nt][1] += p1 + p3;
+                const uint32_t h01 = pack_f16x2(p0, p1), h23 = pack_f16x2(p2, p3);
+                const uint32_t l01 = pack_f16x2(p0 - f16lo_to_f32(h01), p1 - f16hi_to_f32(h01));
+                const uint32_t l23 = pack_f16x2(p2 - f16lo_to_f32(h23), p3 - f16hi_to_f32(h23));
+                bh[mb][nt][0] = movmatrix_trans(h01);
+                bh[mb][nt][1] = movmatrix_trans(h23);
+                bl[mb][nt][0] = movmatrix_trans(l01);
+                bl[mb][nt][1] = movmatrix_trans(l23);
+            }
         }
 
-        // O^T += V^T P^T, one 16-element chunk of head dims per m-tile.
-        // ldmatrix.trans of the 8-bit tile read as 16-bit elements gives each
-        // thread tokens (2cc, 2cc+1) x head dims (2r0, 2r0+1) of a chunk; the
-        // widening regroups them into token pairs at head dims 2r0 (accumulator
-        // row r0) and 2r0 + 1 (row r0 + 8).
+        // O^T += V^T P^T, one 16-element chunk of head dims per m-tile, one
+        // 16-token k-step per block. ldmatrix.trans of the 8-bit tile read as
+        // 16-bit elements gives each thread tokens (2cc, 2cc+1) x head dims
+        // (2r0, 2r0+1) of a chunk; the widening regroups them into token pairs
+        // at head dims 2r0 (accumulator row r0) and 2r0 + 1 (row r0 + 8).
 #pragma unroll
         for (int pc = 0; pc < KC / 2; ++pc) {
             const int chunk = 2 * pc + (mi >> 1);
-            uint32_t a[4];
-            ldsm_x4_trans(v_smem + lrow * kRowBytes + (swz(chunk, lrow) << 4), a[0], a[1], a[2], a[3]);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                // tokens 0..7 (x) and 8..15 (y) of the slice, chunk 2pc + half
-                uint32_t A0, A1, A2, A3;
-                widen_t(a[2 * half], A0, A1);
-                widen_t(a[2 * half + 1], A2, A3);
-                if (valid < kWarpTokens) {   // rows past the end may hold anything (NaN codes): zero them
-                    A0 = keep_tokens(A0, 2 * cc, valid);
-                    A1 = keep_tokens(A1, 2 * cc, valid);
-                    A2 = keep_tokens(A2, 8 + 2 * cc, valid);
-                    A3 = keep_tokens(A3, 8 + 2 * cc, valid);
-                }
+            for (int mb = 0; mb < MB; ++mb) {
+                const int lrow = base + 16 * mb + rr + 8 * (mi & 1);
+                const int vmb = valid - 16 * mb;
+                uint32_t a[4];
+                ldsm_x4_trans(v_smem + lrow * kRowBytes + (swz(chunk, lrow) << 4), a[0], a[1], a[2], a[3]);
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    mma_f16_16816(o[nt][2 * pc + half], A0, A1, A2, A3, bh[nt][0], bh[nt][1]);
-                    mma_f16_16816(o[nt][2 * pc + half], A0, A1, A2, A3, bl[nt][0], bl[nt][1]);
+                for (int half = 0; half < 2; ++half) {
+                    // tokens 0..7 (x) and 8..15 (y) of the block, chunk 2pc + half
+                    uint32_t A0, A1, A2, A3;
+                    widen_t(a[2 * half], A0, A1);
+                    widen_t(a[2 * half + 1], A2, A3);
+                    if (vmb < 16) {   // rows past the end may hold anything (NaN codes): zero them
+                        A0 = keep_tokens(A0, 2 * cc, vmb);
+                        A1 = keep_tokens(A1, 2 * cc, vmb);
+                        A2 = keep_tokens(A2, 8 + 2 * cc, vmb);
+                        A3 = keep_tokens(A3, 8 + 2 * cc, vmb);
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        mma_f16_16816(o[nt][2 * pc + half], A0, A1, A2, A3, bh[mb][nt][0], bh[mb][nt][1]);
+                        mma_f16_16816(o[nt][2 * pc + half], A0, A1, A2, A3, bl[mb][nt][0], bl[mb][nt][1]);
+                    }
                 }
             }
         }

@@ -49,8 +49,11 @@
 
 namespace fd {
 
-constexpr int kGroups = 2;                        // consumer groups alternating tiles
-constexpr int kSliceWarps = 4;                    // warps per group (16 tokens each)
+// Consumers: 8 warps in groups that take turns on tiles. By default two
+// groups of four warps, 16 tokens of each 64-token tile per warp; a consumer
+// type can declare 32 tokens per warp (four groups of two warps).
+constexpr int kGroups = 2;                        // default: consumer groups alternating tiles
+constexpr int kSliceWarps = 4;                    // default: warps per group (16 tokens each)
 constexpr int kConsumerWarps = kGroups * kSliceWarps;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kProducerWarp = kConsumerWarps;     // warp 8
@@ -61,7 +64,7 @@ constexpr int kWorkerThreads = kConsumerThreads + kFinisherThreads;   // all but
 constexpr int kPendingMax = 4;                    // rows a block can complete (a run cuts at most 2)
 constexpr int kBarFinishers = 1, kBarWorkers = 2; // named barrier ids
 constexpr int kPrefetchTiles = 8;                 // tiles guessed into L2 before the dependency wait
-constexpr int kWarpTokens = 16;                   // tokens of a tile owned by one consumer warp
+constexpr int kWarpTokens = 16;                   // default tokens of a tile owned by one consumer warp
 constexpr int kBoxBytes = kTileTokens * 128;      // one TMA box: 64 rows x 128 bytes (64 bf16)
 constexpr int kSmemLimit = 232448;                // 227 KiB opt-in shared memory per block
 #ifdef FD_DEBUG
@@ -156,7 +159,7 @@ struct SplitConfig {
     // Each consumer group owns whole stages: a stage shared by both groups
     // could be waited on two phases ahead of a tile still in flight, where a
     // parity wait would pass on the older phase.
-    static_assert(kStages % kGroups == 0, "each consumer group must own whole stages");
+    static_assert(kStages % 2 == 0, "stages come in pairs");
     static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
     static_assert(kSmemBytes <= kSmemLimit, "shared memory over the limit");
 };
@@ -366,6 +369,7 @@ struct GroupConsumer {
     static constexpr int MT = D / 16;   // m-tiles of the P V contraction
     static constexpr int G = 8 * NT;    // heads held (padded)
     static constexpr int kElemBytes = 2;
+    static constexpr int kWarpTokens = 16;
     static constexpr bool kInterleaved = kInter;
 
     uint32_t qf[NT][KS][2];             // Q^T as the B operand, per n-tile
@@ -545,6 +549,7 @@ template <int D, bool kInter = false>
 struct HeadConsumer {
     static constexpr int G = 1;
     static constexpr int kElemBytes = 2;
+    static constexpr int kWarpTokens = 16;
     static constexpr bool kInterleaved = kInter;
     static constexpr int LPT = D / 8;          // lanes per token (16 bytes = 8 bf16 each)
     static constexpr int TPI = 32 / LPT;       // tokens per warp-wide load
@@ -684,6 +689,13 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                     const SplitParams p) {
     constexpr int G = Consumer::G;
     using Cfg = SplitConfig<D, G, Consumer::kElemBytes>;
+    constexpr int kTok = Consumer::kWarpTokens;          // tokens per consumer warp and tile
+    constexpr int kSlices = kTileTokens / kTok;           // warps per consumer group
+    constexpr int kGroupsC = kConsumerWarps / kSlices;    // groups taking turns on tiles
+    // Each consumer group owns whole stages: a stage shared by two groups could
+    // be waited on two phases ahead of a tile still in flight, where a parity
+    // wait would pass on the older phase.
+    static_assert(Cfg::kStages % kGroupsC == 0, "each consumer group must own whole stages");
     static_assert(!kPaged || Consumer::kElemBytes == 2, "paged caches are bf16");
     constexpr int kStages = Cfg::kStages;
     constexpr int kBufs = Cfg::kMergeBufs;
@@ -711,7 +723,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kSliceWarps);
+            mbar_init(&empty[s], kSlices);
         }
         for (int b = 0; b < kBufs; ++b) {
             mbar_init(&mfull[b], kConsumerWarps);
@@ -801,7 +813,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                 }
                 uint8_t *kt = ring + stage * Cfg::kStageBytes;
                 uint8_t *vt = kt + Cfg::kTileBytes;
-                const bool with_q = k < kGroups;   // each group's first tile of the segment
+                const bool with_q = k < kGroupsC;   // each group's first tile of the segment
                 const uint32_t qb = with_q ? q_bytes : 0u;
 #ifdef FD_DEBUG
                 if (blockIdx.x == 0 && static_cast<int>(seq) == p.debug_withhold) {
@@ -882,7 +894,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     int last_seg = 0;
     if (warp < kConsumerWarps) {
         // ---------------------------------------------------- consumers --
-        const int group = warp / kSliceWarps, slice = warp % kSliceWarps;
+        const int group = warp / kSlices, slice = warp % kSlices;
         Consumer cons;
         cons.init(p);
         uint32_t seq = 0, segctr = 0;
@@ -892,14 +904,14 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             cons.reset();
             cons.set_row(p, c.h);
             for (int k = 0; k < seg; ++k, ++seq) {
-                if (static_cast<int>(seq % kGroups) != group) continue;
+                if (static_cast<int>(seq % kGroupsC) != group) continue;
                 const int stage = static_cast<int>(seq % kStages);
                 const uint32_t phase = (seq / kStages) & 1u;
                 wait_bounded(&full[stage], phase, abort);   // on abort: keep going, outputs are flagged invalid
                 const uint8_t *st = ring + stage * Cfg::kStageBytes;
-                if (k < kGroups) cons.load_q(st + 2 * Cfg::kTileBytes, p.cols);
+                if (k < kGroupsC) cons.load_q(st + 2 * Cfg::kTileBytes, p.cols);
                 const uint32_t kt = smem_addr(st);
-                const int valid = L - ((c.tile + k) * kTileTokens + kWarpTokens * slice);
+                const int valid = L - ((c.tile + k) * kTileTokens + kTok * slice);
                 cons.tile(kt, kt + Cfg::kTileBytes, slice, valid, p.scale_log2e);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[stage]);
