@@ -346,10 +346,18 @@ def run_fd(args, w, rank, world):
         from decode_attention_07_b200.inputs import make_paged
         pgs = [make_paged(x, args.paged, args.layout, seed=7 + i) for i, x in enumerate(xs)]
         for x in xs:   # the contiguous copies are not used by the paged calls
-            x.k = x.v = None
+            if quant:
+                x.k8 = x.v8 = None
+            else:
+                x.k = x.v = None
         torch.cuda.empty_cache()
-        calls = [fd.prepare_decode_paged(x.q, pg.k_pages, pg.v_pages, pg.block_table, x.seqlens, x.scale, out, lse,
-                                         ws, args.layout, S, stream) for x, pg in zip(xs, pgs)]
+        if quant:
+            calls = [fd.prepare_decode_quant_paged(x.q, pg.k_pages, pg.v_pages, x.k_scale, x.v_scale, args.kv,
+                                                   pg.block_table, x.seqlens, x.scale, out, lse, ws, args.layout, S,
+                                                   stream) for x, pg in zip(xs, pgs)]
+        else:
+            calls = [fd.prepare_decode_paged(x.q, pg.k_pages, pg.v_pages, pg.block_table, x.seqlens, x.scale, out,
+                                             lse, ws, args.layout, S, stream) for x, pg in zip(xs, pgs)]
     elif quant:
         calls = [fd.prepare_decode_quant(x.q, x.k8, x.v8, x.k_scale, x.v_scale, args.kv, x.seqlens, x.scale, out, lse,
                                          ws, S, stream) for x in xs]
@@ -642,8 +650,8 @@ def main():
     ap.add_argument("--no-clock-window", action="store_true",
                     help="do not extend clock sampling past the timed region (for profiler runs)")
     args = ap.parse_args()
-    if args.paged and (args.kv != "bf16" or args.q_len != 1):
-        ap.error("--paged reads a bf16 cache with one query per sequence")
+    if args.paged and args.q_len != 1:
+        ap.error("--paged takes one query per sequence")
     if args.cp and (args.paged or args.kv != "bf16" or args.q_len != 1):
         ap.error("--cp shards a contiguous bf16 cache with one query per sequence")
     w = WORKLOADS[args.config]

@@ -63,12 +63,13 @@ def lib() -> ctypes.CDLL:
         L.fd_decode_quant.argtypes = [_i] * 7 + [_p, _p, _p, _p, _p, _p, _f, _p, _p, _p, _sz, _i, _p]
         L.fd_merge_partials.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p]
         L.fd_read_probe.argtypes = [_p, _sz, _p, _p]
+        L.fd_decode_quant_paged.argtypes = [_i] * 10 + [_p] * 7 + [_f, _p, _p, _p, _sz, _i, _p]
         L.fd_strerror.argtypes = [_i]
         L.fd_strerror.restype = ctypes.c_char_p
         L.fd_version.argtypes = []
         for name in ("fd_plan", "fd_plan_for_sms", "fd_decode", "fd_decode_splits", "fd_split", "fd_combine",
                      "fd_segments", "fd_device_status", "fd_version", "fd_workspace_init", "fd_decode_static",
-                     "fd_decode_paged", "fd_decode_multi", "fd_decode_quant", "fd_merge_partials", "fd_read_probe"):
+                     "fd_decode_paged", "fd_decode_multi", "fd_decode_quant", "fd_merge_partials", "fd_read_probe", "fd_decode_quant_paged"):
             getattr(L, name).restype = _i
         _lib = L
     return _lib
@@ -216,21 +217,23 @@ def decode_multi(q, k_cache, v_cache, seqlens, scale, num_splits=None, stream=No
     return out, lse
 
 
-def _paged_shapes(q, k_pages, v_pages, block_table, layout):
+def _paged_shapes(q, k_pages, v_pages, block_table, layout, pool_dtype=torch.bfloat16):
     if layout not in LAYOUTS:
         raise ValueError("layout must be 'HND' ([pages, Hkv, page_size, D]) or 'NHD' ([pages, page_size, Hkv, D])")
-    if q.dim() != 3 or k_pages.dim() != 4 or v_pages.shape != k_pages.shape or block_table.dim() != 2:
-        raise ValueError("expected q [B,Hq,D], k_pages/v_pages 4-D, block_table [B, max_pages]")
-    B, Hq, D = q.shape
+    if q.dim() not in (3, 4) or k_pages.dim() != 4 or v_pages.shape != k_pages.shape or block_table.dim() != 2:
+        raise ValueError("expected q [B,Hq,D] (or [B,q_len,Hq,D]), k_pages/v_pages 4-D, block_table [B, max_pages]")
+    B, Hq, D = q.shape[0], q.shape[-2], q.shape[-1]
     if layout == "HND":
         num_pages, Hkv, page_size, D2 = k_pages.shape
     else:
         num_pages, page_size, Hkv, D2 = k_pages.shape
     if D2 != D or block_table.shape[0] != B:
         raise ValueError("q, pages and block_table disagree on B or D")
-    for t, name in ((q, "q"), (k_pages, "k_pages"), (v_pages, "v_pages")):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if q.dtype != torch.bfloat16 or not q.is_cuda or not q.is_contiguous():
+        raise ValueError("q must be a contiguous bf16 CUDA tensor")
+    for t, name in ((k_pages, "k_pages"), (v_pages, "v_pages")):
+        if t.dtype != pool_dtype or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {pool_dtype} CUDA tensor")
     if block_table.dtype != torch.int32 or not block_table.is_cuda or not block_table.is_contiguous():
         raise ValueError("block_table must be a contiguous int32 CUDA tensor")
     return B, Hq, Hkv, D, page_size, num_pages, block_table.shape[1]
@@ -267,6 +270,57 @@ def prepare_decode_paged(q, k_pages, v_pages, block_table, seqlens, scale, out, 
             raise FdError(rc, "fd_decode_paged")
 
     return call
+
+
+def prepare_decode_quant_paged(q, k_pages, v_pages, k_scale, v_scale, kv_type, block_table, seqlens, scale, out, lse,
+                               workspace=None, layout="HND", num_splits=0, stream=None):
+    """prepare_decode for fd_decode_quant_paged: 8-bit page pools (uint8,
+    layouts as fd_decode_paged), per-kv-head float32 scales, kv_type "e4m3"
+    or "int8"; q [B, Hq, D] or [B, q_len, Hq, D], out / lse shaped to match."""
+    if kv_type not in KV_CODES:
+        raise ValueError("kv_type must be 'e4m3' or 'int8'")
+    B, Hq, Hkv, D, page_size, num_pages, max_pages = _paged_shapes(q, k_pages, v_pages, block_table, layout,
+                                                                   torch.uint8)
+    q_len = 1 if q.dim() == 3 else q.shape[1]
+    for t, name in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        if t.shape != (Hkv,) or t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor of shape [Hkv]")
+    if out.shape != q.shape or lse.shape != q.shape[:-1]:
+        raise ValueError("out must be shaped like q and lse like q without D")
+    for t, name in ((out, "out"), (lse, "lse")):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor")
+    _seqlens(seqlens, B)
+    wp, wb = _ws(workspace)
+    fn = lib().fd_decode_quant_paged
+    args = (B, q_len, Hq, Hkv, D, page_size, num_pages, max_pages, LAYOUTS[layout], KV_CODES[kv_type], q.data_ptr(),
+            k_pages.data_ptr(), v_pages.data_ptr(), k_scale.data_ptr(), v_scale.data_ptr(), block_table.data_ptr(),
+            seqlens.data_ptr(), ctypes.c_float(scale), out.data_ptr(), lse.data_ptr(), wp, wb, int(num_splits),
+            _stream(stream, q.device))
+
+    def call():
+        rc = fn(*args)
+        if rc != 0:
+            raise FdError(rc, "fd_decode_quant_paged")
+
+    return call
+
+
+def decode_quant_paged(q, k_pages, v_pages, k_scale, v_scale, kv_type, block_table, seqlens, scale, layout="HND",
+                       num_splits=None, stream=None):
+    """Allocate out / lse / workspace with torch and run fd_decode_quant_paged."""
+    B, Hq, Hkv, D, page_size, num_pages, max_pages = _paged_shapes(q, k_pages, v_pages, block_table, layout,
+                                                                   torch.uint8)
+    q_len = 1 if q.dim() == 3 else q.shape[1]
+    Lmax = max_pages * page_size
+    S = fd_plan(B, Hq, Hkv, D, Lmax) if num_splits is None else int(num_splits)
+    nbytes = fd_workspace_bytes(B, Hq * q_len, Hkv, D, Lmax, S)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=q.device) if nbytes else None
+    out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    prepare_decode_quant_paged(q, k_pages, v_pages, k_scale, v_scale, kv_type, block_table, seqlens, scale, out, lse,
+                               ws, layout, S, stream)()
+    return out, lse
 
 
 def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale, layout="HND", num_splits=None, stream=None):

@@ -145,43 +145,46 @@ int encode_cache_map(CUtensorMap *map, const void *base, int D, int Lmax, long l
     return r == CUDA_SUCCESS ? FD_OK : FD_ERR_LAUNCH;
 }
 
-// Paged K or V pool as a 4-D tensor, head-dim innermost; the other three dims
-// in increasing-stride order. Head-major pages [num_pages][Hkv][page_size][D]:
-// {D, page_size, Hkv, num_pages}, box {64, rows, 1, 1}. Token-major pages
-// [num_pages][page_size][Hkv][D]: {D, Hkv, page_size, num_pages}, box
-// {64, 1, rows, 1}. rows = min(page_size, 64); 128-byte swizzle as above.
+// Paged K or V pool as a 3-D tensor, head-dim innermost. Head-major pages
+// [num_pages][Hkv][page_size][D]: the token rows of one (page, head) are
+// contiguous, so {D, page_size, num_pages * Hkv}, box {64, rows, 1}, row
+// z = page * Hkv + head. Token-major pages [num_pages][page_size][Hkv][D]:
+// page and token merge into one dimension, {D, Hkv, num_pages * page_size},
+// box {64, 1, rows}, z = page * page_size + token. rows = min(page_size, 64);
+// 128-byte swizzle as above. A page index outside the pool falls outside the
+// tensor either way (TMA fills zeros). 8-bit codes (one_byte): boxes of all D
+// codes of a token (64-byte swizzle for D = 64).
 int encode_paged_map(CUtensorMap *map, const void *base, int D, int page_size, int Hkv, long long num_pages,
-                     bool nhd) {
+                     bool nhd, bool one_byte = false) {
     auto fn = encode_fn();
     if (!fn) return FD_ERR_LAUNCH;
-    const cuuint64_t e = 2;   // bf16
+    const cuuint64_t e = one_byte ? 1 : 2;   // 8-bit codes or bf16
     const cuuint32_t rows = static_cast<cuuint32_t>(page_size < fd::kTileTokens ? page_size : fd::kTileTokens);
-    cuuint64_t dims[4], strides[3];
-    cuuint32_t box[4];
+    const cuuint64_t row = static_cast<cuuint64_t>(D) * e;   // bytes of one token of one head
+    cuuint64_t dims[3], strides[2];
+    cuuint32_t box[3];
     dims[0] = static_cast<cuuint64_t>(D);
-    dims[3] = static_cast<cuuint64_t>(num_pages);
-    box[0] = 64;
-    box[3] = 1;
+    box[0] = one_byte ? static_cast<cuuint32_t>(D) : 64u;
     if (nhd) {
         dims[1] = static_cast<cuuint64_t>(Hkv);
-        dims[2] = static_cast<cuuint64_t>(page_size);
-        strides[0] = D * e;
-        strides[1] = static_cast<cuuint64_t>(Hkv) * D * e;
+        dims[2] = static_cast<cuuint64_t>(num_pages) * page_size;
+        strides[0] = row;
+        strides[1] = static_cast<cuuint64_t>(Hkv) * row;
         box[1] = 1;
         box[2] = rows;
     } else {
         dims[1] = static_cast<cuuint64_t>(page_size);
-        dims[2] = static_cast<cuuint64_t>(Hkv);
-        strides[0] = D * e;
-        strides[1] = static_cast<cuuint64_t>(page_size) * D * e;
+        dims[2] = static_cast<cuuint64_t>(num_pages) * Hkv;
+        strides[0] = row;
+        strides[1] = static_cast<cuuint64_t>(page_size) * row;
         box[1] = rows;
         box[2] = 1;
     }
-    strides[2] = static_cast<cuuint64_t>(page_size) * Hkv * D * e;
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle swz = one_byte && D == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    CUresult r = fn(map, one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FD_OK : FD_ERR_LAUNCH;
 }
 
@@ -305,17 +308,17 @@ int launch_split(int D, int g, const CUtensorMap &tk, const CUtensorMap &tv, con
 }
 
 // 8-bit caches: the tensor-core consumer for every column count (fused form).
-template <bool kE4M3>
+template <bool kE4M3, bool kPaged = false>
 int launch_split_quant(int D, int cols, const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p,
                        cudaStream_t st) {
     // up to 8 columns: four groups of two warps, 32 tokens per warp (more work
     // in flight per warp); 16 columns: the default two groups of four
     if (D == 128) {
-        if (cols <= 8) return launch_split_t<128, fd::QuantConsumer<128, 1, kE4M3, 32>, true, false>(tk, tv, p, st);
-        return launch_split_t<128, fd::QuantConsumer<128, 2, kE4M3, 16>, true, false>(tk, tv, p, st);
+        if (cols <= 8) return launch_split_t<128, fd::QuantConsumer<128, 1, kE4M3, 32>, true, kPaged>(tk, tv, p, st);
+        return launch_split_t<128, fd::QuantConsumer<128, 2, kE4M3, 16>, true, kPaged>(tk, tv, p, st);
     }
-    if (cols <= 8) return launch_split_t<64, fd::QuantConsumer<64, 1, kE4M3, 32>, true, false>(tk, tv, p, st);
-    return launch_split_t<64, fd::QuantConsumer<64, 2, kE4M3, 16>, true, false>(tk, tv, p, st);
+    if (cols <= 8) return launch_split_t<64, fd::QuantConsumer<64, 1, kE4M3, 32>, true, kPaged>(tk, tv, p, st);
+    return launch_split_t<64, fd::QuantConsumer<64, 2, kE4M3, 16>, true, kPaged>(tk, tv, p, st);
 }
 
 int launch_combine(int D, const fd::CombineParams &p, cudaStream_t st, bool after_split) {
@@ -423,6 +426,7 @@ int run_split(const Problem &pr, bool fused, int q_len = 1) {
     p.max_pages = 0;
     p.page_shift = 0;
     p.kv_nhd = 0;
+    p.num_pages = 0;
     p.k_scale = p.v_scale = nullptr;
     p.debug_withhold = debug_withhold();
     // with max_len == 0 every block finds zero tiles and only writes empty rows;
@@ -437,47 +441,60 @@ struct PagedLayout {
     bool nhd;
 };
 
-int run_split_paged(const Problem &pr, const PagedLayout &pl) {
+// Paged caches: bf16 (kv_type 0) or 8-bit codes (FD_KV_E4M3 / FD_KV_INT8 with
+// per-kv-head scales), q_len queries per sequence.
+int run_split_paged(const Problem &pr, const PagedLayout &pl, int q_len = 1, int kv_type = 0,
+                    const float *k_scale = nullptr, const float *v_scale = nullptr) {
     int sms;
     int rc = device_sms(&sms);
     if (rc != FD_OK) return rc;
     CUtensorMap tk, tv;
-    const bool rows_map = pr.D == 128 && pl.page_size < fd::kTileTokens;   // one box per small page
+    const bool quant = kv_type != 0;
+    // bf16 at D = 128 with small pages: one box per page (both 128-byte halves of a row)
+    const bool rows_map = !quant && pr.D == 128 && pl.page_size < fd::kTileTokens;
     if (rows_map) {
         if ((rc = encode_paged_map_rows(&tk, pr.k, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
         if ((rc = encode_paged_map_rows(&tv, pr.v, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
     } else {
-        if ((rc = encode_paged_map(&tk, pr.k, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
-        if ((rc = encode_paged_map(&tv, pr.v, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
+        if ((rc = encode_paged_map(&tk, pr.k, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd, quant)) != FD_OK)
+            return rc;
+        if ((rc = encode_paged_map(&tv, pr.v, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd, quant)) != FD_OK)
+            return rc;
     }
     fd::SplitParams p;
     p.q = pr.q;
     p.seqlens = pr.seqlens;
     p.out = pr.out;
     p.lse = pr.lse;
-    seg_pointers(pr, &p.seg_out, &p.seg_lse, &p.row_tickets);
+    seg_pointers(pr, &p.seg_out, &p.seg_lse, &p.row_tickets, q_len);
     p.B = pr.B;
     p.Hq = pr.Hq;
     p.Hkv = pr.Hkv;
     p.g = pr.Hq / pr.Hkv;
     p.Lmax = pr.max_len;
     p.P = pr.num_splits;
-    p.q_len = 1;
-    p.cols = p.g;
+    p.q_len = q_len;
+    p.cols = p.g * q_len;
     p.scale_log2e = pr.scale * kLog2e;
     p.block_table = pl.block_table;
     p.max_pages = pl.max_pages;
     p.page_shift = 0;
     while ((1 << p.page_shift) < pl.page_size) ++p.page_shift;
     p.kv_nhd = pl.nhd ? 1 : 0;
-    p.k_scale = p.v_scale = nullptr;
+    p.num_pages = pl.num_pages;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
     p.debug_withhold = debug_withhold();
+    if (quant)
+        return kv_type == FD_KV_E4M3 ? launch_split_quant<true, true>(pr.D, p.cols, tk, tv, p, pr.stream)
+                                     : launch_split_quant<false, true>(pr.D, p.cols, tk, tv, p, pr.stream);
     if (rows_map) {
-        if (p.g == 1) return launch_split_t<128, fd::HeadConsumer<128, true>, true, true>(tk, tv, p, pr.stream);
-        if (p.g <= 8) return launch_split_t<128, fd::GroupConsumer<128, 1, true>, true, true>(tk, tv, p, pr.stream);
+        if (p.cols == 1) return launch_split_t<128, fd::HeadConsumer<128, true>, true, true>(tk, tv, p, pr.stream);
+        if (p.cols <= 8)
+            return launch_split_t<128, fd::GroupConsumer<128, 1, true>, true, true>(tk, tv, p, pr.stream);
         return launch_split_t<128, fd::GroupConsumer<128, 2, true>, true, true>(tk, tv, p, pr.stream);
     }
-    return launch_split<true, true>(pr.D, p.g, tk, tv, p, pr.stream);
+    return launch_split<true, true>(pr.D, p.cols, tk, tv, p, pr.stream);
 }
 
 // Fused split kernel over an 8-bit cache (pr.k / pr.v point at the codes).
@@ -512,6 +529,7 @@ int run_split_quant(const Problem &pr, int q_len, int kv_type, const float *k_sc
     p.max_pages = 0;
     p.page_shift = 0;
     p.kv_nhd = 0;
+    p.num_pages = 0;
     p.k_scale = k_scale;
     p.v_scale = v_scale;
     p.debug_withhold = debug_withhold();
@@ -729,8 +747,45 @@ int fd_decode_paged(int B, int Hq, int Hkv, int D, int page_size, int num_pages,
         pr.num_splits = S;
         if ((rc = check_problem(pr, true)) != FD_OK) return rc;   // workspace for the planned count
     }
+    // the flattened page coordinate (page * Hkv or page * page_size) must fit in int32
+    if (static_cast<long long>(num_pages) * (Hkv > page_size ? Hkv : page_size) > 0x7fffffffLL) return FD_ERR_SHAPE;
     PagedLayout pl{block_table, page_size, num_pages, max_pages_per_seq, kv_layout == FD_KV_NHD};
     return run_split_paged(pr, pl);
+}
+
+int fd_decode_quant_paged(int B, int q_len, int Hq, int Hkv, int D, int page_size, int num_pages,
+                          int max_pages_per_seq, int kv_layout, int kv_type, const uint16_t *q, const uint8_t *k_pages,
+                          const uint8_t *v_pages, const float *k_scale, const float *v_scale,
+                          const int32_t *block_table, const int32_t *seqlens, float scale, float *out, float *lse,
+                          void *workspace, size_t workspace_bytes, int num_splits, void *stream) {
+    if (q_len < 1 || q_len > FD_MAX_GROUP) return FD_ERR_SHAPE;
+    if (kv_type != FD_KV_E4M3 && kv_type != FD_KV_INT8) return FD_ERR_SHAPE;
+    if (page_size < 8 || page_size > 4096 || (page_size & (page_size - 1)) != 0) return FD_ERR_SHAPE;
+    if (num_pages < 1 || max_pages_per_seq < 1 || (max_pages_per_seq % 4) != 0) return FD_ERR_SHAPE;
+    if (kv_layout != FD_KV_HND && kv_layout != FD_KV_NHD) return FD_ERR_SHAPE;
+    const long long max_len = static_cast<long long>(max_pages_per_seq) * page_size;
+    if (max_len > 0x7fffffffLL) return FD_ERR_SHAPE;
+    int rc = check_shape(B, Hq, Hkv, D, static_cast<int>(max_len));
+    if (rc != FD_OK) return rc;
+    if (static_cast<long long>(Hq) * q_len / Hkv > FD_MAX_GROUP) return FD_ERR_GROUP;
+    if (!block_table || !k_scale || !v_scale) return FD_ERR_NULL_POINTER;
+    if (!aligned(block_table, 16) || !aligned(k_scale, 4) || !aligned(v_scale, 4)) return FD_ERR_ALIGNMENT;
+    if (num_splits < 0) return FD_ERR_SPLITS;
+    Problem pr = make_problem(B, Hq * q_len, Hkv, D, static_cast<int>(max_len), q,
+                              reinterpret_cast<const uint16_t *>(k_pages), reinterpret_cast<const uint16_t *>(v_pages),
+                              seqlens, scale, out, lse, workspace, workspace_bytes, num_splits == 0 ? 1 : num_splits,
+                              stream);
+    if ((rc = check_problem(pr, true)) != FD_OK) return rc;
+    if (num_splits == 0) {
+        const int S = fd_plan(B, Hq, Hkv, D, static_cast<int>(max_len));
+        if (S < 0) return S;
+        pr.num_splits = S;
+        if ((rc = check_problem(pr, true)) != FD_OK) return rc;
+    }
+    pr.Hq = Hq;
+    if (static_cast<long long>(num_pages) * (Hkv > page_size ? Hkv : page_size) > 0x7fffffffLL) return FD_ERR_SHAPE;
+    PagedLayout pl{block_table, page_size, num_pages, max_pages_per_seq, kv_layout == FD_KV_NHD};
+    return run_split_paged(pr, pl, q_len, kv_type, k_scale, v_scale);
 }
 
 int fd_decode_multi(int B, int q_len, int Hq, int Hkv, int D, int max_len, const uint16_t *q,

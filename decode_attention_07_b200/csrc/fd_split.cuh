@@ -92,6 +92,7 @@ struct SplitParams {
     int max_pages;            // block-table row length (a multiple of 4)
     int page_shift;           // log2(page_size)
     int kv_nhd;               // 0: pages [num_pages, Hkv, page_size, D]; 1: [num_pages, page_size, Hkv, D]
+    int num_pages;            // pages in each pool
     // 8-bit caches only: value of a cached element = scale[kv head] * decode(code)
     const float *k_scale;     // [Hkv]
     const float *v_scale;     // [Hkv]
@@ -696,7 +697,6 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     // be waited on two phases ahead of a tile still in flight, where a parity
     // wait would pass on the older phase.
     static_assert(Cfg::kStages % kGroupsC == 0, "each consumer group must own whole stages");
-    static_assert(!kPaged || Consumer::kElemBytes == 2, "paged caches are bf16");
     constexpr int kStages = Cfg::kStages;
     constexpr int kBufs = Cfg::kMergeBufs;
 
@@ -840,11 +840,21 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                     const int nsub = psize >= kTileTokens ? 1 : min(kTileTokens >> p.page_shift, npages_seq - lp0);
                     const int off = psize >= kTileTokens ? (y & (psize - 1)) : 0;
                     int page[kTileTokens / 8];
-                    for (int j = 0; j < nsub; ++j)
-                        if (!page_of(c.b, lp0 + j, &page[j])) {
+                    int page1 = 0;   // the one page of a tile when page_size >= 64 (kept in a register)
+                    if (psize >= kTileTokens) {
+                        if (c.b == win_b && lp0 >= win_lo && lp0 < win_hi) {
+                            page1 = page_win[lp0 - win_lo];   // the common case: inside the window
+                        } else if (!page_of(c.b, lp0, &page1)) {
                             drain_copies<kStages>(full, seq, pbar, win_pending, win_phase);
                             return;
                         }
+                    } else {
+                        for (int j = 0; j < nsub; ++j)
+                            if (!page_of(c.b, lp0 + j, &page[j])) {
+                                drain_copies<kStages>(full, seq, pbar, win_pending, win_phase);
+                                return;
+                            }
+                    }
                     if constexpr (Consumer::kInterleaved) {
                         // one 5-D box per page, both halves of its tokens: [token][half][128 B].
                         // Coordinates {element, half, token, head, page} (head-major pages)
@@ -857,18 +867,27 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                             tma_load_5d(vt + j * page_bytes, &tm_v, &full[stage], 0, 0, cz, cw, page[j], policy);
                         }
                     } else {
-                        const uint32_t sub_bytes = static_cast<uint32_t>(rows) * 128u;
+                        // a page's rows of one box column land at j * rows box rows
+                        const uint32_t sub_bytes = static_cast<uint32_t>(rows) * Cfg::kBoxRowBytes;
                         mbar_arrive_expect_tx(&full[stage], 2u * nsub * sub_bytes * Cfg::kBoxes + qb);
                         for (int j = 0; j < nsub; ++j) {
+                            const int pgj = psize >= kTileTokens ? page1 : page[j];
 #pragma unroll
                             for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-                                const int dst = bx * kBoxBytes + j * rows * 128;
+                                const int dst = bx * Cfg::kBoxBytes + j * rows * Cfg::kBoxRowBytes;
+                                const int x = Cfg::kBoxCols * bx;
+                                // 3-D page maps: {element, token, page * Hkv + head} (head-major)
+                                // or {element, head, page * page_size + token} (token-major)
+                                // a page outside the pool gets a coordinate outside the tensor (zeros)
+                                const bool inside = pgj >= 0 && pgj < p.num_pages;
                                 if (p.kv_nhd) {
-                                    tma_load_4d(kt + dst, &tm_k, &full[stage], 64 * bx, c.h, off, page[j], policy);
-                                    tma_load_4d(vt + dst, &tm_v, &full[stage], 64 * bx, c.h, off, page[j], policy);
+                                    const int zz = inside ? pgj * (1 << p.page_shift) + off : -kTileTokens;
+                                    tma_load_3d(kt + dst, &tm_k, &full[stage], x, c.h, zz, policy);
+                                    tma_load_3d(vt + dst, &tm_v, &full[stage], x, c.h, zz, policy);
                                 } else {
-                                    tma_load_4d(kt + dst, &tm_k, &full[stage], 64 * bx, off, c.h, page[j], policy);
-                                    tma_load_4d(vt + dst, &tm_v, &full[stage], 64 * bx, off, c.h, page[j], policy);
+                                    const int zz = inside ? pgj * p.Hkv + c.h : -1;
+                                    tma_load_3d(kt + dst, &tm_k, &full[stage], x, off, zz, policy);
+                                    tma_load_3d(vt + dst, &tm_v, &full[stage], x, off, zz, policy);
                                 }
                             }
                         }

@@ -108,9 +108,13 @@ def make_paged(x: DecodeInputs, page_size: int, layout: str = "HND", seed: int =
     Sequence b needs ceil(seqlens[b] / page_size) pages; the pool holds those
     plus `spare_pages` more, in an order drawn from a CPU generator seeded
     `seed`. Block-table entries past a sequence's pages are `unused_entry`;
-    pool slots that no sequence position maps to are NaN."""
+    pool slots that no sequence position maps to are NaN (for an 8-bit cache,
+    QuantInputs: its padding code, and the pools hold codes)."""
     w = x.workload
-    dev = x.k.device
+    quant = hasattr(x, "k8")
+    src_k, src_v = (x.k8, x.v8) if quant else (x.k, x.v)
+    fill = (0x7F if x.kv_type == "e4m3" else 0x80) if quant else float("nan")
+    dev = src_k.device
     lens = np.clip(x.seqlens_host.astype(np.int64), 0, w.Lmax)
     need = [int(-(-int(L) // page_size)) for L in lens]
     max_pages = max(1, -(-w.Lmax // page_size))
@@ -120,8 +124,8 @@ def make_paged(x: DecodeInputs, page_size: int, layout: str = "HND", seed: int =
     order = torch.randperm(total, generator=g).numpy()
     table = np.full((w.B, max_pages), unused_entry, dtype=np.int32)
     shape = (total, w.Hkv, page_size, w.D) if layout == "HND" else (total, page_size, w.Hkv, w.D)
-    k_pages = torch.full(shape, float("nan"), dtype=torch.bfloat16, device=dev)
-    v_pages = torch.full(shape, float("nan"), dtype=torch.bfloat16, device=dev)
+    k_pages = torch.full(shape, fill, dtype=src_k.dtype, device=dev)
+    v_pages = torch.full(shape, fill, dtype=src_k.dtype, device=dev)
     nxt = 0
     for b in range(w.B):
         n = need[b]
@@ -131,10 +135,10 @@ def make_paged(x: DecodeInputs, page_size: int, layout: str = "HND", seed: int =
         nxt += n
         table[b, :n] = ids
         span = n * page_size
-        for src, dst in ((x.k, k_pages), (x.v, v_pages)):
+        for src, dst in ((src_k, k_pages), (src_v, v_pages)):
             part = src[b, :, :min(span, w.Lmax)]                           # [Hkv, tokens, D]
             if part.shape[1] < span:
-                pad = torch.full((w.Hkv, span - part.shape[1], w.D), float("nan"), dtype=part.dtype, device=dev)
+                pad = torch.full((w.Hkv, span - part.shape[1], w.D), fill, dtype=part.dtype, device=dev)
                 part = torch.cat([part, pad], dim=1)
             part = part.reshape(w.Hkv, n, page_size, w.D)
             part = part.permute(1, 0, 2, 3) if layout == "HND" else part.permute(1, 2, 0, 3)

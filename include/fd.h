@@ -234,6 +234,22 @@ FD_API int fd_decode_paged(int B, int Hq, int Hkv, int D, int page_size, int num
                            float *out, float *lse, void *workspace, size_t workspace_bytes,
                            int num_splits, void *stream);
 
+/* fd_decode_quant over a PAGED 8-bit cache: the page pools k_pages /
+ * v_pages hold codes (one byte per element) in the layouts of
+ * fd_decode_paged (kv_layout FD_KV_HND or FD_KV_NHD), found through the
+ * block table as there, and each element is dequantised with its kv head's
+ * scale as in fd_decode_quant (kv_type FD_KV_E4M3 or FD_KV_INT8). q_len
+ * queries per sequence as in fd_decode_multi. Page and block-table rules,
+ * alignment and errors: those of fd_decode_paged and fd_decode_quant;
+ * workspace: fd_workspace_bytes(B, Hq * q_len, Hkv, D,
+ * max_pages_per_seq * page_size, num_splits). */
+FD_API int fd_decode_quant_paged(int B, int q_len, int Hq, int Hkv, int D, int page_size, int num_pages,
+                                 int max_pages_per_seq, int kv_layout, int kv_type, const uint16_t *q,
+                                 const uint8_t *k_pages, const uint8_t *v_pages, const float *k_scale,
+                                 const float *v_scale, const int32_t *block_table, const int32_t *seqlens,
+                                 float scale, float *out, float *lse, void *workspace, size_t workspace_bytes,
+                                 int num_splits, void *stream);
+
 /* Split stage alone (one kernel): for each run of tiles, writes out/lse of
  * the rows it holds whole and the segments of the rows it holds in part.
  * Rows with no tokens and rows cut into several segments are left for

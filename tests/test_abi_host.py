@@ -211,6 +211,25 @@ def test_read_probe_argument_errors_without_a_device():
         assert L.fd_read_probe(p, 64, p, None) == -8
 
 
+def test_quant_paged_argument_errors_without_a_device():
+    L = fd.lib()
+    buf = (ctypes.c_uint8 * 4096)()
+    a16 = (ctypes.addressof(buf) + 15) // 16 * 16
+    p = ctypes.c_void_p(a16)
+
+    def qp(page_size=16, max_pages=4, layout=0, kv_type=1, q_len=1, Hq=4, D=128, bt=p, ks=p, S=1):
+        return L.fd_decode_quant_paged(1, q_len, Hq, 2, D, page_size, 8, max_pages, layout, kv_type, p, p, p, ks, p,
+                                       bt, p, 0.1, p, p, p, 4096, S, None)
+
+    assert qp(page_size=24) == -2 and qp(max_pages=6) == -2 and qp(layout=2) == -2
+    assert qp(kv_type=0) == -2 and qp(q_len=0) == -2
+    assert qp(q_len=9) == -3 and qp(Hq=3) == -3 and qp(D=96) == -4 and qp(S=-1) == -7
+    assert qp(bt=None) == -1 and qp(ks=None) == -1
+    assert qp(bt=ctypes.c_void_p(a16 + 4)) == -5 and qp(ks=ctypes.c_void_p(a16 + 2)) == -5
+    if not os.path.exists("/dev/nvidia0"):
+        assert qp() == -8
+
+
 def segments_rule(B, Hkv, Lmax, seqlens, P):
     """Independent statement of the documented partition: rows u = b*Hkv + j
     in order, ceil(L_b/64) tiles each, run i = flat tiles

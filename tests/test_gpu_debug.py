@@ -77,9 +77,14 @@ def run_child(debug, withhold=False):
     return json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("RESULT ")][-1][len("RESULT "):])
 
 
+@pytest.fixture(scope="module", autouse=True)
+def debug_library():
+    """The debug build, brought up to date with the sources (no-op when it is)."""
+    from decode_attention_07_b200 import build as lib_build
+    return lib_build.build(debug=True)
+
+
 def test_debug_build_checks_pass_and_match_release():
-    from decode_attention_07_b200 import _lib
-    assert os.path.exists(_lib.DEBUG_LIBRARY), "the debug build is made by __graft_entry__.build()"
     dbg = run_child(True)
     rel = run_child(False)
     for name, (status, osum, lsum) in dbg.items():

@@ -154,3 +154,52 @@ def test_lazy_max_fallback(kv_type, profile):
     for S in (1, 9, 148):
         out, lse = run(x, S=S)
         compare(out, lse, ref_o, ref_l, f"{kv_type} {profile} S={S}")
+
+
+# ------------------------------------------------------- paged 8-bit pools --
+
+from decode_attention_07_b200.inputs import make_paged  # noqa: E402
+
+
+@pytest.mark.parametrize("kv_type", KV)
+@pytest.mark.parametrize("page,layout,g,D", [(16, "HND", 4, 128), (8, "NHD", 1, 128), (64, "HND", 8, 128),
+                                             (256, "NHD", 16, 128), (16, "HND", 4, 64), (32, "NHD", 1, 64)])
+def test_paged_quant_equals_contiguous_and_oracle(kv_type, page, layout, g, D):
+    w = Workload("q8p", B=3, Hq=2 * g, Hkv=2, D=D, Lmax=1100, ragged=False, nan_pad=True)
+    x = make_quant(w, kv_type, seed=12, device="cuda", seqlens=[1100, 17, 530])
+    pg = make_paged(x, page, layout, seed=13, unused_entry=10 ** 6)
+    ref_o, ref_l = oracle_quant(x)
+    for S in (1, 23):
+        out, lse = fd.decode_quant_paged(x.q, pg.k_pages, pg.v_pages, x.k_scale, x.v_scale, kv_type, pg.block_table,
+                                         x.seqlens, x.scale, layout, num_splits=S)
+        o2, l2 = run(x, S=S)
+        torch.cuda.synchronize()
+        assert torch.equal(out, o2) and torch.equal(lse, l2), f"{kv_type} page {page} {layout} S={S}"
+        compare(out, lse, ref_o, ref_l, f"{kv_type} paged {page} {layout} g={g} D={D} S={S}")
+
+
+@pytest.mark.parametrize("kv_type", KV)
+def test_paged_quant_several_queries(kv_type):
+    w = Workload("q8p", B=2, Hq=8, Hkv=2, D=128, Lmax=900, ragged=False, nan_pad=True)
+    x = make_quant(w, kv_type, seed=14, device="cuda", seqlens=[900, 3])
+    g = torch.Generator(device="cuda").manual_seed(15)
+    q = torch.randn((w.B, 3, w.Hq, w.D), generator=g, device="cuda").to(torch.bfloat16)
+    pg = make_paged(x, 16, "HND", seed=16)
+    ref_o, ref_l = oracle_quant(x, q)
+    out, lse = fd.decode_quant_paged(q, pg.k_pages, pg.v_pages, x.k_scale, x.v_scale, kv_type, pg.block_table,
+                                     x.seqlens, x.scale, "HND", num_splits=11)
+    torch.cuda.synchronize()
+    compare(out, lse, ref_o, ref_l, f"{kv_type} paged, 3 queries")
+
+
+def test_paged_quant_full_size():
+    """ragged_64k with an E4M3 cache in 16-token pages, planned launch."""
+    w = WORKLOADS["ragged_64k"]
+    x = make_quant(w, "e4m3", seed=0, device="cuda")
+    pg = make_paged(x, 16, "HND", seed=1)
+    out, lse = fd.decode_quant_paged(x.q, pg.k_pages, pg.v_pages, x.k_scale, x.v_scale, "e4m3", pg.block_table,
+                                     x.seqlens, x.scale, "HND")
+    torch.cuda.synchronize()
+    bs = [0, w.B // 2, w.B - 1]
+    ref_o, ref_l = oracle_quant(x, bs=bs)
+    compare(out[bs], lse[bs], ref_o, ref_l, "ragged_64k e4m3 in 16-token pages")
