@@ -253,6 +253,17 @@ int debug_withhold() {
 #endif
 }
 
+// Debug builds: FD_DEBUG_SPOIL_GUESS=1 makes the split kernel's pre-wait guess
+// of each block's start wrong, to run the restart path. Release builds: off.
+int debug_spoil_guess() {
+#ifdef FD_DEBUG
+    const char *v = std::getenv("FD_DEBUG_SPOIL_GUESS");
+    return v != nullptr && v[0] == '1' ? 1 : 0;
+#else
+    return 0;
+#endif
+}
+
 // ---------------------------------------------------------------- launches --
 template <int D, class Consumer, bool kFused, bool kPaged>
 int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p, cudaStream_t st) {
@@ -429,6 +440,7 @@ int run_split(const Problem &pr, bool fused, int q_len = 1) {
     p.num_pages = 0;
     p.k_scale = p.v_scale = nullptr;
     p.debug_withhold = debug_withhold();
+    p.debug_spoil_guess = debug_spoil_guess();
     // with max_len == 0 every block finds zero tiles and only writes empty rows;
     // the (unused) tensor maps stay zeroed
     return fused ? launch_split<true>(pr.D, p.cols, tk, tv, p, pr.stream)
@@ -485,6 +497,7 @@ int run_split_paged(const Problem &pr, const PagedLayout &pl, int q_len = 1, int
     p.k_scale = k_scale;
     p.v_scale = v_scale;
     p.debug_withhold = debug_withhold();
+    p.debug_spoil_guess = debug_spoil_guess();
     if (quant)
         return kv_type == FD_KV_E4M3 ? launch_split_quant<true, true>(pr.D, p.cols, tk, tv, p, pr.stream)
                                      : launch_split_quant<false, true>(pr.D, p.cols, tk, tv, p, pr.stream);
@@ -533,6 +546,7 @@ int run_split_quant(const Problem &pr, int q_len, int kv_type, const float *k_sc
     p.k_scale = k_scale;
     p.v_scale = v_scale;
     p.debug_withhold = debug_withhold();
+    p.debug_spoil_guess = debug_spoil_guess();
     return kv_type == FD_KV_E4M3 ? launch_split_quant<true>(pr.D, p.cols, tk, tv, p, pr.stream)
                                  : launch_split_quant<false>(pr.D, p.cols, tk, tv, p, pr.stream);
 }

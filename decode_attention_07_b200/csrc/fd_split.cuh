@@ -97,6 +97,7 @@ struct SplitParams {
     const float *k_scale;     // [Hkv]
     const float *v_scale;     // [Hkv]
     int debug_withhold;       // debug builds: block 0 issues no copy for this tile (a wait then runs out); -1: off
+    int debug_spoil_guess;    // debug builds: make every block's pre-wait guess of its start wrong
 };
 
 // Sizes the debug checks compare with.
@@ -181,6 +182,7 @@ struct StartInfo {
     long long first;          // flat index of the start row's first tile
     int b, h, tile, n;
     int abort;                // set when a bounded wait gave up
+    int restart;              // the producer's guessed first tiles were wrong: the ring restarts one phase on
     int last_buf;             // merge buffer holding the run's last segment
     int npending;             // rows this block completed (fused form)
     PendingRow pending[kPendingMax];
@@ -296,6 +298,7 @@ __device__ __forceinline__ void find_start(const SplitParams &p, StartInfo *info
         }
     }
     if (lane == 0) {
+        info->restart = 0;
         info->count = t1 - t0;
         info->N = N;
         info->first = first;
@@ -710,7 +713,11 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     uint64_t *mempty = mfull + kBufs;                                      // merge buffer drained (finishers)
     uint64_t *pbar = mempty + kBufs;                                       // block-table window landed
     StartInfo *info = reinterpret_cast<StartInfo *>(pbar + 1);
-    float *weights = reinterpret_cast<float *>(info + 1);                  // [G][8] merge weights, [G] lse
+    StartInfo *guess = info + 1;                                           // the start as guessed before the wait
+    float *weights = reinterpret_cast<float *>(guess + 1);                 // [G][8] merge weights, [G] lse
+    static_assert((2 * kStages + 2 * kBufs + 1) * 8 + 2 * sizeof(StartInfo) + (G * kConsumerWarps + G) * 4 <=
+                      Cfg::kCtrlBytes,
+                  "control block over its bytes");
     int32_t *page_win = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(merge) +
                                                     kBufs * Cfg::kMergeFloats * 4 + Cfg::kCtrlBytes);
 
@@ -741,25 +748,86 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     // point of coherence, so a stale guess only wastes bandwidth; everything
     // below is recomputed from the real inputs after the wait.
     if (!kPaged && warp == 0) {
-        find_start<true>(p, info);
+        find_start<true>(p, guess);
+#ifdef FD_DEBUG
+        if (lane == 0 && p.debug_spoil_guess) guess->tile = guess->tile > 0 ? guess->tile - 1 : guess->tile + 1;
+#endif
         __syncwarp();
-        if (lane < 2 * kPrefetchTiles && info->count > 0) {
+        if (lane < 2 * kPrefetchTiles && guess->count > 0) {
             const int t = lane >> 1;
-            const int tile = info->tile + t;
-            if (t < info->count && tile < info->n) {
+            const int tile = guess->tile + t;
+            if (t < guess->count && tile < guess->n) {
                 const CUtensorMap *map = (lane & 1) ? &tm_v : &tm_k;
-                const int z = info->b * p.Hkv + info->h;
+                const int z = guess->b * p.Hkv + guess->h;
                 for (int bx = 0; bx < Cfg::kBoxes; ++bx)
                     tma_prefetch_l2_3d(map, Cfg::kBoxCols * bx, tile * kTileTokens, z);
             }
         }
         __syncwarp();
     }
+    __syncthreads();   // barrier inits and the guess are visible to every warp
     // Launched as a programmatic dependent of the previous kernel on the
     // stream: everything above overlaps its tail; inputs are read only after it.
     grid_dependency_wait();
-    if (warp == 0) find_start<false>(p, info);
+    // The producer starts on the guessed first tiles (up to one ring's worth,
+    // inside the first row) while warp 0 works out the real start from the
+    // inputs as they are now. When the two differ (the lengths changed under
+    // the guess), the ring restarts one phase on (below).
+    uint32_t n_spec = 0;
+    if (!kPaged && warp == kProducerWarp && lane == 0 && guess->count > 0) {
+        n_spec = static_cast<uint32_t>(min(static_cast<long long>(kStages),
+                                           min(static_cast<long long>(guess->n - guess->tile), guess->count)));
+        const uint64_t policy = l2_policy_evict_first();
+        const int z = guess->b * p.Hkv + guess->h;
+        const uint16_t *q_row =
+            p.q + (static_cast<size_t>(guess->b) * p.q_len * p.Hq + static_cast<size_t>(guess->h) * p.g) * D;
+        const uint32_t q_run = static_cast<uint32_t>(p.g) * D * 2;
+        const uint32_t q_bytes = static_cast<uint32_t>(p.cols) * D * 2;
+        for (uint32_t t = 0; t < n_spec; ++t) {   // tile t of the first segment into stage t, phase 0
+            uint8_t *kt = ring + t * Cfg::kStageBytes;
+            uint8_t *vt = kt + Cfg::kTileBytes;
+            const bool with_q = static_cast<int>(t) < kGroupsC;
+            const int y = (guess->tile + static_cast<int>(t)) * kTileTokens;
+            mbar_arrive_expect_tx(&full[t], 2 * Cfg::kTileBytes + (with_q ? q_bytes : 0u));
+#ifdef FD_DEBUG
+            if (blockIdx.x == 0 && static_cast<int>(t) == p.debug_withhold) continue;   // armed, never filled
+#endif
+#pragma unroll
+            for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+                tma_load_3d(kt + bx * Cfg::kBoxBytes, &tm_k, &full[t], Cfg::kBoxCols * bx, y, z, policy);
+                tma_load_3d(vt + bx * Cfg::kBoxBytes, &tm_v, &full[t], Cfg::kBoxCols * bx, y, z, policy);
+            }
+            if (with_q)
+                for (int j = 0; j < p.q_len; ++j)
+                    bulk_load(vt + Cfg::kTileBytes + j * q_run, q_row + static_cast<size_t>(j) * p.Hq * D, q_run,
+                              &full[t]);
+        }
+    }
+    if (warp == 0) {
+        find_start<false>(p, info);
+        if (lane == 0 && !kPaged && guess->count > 0)
+            info->restart = !(info->count == guess->count && info->N == guess->N && info->first == guess->first &&
+                              info->b == guess->b && info->h == guess->h && info->tile == guess->tile &&
+                              info->n == guess->n);
+    }
     __syncthreads();
+    // After a wrong guess (the same decision in every thread): the producer lets
+    // the guessed copies land (bounded), completes phase 0 of every stage with
+    // nothing else in it, and everyone goes on from sequence number kStages
+    // (stage s, phase 1). This finishes before any consumer waits on a stage:
+    // a wait for phase 1 while phase 0 is still open would pass at once.
+    const bool restart = info->restart != 0;
+    if (restart) {
+        if (warp == kProducerWarp && lane == 0)
+            for (int s2 = 0; s2 < kStages; ++s2) {
+                if (static_cast<uint32_t>(s2) < n_spec)
+                    drain_phase(&full[s2], 0);
+                else
+                    mbar_arrive(&full[s2]);
+                mbar_arrive_cnt(&empty[s2], kSlices);
+            }
+        __syncthreads();
+    }
 
     long long remaining = info->count;
     Cursor c{info->b, info->h, info->tile, info->n, info->first};
@@ -793,7 +861,9 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             *page = page_win[lp - win_lo];
             return true;
         };
-        uint32_t seq = 0;
+        // without a restart the guessed tiles already issued are the real first
+        // ones: skip them below; after a restart, go on from kStages
+        uint32_t seq = restart ? kStages : 0, skip = restart ? 0 : n_spec;
         while (remaining > 0) {
             const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
             const int z = c.b * p.Hkv + c.h;
@@ -803,6 +873,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             const uint32_t q_run = static_cast<uint32_t>(p.g) * D * 2;
             const int L = kPaged ? clamp_len(__ldg(p.seqlens + c.b), p.Lmax) : 0;
             for (int k = 0; k < seg; ++k, ++seq) {
+                if (seq < skip) continue;   // issued before the barrier, from the guess
                 const int stage = static_cast<int>(seq % kStages);
                 const uint32_t phase = (seq / kStages) & 1u;
                 // once a wait anywhere in the block gave up, issue nothing more (a
@@ -916,7 +987,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         const int group = warp / kSlices, slice = warp % kSlices;
         Consumer cons;
         cons.init(p);
-        uint32_t seq = 0, segctr = 0;
+        uint32_t seq = restart ? kStages : 0, segctr = 0;
         while (remaining > 0) {
             const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
             const int L = clamp_len(__ldg(p.seqlens + c.b), p.Lmax);

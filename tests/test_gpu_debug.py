@@ -68,6 +68,8 @@ def run_child(debug, withhold=False):
     env["FD_DEBUG"] = "1" if debug else "0"
     env.pop("FD_DEBUG_WITHHOLD", None)
     env.pop("FD_TEST_FAIL_LAUNCH", None)
+    if not debug:
+        env.pop("FD_DEBUG_SPOIL_GUESS", None)
     if withhold:
         env["WITHHOLD_TEST"] = "1"
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -91,6 +93,21 @@ def test_debug_build_checks_pass_and_match_release():
         assert status == 0, f"{name}: device status {status} in the debug build"
         assert rel[name][0] == 0
         assert (osum, lsum) == (rel[name][1], rel[name][2]), f"{name}: debug and release results differ"
+
+
+def test_a_wrong_start_guess_restarts_the_ring():
+    """FD_DEBUG_SPOIL_GUESS=1 makes every block's pre-wait guess of its start
+    wrong: the tiles issued from it are drained and the ring restarts one
+    phase on. Results must equal the release build's, with no error."""
+    os.environ["FD_DEBUG_SPOIL_GUESS"] = "1"
+    try:
+        dbg = run_child(True)
+    finally:
+        del os.environ["FD_DEBUG_SPOIL_GUESS"]
+    rel = run_child(False)
+    for name, (status, osum, lsum) in dbg.items():
+        assert status == 0, f"{name}: device status {status} with a spoiled guess"
+        assert (osum, lsum) == (rel[name][1], rel[name][2]), f"{name}: results differ after a restart"
 
 
 def test_a_wait_that_runs_out_is_reported():
