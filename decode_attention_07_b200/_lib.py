@@ -515,8 +515,9 @@ def fd_read_probe(buf, sink, stream=None):
 
 
 def workspace_layout(B, Hq, Hkv, D, num_splits):
-    """(slots, g, byte offset of seg_lse, byte offset of the row counters) of
-    the documented workspace layout."""
+    """(slots, g, byte offset of seg_lse, byte offset of the counters) of the
+    documented workspace layout. The counters are B*Hkv row counters followed
+    by `slots` chunk counters, all int32."""
     slots = num_splits + B * Hkv - 1
     g = Hq // Hkv
     off = (slots * g * D * 4 + 255) // 256 * 256

@@ -44,7 +44,8 @@ long long num_slots(int B, int Hkv, int num_splits) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Workspace: seg_out [slots][g][D] fp32 | seg_lse [slots][g] fp32 | row tickets [B*Hkv] int32,
+// Workspace: seg_out [slots][g][D] fp32 | seg_lse [slots][g] fp32 | row tickets [B*Hkv] int32
+// followed by chunk tickets [slots] int32,
 // each part 256-byte aligned.
 struct WorkspaceLayout {
     size_t seg_out, seg_lse, tickets, total;
@@ -58,7 +59,7 @@ WorkspaceLayout workspace_layout(int B, int Hq, int Hkv, int D, int num_splits) 
     w.seg_out = 0;
     w.seg_lse = align256(slots * g * D * sizeof(float));
     w.tickets = w.seg_lse + align256(slots * g * sizeof(float));
-    w.total = w.tickets + align256(static_cast<size_t>(B) * Hkv * sizeof(int));
+    w.total = w.tickets + align256((static_cast<size_t>(B) * Hkv + slots) * sizeof(int));
     return w;
 }
 
@@ -424,6 +425,7 @@ int run_split(const Problem &pr, bool fused, int q_len = 1) {
     p.out = pr.out;
     p.lse = pr.lse;
     seg_pointers(pr, &p.seg_out, &p.seg_lse, &p.row_tickets, q_len);
+    p.chunk_tickets = p.row_tickets ? p.row_tickets + static_cast<size_t>(pr.B) * pr.Hkv : nullptr;
     p.B = pr.B;
     p.Hq = pr.Hq;
     p.Hkv = pr.Hkv;
@@ -479,6 +481,7 @@ int run_split_paged(const Problem &pr, const PagedLayout &pl, int q_len = 1, int
     p.out = pr.out;
     p.lse = pr.lse;
     seg_pointers(pr, &p.seg_out, &p.seg_lse, &p.row_tickets, q_len);
+    p.chunk_tickets = p.row_tickets ? p.row_tickets + static_cast<size_t>(pr.B) * pr.Hkv : nullptr;
     p.B = pr.B;
     p.Hq = pr.Hq;
     p.Hkv = pr.Hkv;
@@ -529,6 +532,7 @@ int run_split_quant(const Problem &pr, int q_len, int kv_type, const float *k_sc
     p.out = pr.out;
     p.lse = pr.lse;
     seg_pointers(pr, &p.seg_out, &p.seg_lse, &p.row_tickets, q_len);
+    p.chunk_tickets = p.row_tickets ? p.row_tickets + static_cast<size_t>(pr.B) * pr.Hkv : nullptr;
     p.B = pr.B;
     p.Hq = pr.Hq;
     p.Hkv = pr.Hkv;

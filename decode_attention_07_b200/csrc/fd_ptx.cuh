@@ -103,6 +103,16 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         : "memory");
 }
 
+// 16 bytes global -> shared without passing through registers (the copy
+// reads at L2, bypassing L1). Both addresses 16-byte aligned. Completed by
+// cp_async_wait_all() in the issuing thread.
+__device__ __forceinline__ void cp_async_16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Ask for one 3-D tile to be brought into L2 (no shared memory, no barrier).
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int x, int y, int z) {
     asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
@@ -248,6 +258,16 @@ __device__ __forceinline__ void grid_dependents_launch() {
 }
 __device__ __forceinline__ void grid_dependency_wait() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Device-scope fetch-and-add with acquire-release semantics: the writes that
+// precede it (the calling thread's, and those it has seen through a block
+// barrier) are visible at device scope before the add, and whatever the
+// caller reads after it sees the writes released before earlier adds.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int *ptr, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+    return old;
 }
 
 __device__ __forceinline__ void named_barrier_sync(int id, int threads) {

@@ -61,7 +61,8 @@ constexpr int kFinisherWarps = 2;                 // warps 9, 10
 constexpr int kFinisherThreads = kFinisherWarps * 32;
 constexpr int kSplitThreads = kConsumerThreads + 32 + kFinisherThreads;
 constexpr int kWorkerThreads = kConsumerThreads + kFinisherThreads;   // all but the producer
-constexpr int kPendingMax = 4;                    // rows a block can complete (a run cuts at most 2)
+constexpr int kPendingMax = 4;                    // rows or chunks a block completes (a run cuts at most 2
+                                                  // rows; each completed chunk may complete its row)
 constexpr int kBarFinishers = 1, kBarWorkers = 2; // named barrier ids
 constexpr int kPrefetchTiles = 8;                 // tiles guessed into L2 before the dependency wait
 constexpr int kWarpTokens = 16;                   // default tokens of a tile owned by one consumer warp
@@ -83,6 +84,7 @@ struct SplitParams {
     float *seg_out;           // [slots, g, D]
     float *seg_lse;           // [slots, g]
     int *row_tickets;         // [B * Hkv], zero between calls (fused form only)
+    int *chunk_tickets;       // [slots], one per possible chunk start, zero between calls (fused form only)
     int B, Hq, Hkv, g, Lmax, P;
     int q_len;                // queries per sequence (1: plain decode)
     int cols;                 // g * q_len: (query, head) columns per (sequence, kv head) row
@@ -172,8 +174,9 @@ struct Cursor {
 };
 
 struct PendingRow {
-    long long first;          // flat index of the row's first tile
-    int b, h, n;              // the row and its tile count
+    int b, h;                 // the row
+    int chunk;                // -1: the row is complete; c >= 0: chunk c of a two-level row is
+    RowRuns rr;               // the runs holding the row's tiles
 };
 
 struct StartInfo {
@@ -186,6 +189,7 @@ struct StartInfo {
     int last_buf;             // merge buffer holding the run's last segment
     int npending;             // rows this block completed (fused form)
     PendingRow pending[kPendingMax];
+    RowRuns last_rr;          // the runs of the run's last segment's row (worked out ahead of its ticket)
 };
 
 // Bounded mbarrier wait. Returns false if the block is aborting or the limit
@@ -310,6 +314,65 @@ __device__ __forceinline__ void find_start(const SplitParams &p, StartInfo *info
         info->last_buf = 0;
         info->npending = 0;
     }
+}
+
+// What the end of a run merges, one entry per queued row or chunk, worked
+// out when it is queued (from runs worked out ahead: the partition
+// arithmetic divides 64-bit integers, too slow for the end of the run).
+enum EndMode : int { kEndChunk = 0, kEndDirect = 1, kEndStaged = 2, kEndFromL2 = 3 };
+constexpr int kDirectUnits = 8;   // units read straight from L2 (one round trip)
+struct EndPlan {
+    Units m[kPendingMax];      // the units the entry folds
+    int mode[kPendingMax];     // EndMode
+};
+
+// Queue a completed row (chunk = -1) or chunk, with its plan. `stage_floats`:
+// the floats of shared memory free at the end of the run.
+template <int D>
+__device__ __forceinline__ void queue_pending(const SplitParams &p, StartInfo *info, EndPlan *plan, int b, int h,
+                                              int chunk, const RowRuns &rr, long long stage_floats) {
+    if (!FD_DCHECK(info->npending < kPendingMax)) return;
+    const int k = info->npending++;
+    info->pending[k] = PendingRow{b, h, chunk, rr};
+    const long long u = static_cast<long long>(b) * p.Hkv + h;
+    if (chunk >= 0) {
+        plan->m[k] = chunk_units(rr, u, chunk);
+        plan->mode[k] = kEndChunk;
+    } else {
+        const Units m = final_units(rr, u);
+        plan->m[k] = m;
+        plan->mode[k] = m.count <= kDirectUnits                                    ? kEndDirect
+                        : staged_floats(m.count, p.cols, D) <= stage_floats ? kEndStaged
+                                                                             : kEndFromL2;
+    }
+}
+
+// ------------------------------------------------------------------ tickets --
+// Called by one thread once the block's segment of row c (runs rr) is stored
+// and ordered before this call by a block barrier: take the segment's
+// ticket, on the row or, for a two-level row, on the segment's chunk (the
+// block's run is blockIdx.x). The acquire-release add makes the stores
+// visible at device scope before the count moves, and orders the completing
+// block's reads of the other segments after it. A ticket that completes its
+// row or chunk queues it; nothing ever waits.
+template <int D>
+__device__ __forceinline__ void take_ticket(const SplitParams &p, StartInfo *info, EndPlan *plan, const Cursor &c,
+                                            const RowRuns &rr, long long N, long long stage_floats) {
+    const long long u = static_cast<long long>(c.b) * p.Hkv + c.h;
+    int *counter, need, chunk = -1;
+    if (!is_two_level(rr)) {
+        if (!FD_DCHECK(u < static_cast<long long>(p.B) * p.Hkv)) return;
+        counter = p.row_tickets + u;
+        need = rr.count;
+    } else {
+        chunk = (static_cast<int>(blockIdx.x) - rr.i0) / kFanIn;
+        const size_t slot = static_cast<size_t>(rr.i0) + static_cast<size_t>(chunk) * kFanIn + static_cast<size_t>(u);
+        if (!FD_DCHECK(chunk >= 0 && chunk < num_chunks(rr) && (slot + 1) * p.cols <= seg_rows(p))) return;
+        counter = p.chunk_tickets + slot;
+        need = chunk_count(rr, chunk, N, p.P);
+    }
+    const int prev = atom_add_acq_rel_gpu(counter, 1);
+    if (prev == need - 1) queue_pending<D>(p, info, plan, c.b, c.h, chunk, rr, stage_floats);
 }
 
 // ------------------------------------------------------------ merge + store --
@@ -715,7 +778,11 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     StartInfo *info = reinterpret_cast<StartInfo *>(pbar + 1);
     StartInfo *guess = info + 1;                                           // the start as guessed before the wait
     float *weights = reinterpret_cast<float *>(guess + 1);                 // [G][8] merge weights, [G] lse
-    static_assert((2 * kStages + 2 * kBufs + 1) * 8 + 2 * sizeof(StartInfo) + (G * kConsumerWarps + G) * 4 <=
+    constexpr int kWeightFloats = (G * kConsumerWarps + G + 3) / 4 * 4;
+    // shared memory free at the end of the run (the ring and merge buffers), in floats
+    constexpr long long kStageFloats = (static_cast<long long>(Cfg::kRingBytes) + kBufs * Cfg::kMergeFloats * 4) / 4;
+    EndPlan *plan = reinterpret_cast<EndPlan *>(weights + kWeightFloats);  // what the end of the run merges
+    static_assert((2 * kStages + 2 * kBufs + 1) * 8 + 2 * sizeof(StartInfo) + kWeightFloats * 4 + sizeof(EndPlan) <=
                       Cfg::kCtrlBytes,
                   "control block over its bytes");
     int32_t *page_win = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(merge) +
@@ -1022,12 +1089,28 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     } else {
         // ---------------------------------------------------- finishers --
         const int ftid = tid - (kProducerWarp + 1) * 32;
+        if (kFused) {
+            // rows without tokens (no segment, no ticket): out = 0, lse = -inf,
+            // written by block u % P while the first tiles are on their way
+            for (long long u = blockIdx.x; u < static_cast<long long>(p.B) * p.Hkv; u += p.P) {
+                const int b = static_cast<int>(u / p.Hkv), h = static_cast<int>(u % p.Hkv);
+                if (clamp_len(__ldg(p.seqlens + b), p.Lmax) != 0) continue;
+                for (int idx = ftid; idx < p.cols * (D / 4); idx += kFinisherThreads) {
+                    const int col = idx / (D / 4), d4 = idx - col * (D / 4);
+                    const size_t row = out_row(p, b, h, col);
+                    if (!FD_DCHECK(row < out_rows(p))) continue;
+                    reinterpret_cast<float4 *>(p.out + row * D)[d4] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (d4 == 0) p.lse[row] = -INFINITY;
+                }
+            }
+        }
         uint32_t segctr = 0;
         while (remaining > 0) {
             const int seg = static_cast<int>(min(static_cast<long long>(c.n - c.tile), remaining));
             if (seg == remaining) {   // the last segment: left for all workers at the end
                 last_c = c;
                 last_seg = seg;
+                if (kFused && ftid == 0) info->last_rr = row_runs(c.first, c.n, N, p.P);   // ahead of its ticket
                 break;
             }
             const bool whole = c.tile == 0 && seg == c.n;
@@ -1039,18 +1122,9 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                                         kFinisherThreads, [] { named_barrier_sync(kBarFinishers, kFinisherThreads); });
             named_barrier_sync(kBarFinishers, kFinisherThreads);   // every finisher is done with the buffer
             if (lane == 0) mbar_arrive(&mempty[buf]);
-            if (kFused && !whole) {
-                // ticket on the row; the block that completes it merges the row later
-                __threadfence();
-                named_barrier_sync(kBarFinishers, kFinisherThreads);
-                if (ftid == 0) {
-                    const RowRuns rr = row_runs(c.first, c.n, N, p.P);
-                    const int prev = FD_DCHECK(u < static_cast<long long>(p.B) * p.Hkv) ? atomicAdd(p.row_tickets + u, 1) : -1;
-                    if (prev == rr.count - 1 && info->npending < kPendingMax)
-                        info->pending[info->npending++] = PendingRow{c.first, c.b, c.h, c.n};
-                    __threadfence();   // acquire: the row's other segments are read after this
-                }
-            }
+            // the barrier above orders every finisher's stores before the ticket
+            if (kFused && !whole && ftid == 0)
+                take_ticket<D>(p, info, plan, c, row_runs(c.first, c.n, N, p.P), N, kStageFloats);
             ++segctr;
             remaining -= seg;
             if (remaining > 0) next_row(c, p);
@@ -1071,55 +1145,144 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         merge_warps_and_store<D, G>(merge + buf * Cfg::kMergeFloats, weights, p, last_c, whole, slot, wtid,
                                     kWorkerThreads, workers_sync);
         if (kFused && !whole) {
-            // ticket on the row: the writes above happen before the fence by
-            // the block barrier; the fence orders them before the atomic
-            workers_sync();
-            if (wtid == 0) {
-                __threadfence();
-                const RowRuns rr = row_runs(last_c.first, last_c.n, N, p.P);
-                const int prev = FD_DCHECK(u < static_cast<long long>(p.B) * p.Hkv) ? atomicAdd(p.row_tickets + u, 1) : -1;
-                if (prev == rr.count - 1 && info->npending < kPendingMax)
-                    info->pending[info->npending++] = PendingRow{last_c.first, last_c.b, last_c.h, last_c.n};
-                __threadfence();
-            }
+            workers_sync();   // the stores above, before the ticket
+            if (wtid == 0) take_ticket<D>(p, info, plan, last_c, info->last_rr, N, kStageFloats);
         }
         workers_sync();
     }
     if (kFused) {
-        // all queued rows at once: one float4 output per thread and step
-        const int npending = *reinterpret_cast<volatile int *>(&info->npending);
+        // Everything this block's tickets completed, with every worker:
+        //  1. chunks of two-level rows: merge the chunk's segments (at most
+        //     kFanIn: one L2 round trip) into its partial, written over the
+        //     slot of the chunk's first segment, then take the row's ticket;
+        //  2. complete rows: fold their units (segments, or the chunks'
+        //     partials) in order. Few units are read straight from L2 (one
+        //     round trip); more are staged in the ring and merge buffers (all
+        //     free now) with every copy in flight at once, as many rows
+        //     together as fit, and folded from there; a row too large to
+        //     stage is read from L2.
+        // One float4 output per thread and step throughout.
         constexpr int kVec = D / 4;
-        for (int idx = wtid; idx < npending * p.cols * kVec; idx += kWorkerThreads) {
-            const int i = idx / (p.cols * kVec), rem = idx - i * p.cols * kVec;
-            const int head = rem / kVec, d4 = rem - head * kVec;
-            const PendingRow r = info->pending[i];
-            const long long u = static_cast<long long>(r.b) * p.Hkv + r.h;
-            const RowRuns rr = row_runs(r.first, r.n, N, p.P);
-            const size_t row = out_row(p, r.b, r.h, head);
-            if (!FD_DCHECK(row < out_rows(p) &&
-                           (static_cast<size_t>(rr.i1) + u + 1) * p.cols <= seg_rows(p)))
-                continue;
-            float lse;
-            const float4 v = merge_row_vec<D>(p.seg_out, p.seg_lse, p.cols, static_cast<size_t>(rr.i0) + u,
-                                              rr.i1 - rr.i0 + 1, rr.i0, N, p.P, head, d4, &lse);
+        float *staged = reinterpret_cast<float *>(ring);
+        const int row_vec = p.cols * kVec;
+        auto entry_ok = [&](int k) {   // the entry's outputs and units lie inside their buffers
+            return FD_DCHECK(out_row(p, info->pending[k].b, info->pending[k].h, p.cols - 1) < out_rows(p) &&
+                             (plan->m[k].slot0 + static_cast<size_t>(plan->m[k].count - 1) * plan->m[k].stride + 1) *
+                                     p.cols <=
+                                 seg_rows(p));
+        };
+        auto store = [&](int k, int head, int d4, float4 v, float lse) {
+            const size_t row = out_row(p, info->pending[k].b, info->pending[k].h, head);
             reinterpret_cast<float4 *>(p.out + row * D)[d4] = v;
             if (d4 == 0) p.lse[row] = lse;
+        };
+
+        // (every entry and its plan were written before the last barrier)
+        int npending = *reinterpret_cast<volatile int *>(&info->npending);
+        bool any_chunk = false;
+        for (int k = 0; k < npending; ++k) any_chunk |= plan->mode[k] == kEndChunk;
+        if (any_chunk) {
+            // 1. outputs first; a chunk's lse is written only after the barrier,
+            //    since every thread of a head reads the lse slot it overwrites
+            for (int idx = wtid; idx < npending * row_vec; idx += kWorkerThreads) {
+                const int k = idx / row_vec, rem = idx - k * row_vec;
+                if (plan->mode[k] != kEndChunk || !entry_ok(k)) continue;
+                const Units m = plan->m[k];
+                const int head = rem / kVec, d4 = rem % kVec;
+                float lse;
+                const float4 v =
+                    merge_l2<D, 1>(p.seg_out, p.seg_lse, p.cols, m.slot0, m.count, m.i0, m.i1, N, p.P, head, d4, &lse);
+                reinterpret_cast<float4 *>(p.seg_out + (m.slot0 * p.cols + head) * D)[d4] = v;
+                if (d4 == 0) staged[k * p.cols + head] = lse;
+            }
+            workers_sync();
+            for (int v = wtid; v < npending * p.cols; v += kWorkerThreads) {
+                const int k = v / p.cols, head = v - k * p.cols;
+                if (plan->mode[k] != kEndChunk || !entry_ok(k)) continue;
+                const size_t slot0 = plan->m[k].slot0;
+                p.seg_lse[slot0 * p.cols + head] = staged[v];
+                if (head == 0) p.chunk_tickets[slot0] = 0;   // every segment of the chunk has arrived
+            }
+            workers_sync();   // the partials, before their row's ticket
+            if (wtid == 0) {
+                const int n0 = npending;
+                for (int k = 0; k < n0; ++k) {
+                    if (plan->mode[k] != kEndChunk) continue;
+                    const PendingRow r = info->pending[k];
+                    const long long u = static_cast<long long>(r.b) * p.Hkv + r.h;
+                    if (!FD_DCHECK(u < static_cast<long long>(p.B) * p.Hkv)) continue;
+                    const int prev = atom_add_acq_rel_gpu(p.row_tickets + u, 1);
+                    if (prev == row_chunk_count(r.rr, N, p.P) - 1)
+                        queue_pending<D>(p, info, plan, r.b, r.h, -1, r.rr, kStageFloats);
+                }
+            }
+            workers_sync();
+            npending = *reinterpret_cast<volatile int *>(&info->npending);
         }
-        if (wtid < npending) {   // every segment of that row has arrived: reset for the next call
+
+        // 2. complete rows: the direct ones together (one round trip for all)
+        for (int idx = wtid; idx < npending * row_vec; idx += kWorkerThreads) {
+            const int k = idx / row_vec, rem = idx - k * row_vec;
+            if (plan->mode[k] != kEndDirect || !entry_ok(k)) continue;
+            const int head = rem / kVec, d4 = rem % kVec;
+            const Units m = plan->m[k];
+            float lse;
+            const float4 v = merge_units_l2<D>(p.seg_out, p.seg_lse, p.cols, m, N, p.P, head, d4, &lse);
+            store(k, head, d4, v, lse);
+        }
+        for (int k = 0; k < npending; ++k) {   // too large to stage
+            if (plan->mode[k] != kEndFromL2 || !entry_ok(k)) continue;
+            const Units m = plan->m[k];
+            for (int idx = wtid; idx < row_vec; idx += kWorkerThreads) {
+                const int head = idx / kVec, d4 = idx % kVec;
+                float lse;
+                const float4 v = merge_units_l2<D>(p.seg_out, p.seg_lse, p.cols, m, N, p.P, head, d4, &lse);
+                store(k, head, d4, v, lse);
+            }
+        }
+        int i = 0;   // staged rows, as many together as fit
+        while (i < npending) {
+            if (plan->mode[i] != kEndStaged) {
+                ++i;
+                continue;
+            }
+            int j = i;
+            long long used = 0;
+            while (j < npending) {
+                const long long need =
+                    plan->mode[j] == kEndStaged ? staged_floats(plan->m[j].count, p.cols, D) : 0;
+                if (used + need > kStageFloats) break;
+                used += need;
+                ++j;
+            }
+            long long off = 0;
+            for (int k = i; k < j; ++k) {
+                if (plan->mode[k] != kEndStaged) continue;
+                if (entry_ok(k)) stage_units<D>(staged + off, p.seg_out, p.seg_lse, p.cols, plan->m[k], wtid, kWorkerThreads);
+                off += staged_floats(plan->m[k].count, p.cols, D);
+            }
+            cp_async_wait_all();
+            workers_sync();
+            off = 0;
+            for (int k = i; k < j; ++k) {
+                if (plan->mode[k] != kEndStaged) continue;
+                if (entry_ok(k)) {
+                    const Units m = plan->m[k];
+                    for (int idx = wtid; idx < row_vec; idx += kWorkerThreads) {
+                        const int head = idx / kVec, d4 = idx % kVec;
+                        float lse;
+                        const float4 v = merge_staged_vec<D>(staged + off, p.cols, m, N, p.P, head, d4, &lse);
+                        store(k, head, d4, v, lse);
+                    }
+                }
+                off += staged_floats(plan->m[k].count, p.cols, D);
+            }
+            workers_sync();   // before the next rows are staged over these
+            i = j;
+        }
+        if (wtid < npending && plan->mode[wtid] != kEndChunk) {   // every unit has arrived: reset for the next call
             const PendingRow r = info->pending[wtid];
             p.row_tickets[static_cast<long long>(r.b) * p.Hkv + r.h] = 0;
-        }
-        // rows without tokens: out = 0, lse = -inf, written by block u % P
-        for (long long u = blockIdx.x; u < static_cast<long long>(p.B) * p.Hkv; u += p.P) {
-            const int b = static_cast<int>(u / p.Hkv), h = static_cast<int>(u % p.Hkv);
-            if (clamp_len(__ldg(p.seqlens + b), p.Lmax) != 0) continue;
-            for (int idx = wtid; idx < p.cols * (D / 4); idx += kWorkerThreads) {
-                const int col = idx / (D / 4), d4 = idx - col * (D / 4);
-                const size_t row = out_row(p, b, h, col);
-                if (!FD_DCHECK(row < out_rows(p))) continue;
-                reinterpret_cast<float4 *>(p.out + row * D)[d4] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (d4 == 0) p.lse[row] = -INFINITY;
-            }
         }
     }
 }

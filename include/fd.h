@@ -28,9 +28,12 @@
  *              lse = -inf.
  * fd_decode runs both in ONE kernel: after writing a segment, a block takes a
  * ticket on its row (an atomic counter in the workspace; nothing waits), and
- * the block that completes the row performs its reduction. fd_split and
- * fd_combine run the two stages as separate kernels (same arithmetic, same
- * results bit for bit).
+ * the block that completes the row performs its reduction. A row cut into
+ * more than 32 segments is reduced in two levels: its segments 8 at a time
+ * (each group by the block completing it, through a counter of its own),
+ * then the groups' results. fd_split and fd_combine run the two stages as
+ * separate kernels (same arithmetic, same grouping, same results bit for
+ * bit).
  *
  * LAYOUTS (all row-major, contiguous, device memory unless stated)
  *   q        [B, Hq, D]          bf16 bit patterns (uint16_t), 16-byte aligned
@@ -110,11 +113,13 @@ FD_API int fd_plan_for_sms(int B, int Hq, int Hkv, int D, int max_len, int num_s
 
 /* Workspace bytes that fd_decode / fd_split / fd_combine need for
  * num_splits splits: room for (num_splits + B*Hkv - 1) segments of
- * Hq/Hkv rows, each D fp32 outputs plus one fp32 log-sum-exp, and one int32
- * counter per (sequence, kv-head) row, laid out as (each part 256-byte aligned)
+ * Hq/Hkv rows, each D fp32 outputs plus one fp32 log-sum-exp, one int32
+ * counter per (sequence, kv-head) row and one per segment slot (for the
+ * chunks of rows reduced in two levels), laid out as (each part 256-byte
+ * aligned)
  *     seg_out [num_segments][Hq/Hkv][D]  fp32
  *     seg_lse [num_segments][Hq/Hkv]     fp32
- *     tickets [B*Hkv]                    int32 (fd_decode only)
+ *     tickets [B*Hkv + num_segments]     int32 (fd_decode only)
  * Returns 0 when num_splits == 1 (no row is ever cut) or the arguments are
  * invalid. */
 FD_API size_t fd_workspace_bytes(int B, int Hq, int Hkv, int D, int max_len, int num_splits);

@@ -85,7 +85,7 @@ def test_workspace_bytes_formula():
         slots, g, off, tick = fd.workspace_layout(B, Hq, Hkv, D, S)
         assert off == (slots * g * D * 4 + 255) // 256 * 256
         assert tick == off + (slots * g * 4 + 255) // 256 * 256
-        want = tick + (B * Hkv * 4 + 255) // 256 * 256
+        want = tick + ((B * Hkv + slots) * 4 + 255) // 256 * 256   # row counters, then chunk counters
         assert fd.fd_workspace_bytes(B, Hq, Hkv, D, 1000, S) == want
         assert fd.fd_workspace_bytes(B, Hq, Hkv, D, 1000, 1) == 0
     assert fd.fd_workspace_bytes(1, 3, 2, 64, 10, 4) == 0          # invalid shape

@@ -56,6 +56,20 @@ def test_multi_query_against_oracle(q_len, g, D):
         compare(out, lse, ref_o, ref_l, f"q_len={q_len} g={g} D={D} S={S}")
 
 
+@pytest.mark.parametrize("q_len,Hq,Hkv,L", [(2, 32, 8, 8192), (2, 64, 8, 8192), (2, 16, 4, 8192),
+                                         (2, 8, 1, 16384)])
+def test_multi_query_long_rows(q_len, Hq, Hkv, L):
+    """Rows of ~19 segments (148 splits over 8 rows) with 8 and 16 columns
+    each (q_len * g; staged in shared memory), of ~37 segments (two levels)
+    and one row of 148 segments of 16 columns (two levels, 19 partials)."""
+    w = Workload("mq_long", B=1, Hq=Hq, Hkv=Hkv, D=128, Lmax=L, ragged=False, sigma_k=2.0)
+    x, q = multi_case(w, 6, q_len)
+    ref_o, ref_l = oracle_multi(x, q)
+    out, lse = fd.decode_multi(q, x.k, x.v, x.seqlens, x.scale, num_splits=148)
+    torch.cuda.synchronize()
+    compare(out, lse, ref_o, ref_l, f"q_len={q_len} Hq={Hq} Hkv={Hkv}")
+
+
 def test_queries_before_the_cache_start_are_empty():
     """A sequence shorter than q_len: the first queries see no token and
     give out = 0, lse = -inf."""

@@ -307,6 +307,51 @@ def test_fused_equals_two_stages(g, D, S):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+# Shapes that send the rows a block completes down each merge path of the
+# fused reduction: at most 8 segments (merged straight from L2), 9 to 32
+# (staged in shared memory, alone or two rows together, or from L2 when too
+# large), more than 32 (two levels: chunks of 8 segments, then the chunks'
+# partials, direct, staged or from L2), and more runs than tiles (empty runs
+# and empty chunks). Each is checked against the oracle, and bitwise against
+# the standalone combine kernel, which reads every segment from L2.
+MERGE_PATHS = [
+    # B, Hq, Hkv, D, Lmax, lens, S
+    (1, 32, 32, 128, 16384, None, None),        # 4-6 segments per row: direct
+    (1, 8, 8, 128, 8192, None, 148),            # ~19 segments, one column: staged
+    (1, 64, 8, 128, 8192, None, 148),           # ~19 segments of 8 columns, up to two rows a block
+    (1, 32, 2, 128, 8192, None, 60),            # 30 segments of 16 columns: too large to stage
+    (1, 4, 4, 64, 16384, None, 148),            # ~37 segments at D = 64: two levels, 5 partials
+    (1, 8, 1, 128, 65536, None, 148),           # one row of 148 segments: 19 partials, staged
+    (1, 16, 1, 64, 32768, None, 148),           # 16 columns at D = 64
+    (1, 16, 1, 128, 65536, None, 400),          # 400 segments of 16 columns: 50 partials, from L2
+    (1, 8, 1, 128, 6400, None, 148),            # 100 tiles over 148 runs: empty runs and chunks
+    (3, 24, 3, 128, 20000, (20000, 9000, 0), 148),   # long and short rows mixed, one sequence empty
+]
+
+
+@pytest.mark.parametrize("case", MERGE_PATHS, ids=lambda c: f"B{c[0]}-Hq{c[1]}-Hkv{c[2]}-D{c[3]}-L{c[4]}")
+def test_completed_row_merge_paths(case):
+    B, Hq, Hkv, D, Lmax, lens, S = case
+    w = Workload("merge", B=B, Hq=Hq, Hkv=Hkv, D=D, Lmax=Lmax, ragged=False, sigma_k=2.0)
+    x = make_inputs(w, 11, device="cuda", seqlens=list(lens) if lens else None)
+    S = S or fd.fd_plan(B, Hq, Hkv, D, Lmax)
+    nbytes = fd.fd_workspace_bytes(B, Hq, Hkv, D, Lmax, S)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    o1 = torch.empty((B, Hq, D), device="cuda")
+    l1 = torch.empty((B, Hq), device="cuda")
+    for _ in range(2):   # the second call reuses the row counters the first one reset
+        fd.fd_decode_splits(x.q, x.k, x.v, x.seqlens, x.scale, o1, l1, ws, S)
+    o2 = torch.full_like(o1, 5.0)
+    l2 = torch.full_like(l1, 5.0)
+    ws2 = torch.zeros_like(ws)
+    fd.fd_split(x.q, x.k, x.v, x.seqlens, x.scale, o2, l2, ws2, S)
+    fd.fd_combine(B, Hq, Hkv, D, Lmax, x.seqlens, o2, l2, ws2, S)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    ref_o, ref_l = oracle_rows(x)
+    compare(o1, l1, ref_o, ref_l, f"merge paths {case}")
+
+
 def test_workspace_reuse_leaves_counters_at_zero():
     """One workspace across calls with different inputs and lengths: every
     call is right, and the row counters are back at zero after each."""
@@ -315,7 +360,7 @@ def test_workspace_reuse_leaves_counters_at_zero():
     nbytes = fd.fd_workspace_bytes(w.B, w.Hq, w.Hkv, w.D, w.Lmax, S)
     ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
     fd.fd_workspace_init(ws)
-    _, _, _, tick = fd.workspace_layout(w.B, w.Hq, w.Hkv, w.D, S)
+    slots, _, _, tick = fd.workspace_layout(w.B, w.Hq, w.Hkv, w.D, S)
     out = torch.empty((w.B, w.Hq, w.D), device="cuda")
     lse = torch.empty((w.B, w.Hq), device="cuda")
     for seed, lens in ((1, [3000, 17, 0, 2999]), (2, [64, 3000, 1500, 1]), (3, [0, 0, 0, 700])):
@@ -324,4 +369,4 @@ def test_workspace_reuse_leaves_counters_at_zero():
         torch.cuda.synchronize()
         ref_o, ref_l = oracle_rows(x)
         compare(out, lse, ref_o, ref_l, f"reuse seed {seed}")
-        assert torch.all(ws[tick:tick + 4 * w.B * w.Hkv] == 0)
+        assert torch.all(ws[tick:tick + 4 * (w.B * w.Hkv + slots)] == 0)
