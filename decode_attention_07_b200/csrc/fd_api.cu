@@ -20,6 +20,7 @@ namespace {
 
 constexpr int kVersion = 100;               // 0.1.0
 constexpr int kMinTilesPerSplit = 4;        // a split streams at least 256 tokens per kv head
+constexpr int kMidTilesPerSm = 16;          // up to this many tiles per SM, splits come in multiples of 32
 constexpr int kMaxDevices = 64;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -638,6 +639,15 @@ int fd_plan_for_sms(int B, int Hq, int Hkv, int D, int max_len, int num_sms) {
     long long want = (tiles + kMinTilesPerSplit - 1) / kMinTilesPerSplit;
     if (want < 1) want = 1;
     if (want > num_sms) want = num_sms;
+    // Mid-size batches (at most kMidTilesPerSm tiles per SM): the reduction at
+    // the end of the runs weighs more than the last SMs' bandwidth, so use a
+    // multiple of 32 splits. Runs then line up with power-of-two row and tile
+    // counts, and fewer rows are cut (measured on B200: 8 rows of 128 tiles
+    // take 13.7 us with 128 splits, 20.6 us with 148).
+    if (num_sms >= 64 && tiles <= static_cast<long long>(kMidTilesPerSm) * num_sms) {
+        const long long aligned = num_sms / 32 * 32;
+        if (want > aligned) want = aligned;
+    }
     if (want > FD_MAX_SPLITS) want = FD_MAX_SPLITS;
     return static_cast<int>(want);
 }

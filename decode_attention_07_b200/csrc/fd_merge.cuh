@@ -9,7 +9,9 @@
 // Used by the split kernel's last block on a row (in-kernel combine) and by
 // the standalone combine kernel, so both produce bitwise the same values.
 //
-// A row cut into more than kTwoLevelSegs segments is reduced in two levels
+// A row cut into more than kTwoLevelSegs segments, or whose segments would
+// not fit the shared memory a block has free at the end of its run
+// (kStageBudgetFloats), is reduced in two levels
 // (the same formula applied to groups, which the formula allows: merging
 // merged groups gives the merge of all): its segments are taken kFanIn at a
 // time in slot order ("chunks"), each chunk is merged into one partial
@@ -42,9 +44,9 @@ __device__ __forceinline__ RowRuns row_runs(long long first, int n, long long N,
     RowRuns r;
     r.i0 = run_of_tile(first, N, P);
     r.i1 = run_of_tile(first + n - 1, N, P);
-    r.count = r.i1 - r.i0 + 1;
-    if (N < P)
-        for (int i = r.i0; i <= r.i1; ++i) r.count -= run_is_empty(i, N, P) ? 1 : 0;
+    // with more runs than tiles every run holds at most one tile, so the
+    // runs holding the row's n tiles are n distinct ones
+    r.count = N < P ? n : r.i1 - r.i0 + 1;
     return r;
 }
 
@@ -98,10 +100,26 @@ __device__ __forceinline__ float4 merge_end(const MergeState &st, float *lse) {
 }
 
 constexpr int kFanIn = 8;            // segments per chunk of a two-level row
-constexpr int kTwoLevelSegs = 32;    // rows with more segment slots are reduced in two levels
+constexpr int kTwoLevelSegs = 64;    // rows with more segment slots are reduced in two levels
+// Rows whose segments take more floats than this staged (outputs and lse)
+// are reduced in two levels too. Every split-kernel configuration that runs
+// more than one column has more shared memory free at the end of its run
+// (its ring and merge buffers); one column never gets near it.
+constexpr long long kStageBudgetFloats = 160 * 1024 / 4;
 
 __device__ __forceinline__ int row_slots(const RowRuns &rr) { return rr.i1 - rr.i0 + 1; }
-__device__ __forceinline__ bool is_two_level(const RowRuns &rr) { return row_slots(rr) > kTwoLevelSegs; }
+// Floats a merge's units take when staged in shared memory by stage_units:
+// outputs [count][g][D], then the lse values [count][g] padded to a multiple
+// of four (the next staged merge starts 16-byte aligned).
+__device__ __forceinline__ long long staged_floats(int count, int g, int D) {
+    const long long n = static_cast<long long>(count) * g;
+    return n * D + ((n + 3) & ~3LL);
+}
+
+// g: columns per row (query heads per kv head, times queries per sequence).
+__device__ __forceinline__ bool is_two_level(const RowRuns &rr, int g, int D) {
+    return row_slots(rr) > kTwoLevelSegs || staged_floats(row_slots(rr), g, D) > kStageBudgetFloats;
+}
 __device__ __forceinline__ int num_chunks(const RowRuns &rr) { return (row_slots(rr) + kFanIn - 1) / kFanIn; }
 
 // Runs of chunk c that hold tiles of the row: the chunk's ticket count.
@@ -144,8 +162,8 @@ __device__ __forceinline__ Units partial_units(const RowRuns &rr, long long u) {
     return Units{static_cast<size_t>(rr.i0) + static_cast<size_t>(u), kFanIn, num_chunks(rr), rr.i0, rr.i1};
 }
 // What the last reduction of a row folds.
-__device__ __forceinline__ Units final_units(const RowRuns &rr, long long u) {
-    return is_two_level(rr) ? partial_units(rr, u) : segment_units(rr, u);
+__device__ __forceinline__ Units final_units(const RowRuns &rr, long long u, int g, int D) {
+    return is_two_level(rr, g, D) ? partial_units(rr, u) : segment_units(rr, u);
 }
 
 // Runs a..b (a chunk) hold no tile: only possible with more runs than tiles.
@@ -216,7 +234,7 @@ __device__ __forceinline__ float4 merge_row_vec(const float *seg_out, const floa
                                                 const RowRuns &rr, long long N, int P, int head, int d4,
                                                 float *lse) {
     const size_t slot0 = static_cast<size_t>(rr.i0) + static_cast<size_t>(u);
-    if (!is_two_level(rr))
+    if (!is_two_level(rr, g, D))
         return merge_l2<D, 1>(seg_out, seg_lse, g, slot0, row_slots(rr), rr.i0, rr.i1, N, P, head, d4, lse);
     MergeState row = merge_begin();
     const int nc = num_chunks(rr);
@@ -229,14 +247,6 @@ __device__ __forceinline__ float4 merge_row_vec(const float *seg_out, const floa
         merge_fold(row, lc, oc);
     }
     return merge_end(row, lse);
-}
-
-// Floats a merge's units take when staged in shared memory by stage_units:
-// outputs [count][g][D], then the lse values [count][g] padded to a multiple
-// of four (the next staged merge starts 16-byte aligned).
-__device__ __forceinline__ long long staged_floats(int count, int g, int D) {
-    const long long n = static_cast<long long>(count) * g;
-    return n * D + ((n + 3) & ~3LL);
 }
 
 // Copy a merge's units to shared memory at dst, spread over `nthreads`

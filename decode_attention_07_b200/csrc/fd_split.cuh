@@ -339,7 +339,7 @@ __device__ __forceinline__ void queue_pending(const SplitParams &p, StartInfo *i
         plan->m[k] = chunk_units(rr, u, chunk);
         plan->mode[k] = kEndChunk;
     } else {
-        const Units m = final_units(rr, u);
+        const Units m = final_units(rr, u, p.cols, D);
         plan->m[k] = m;
         plan->mode[k] = m.count <= kDirectUnits                                    ? kEndDirect
                         : staged_floats(m.count, p.cols, D) <= stage_floats ? kEndStaged
@@ -360,7 +360,7 @@ __device__ __forceinline__ void take_ticket(const SplitParams &p, StartInfo *inf
                                             const RowRuns &rr, long long N, long long stage_floats) {
     const long long u = static_cast<long long>(c.b) * p.Hkv + c.h;
     int *counter, need, chunk = -1;
-    if (!is_two_level(rr)) {
+    if (!is_two_level(rr, p.cols, D)) {
         if (!FD_DCHECK(u < static_cast<long long>(p.B) * p.Hkv)) return;
         counter = p.row_tickets + u;
         need = rr.count;
@@ -781,6 +781,9 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     constexpr int kWeightFloats = (G * kConsumerWarps + G + 3) / 4 * 4;
     // shared memory free at the end of the run (the ring and merge buffers), in floats
     constexpr long long kStageFloats = (static_cast<long long>(Cfg::kRingBytes) + kBufs * Cfg::kMergeFloats * 4) / 4;
+    // a row reduced in one level always fits it
+    static_assert(kStageFloats >= (G == 1 ? kTwoLevelSegs * (D + 1) + 4 : kStageBudgetFloats),
+                  "a one-level row must fit the shared memory free at the end of the run");
     EndPlan *plan = reinterpret_cast<EndPlan *>(weights + kWeightFloats);  // what the end of the run merges
     static_assert((2 * kStages + 2 * kBufs + 1) * 8 + 2 * sizeof(StartInfo) + kWeightFloats * 4 + sizeof(EndPlan) <=
                       Cfg::kCtrlBytes,

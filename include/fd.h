@@ -100,7 +100,9 @@ extern "C" {
 
 /* Number of splits (thread blocks of the split stage) for a problem shape,
  * sized to the current device's SM count: one block per SM while the batch
- * holds at least 4 tiles (256 tokens) per block, fewer for small problems.
+ * holds at least 4 tiles (256 tokens) per block, fewer for small problems;
+ * with at most 16 tiles per SM (and at least 64 SMs) the count is also
+ * capped at the SM count rounded down to a multiple of 32 (128 on B200).
  * Pure function of its arguments and the SM count (queried once per device).
  * Returns num_splits >= 1, or a negative FD_ERR_* code.
  * Reading of the page's dispatcher (the library picks Flash-Decoding or a

@@ -53,9 +53,13 @@ def test_strerror_and_version():
 
 def plan_rule(B, Hq, Hkv, D, Lmax, sms):
     """The documented planner: one split per SM while every split keeps at
-    least 4 tiles of 64 tokens per kv head, fewer splits for small batches."""
+    least 4 tiles of 64 tokens per kv head, fewer splits for small batches;
+    with at most 16 tiles per SM (and 64 SMs or more) a multiple of 32."""
     tiles = B * Hkv * -(-Lmax // 64)
-    return max(1, min(sms, -(-tiles // 4)))
+    want = max(1, min(sms, -(-tiles // 4)))
+    if sms >= 64 and tiles <= 16 * sms:
+        want = min(want, sms // 32 * 32)
+    return want
 
 
 @pytest.mark.parametrize("name", list(WORKLOADS))
@@ -70,6 +74,9 @@ def test_plan_small_and_edge_shapes():
     assert fd.fd_plan_for_sms(1, 1, 1, 64, 1, 148) == 1
     assert fd.fd_plan_for_sms(1, 1, 1, 64, 0, 148) == 1
     assert fd.fd_plan_for_sms(2, 4, 2, 128, 64 * 4 * 10, 148) == 40   # 2*2*40 tiles / 4
+    assert fd.fd_plan_for_sms(1, 64, 8, 128, 8192, 148) == 128      # 1024 tiles: mid-size, a multiple of 32
+    assert fd.fd_plan_for_sms(1, 64, 8, 128, 8192 * 3, 148) == 148  # 3072 tiles: one per SM
+    assert fd.fd_plan_for_sms(1, 64, 8, 128, 8192, 60) == 60        # too few SMs to round
     L = fd.lib()
     assert L.fd_plan_for_sms(1, 3, 2, 128, 64, 148) == -3      # Hq % Hkv
     assert L.fd_plan_for_sms(1, 34, 2, 128, 64, 148) == -3     # group 17

@@ -60,8 +60,9 @@ def test_multi_query_against_oracle(q_len, g, D):
                                          (2, 8, 1, 16384)])
 def test_multi_query_long_rows(q_len, Hq, Hkv, L):
     """Rows of ~19 segments (148 splits over 8 rows) with 8 and 16 columns
-    each (q_len * g; staged in shared memory), of ~37 segments (two levels)
-    and one row of 148 segments of 16 columns (two levels, 19 partials)."""
+    each (q_len * g; staged in shared memory), of ~37 segments of 8 columns
+    (staged) and one row of 148 segments of 16 columns (two levels, 19
+    partials)."""
     w = Workload("mq_long", B=1, Hq=Hq, Hkv=Hkv, D=128, Lmax=L, ragged=False, sigma_k=2.0)
     x, q = multi_case(w, 6, q_len)
     ref_o, ref_l = oracle_multi(x, q)

@@ -308,19 +308,21 @@ def test_fused_equals_two_stages(g, D, S):
 
 
 # Shapes that send the rows a block completes down each merge path of the
-# fused reduction: at most 8 segments (merged straight from L2), 9 to 32
-# (staged in shared memory, alone or two rows together, or from L2 when too
-# large), more than 32 (two levels: chunks of 8 segments, then the chunks'
-# partials, direct, staged or from L2), and more runs than tiles (empty runs
-# and empty chunks). Each is checked against the oracle, and bitwise against
-# the standalone combine kernel, which reads every segment from L2.
+# fused reduction: at most 8 segments (merged straight from L2); up to 64
+# whose outputs fit 160 KB (staged in shared memory, alone or two rows
+# together); more, or larger (two levels: chunks of 8 segments, then the
+# chunks' partials, direct, staged or from L2); more runs than tiles (empty
+# runs and empty chunks). Each is checked against the oracle, and bitwise
+# against the standalone combine kernel, which reads every segment from L2.
 MERGE_PATHS = [
     # B, Hq, Hkv, D, Lmax, lens, S
     (1, 32, 32, 128, 16384, None, None),        # 4-6 segments per row: direct
     (1, 8, 8, 128, 8192, None, 148),            # ~19 segments, one column: staged
     (1, 64, 8, 128, 8192, None, 148),           # ~19 segments of 8 columns, up to two rows a block
-    (1, 32, 2, 128, 8192, None, 60),            # 30 segments of 16 columns: too large to stage
-    (1, 4, 4, 64, 16384, None, 148),            # ~37 segments at D = 64: two levels, 5 partials
+    (1, 4, 4, 64, 16384, None, 148),            # ~37 segments at D = 64: staged
+    (1, 32, 4, 128, 16384, None, 148),          # ~37 segments of 8 columns (148 KB): staged
+    (1, 24, 3, 128, 16384, None, 148),          # ~49 segments of 8 columns (196 KB): two levels, 7 partials direct
+    (1, 32, 2, 128, 8192, None, 60),            # 30 segments of 16 columns (240 KB): two levels, 4 partials
     (1, 8, 1, 128, 65536, None, 148),           # one row of 148 segments: 19 partials, staged
     (1, 16, 1, 64, 32768, None, 148),           # 16 columns at D = 64
     (1, 16, 1, 128, 65536, None, 400),          # 400 segments of 16 columns: 50 partials, from L2
