@@ -339,7 +339,10 @@ def run_fd(args, w, rank, world):
             g = torch.Generator(device=dev).manual_seed(rank_seed(args.seed, rank) + 77 + i)
             x.q = (torch.randn((w.B, Q, w.Hq, w.D), generator=g, device=dev) * w.sigma_q).to(torch.bfloat16)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if n_copies == 1 else None
-    counts = byte_counts(w, xs[0].seqlens_host, S, Q, 1 if quant else 2)
+    # the timed calls alternate over the copies, whose lengths differ on ragged
+    # workloads: the bytes of one launch are the copies' mean
+    per_copy = [byte_counts(w, x.seqlens_host, S, Q, 1 if quant else 2) for x in xs]
+    counts = {k: sum(c[k] for c in per_copy) / n_copies for k in per_copy[0]}
     kv_bytes = sum(x.kv_bytes() for x in xs) / n_copies
     if args.paged:
         # the same logical caches, scattered into shuffled page pools
