@@ -44,6 +44,12 @@ pg = make_paged(x, 16, "HND", seed=4)
 o, l = fd.decode_paged(x.q, pg.k_pages, pg.v_pages, pg.block_table, x.seqlens, x.scale, "HND", num_splits=9)
 torch.cuda.synchronize()
 res["paged"] = [fd.fd_device_status(), o.double().sum().item(), l[torch.isfinite(l)].double().sum().item()]
+wm = Workload("d4m", B=2, Hq=4, Hkv=4, D=128, Lmax=1500, ragged=False)
+xm = make_inputs(wm, 7, device="cuda", seqlens=[1500, 37])
+pg = make_paged(xm, 8, "NHD", seed=8, unused_entry=987654321)
+o, l = fd.decode_paged(xm.q, pg.k_pages, pg.v_pages, pg.block_table, xm.seqlens, xm.scale, "NHD", num_splits=5)
+torch.cuda.synchronize()
+res["paged_nhd8"] = [fd.fd_device_status(), o.double().sum().item(), l[torch.isfinite(l)].double().sum().item()]
 xq = make_quant(w, "e4m3", 5, device="cuda", seqlens=[1500, 700])
 o, l = fd.decode_quant(xq.q, xq.k8, xq.v8, xq.k_scale, xq.v_scale, "e4m3", xq.seqlens, xq.scale, num_splits=9)
 torch.cuda.synchronize()

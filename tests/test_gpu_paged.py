@@ -37,7 +37,7 @@ def paged_vs_contiguous(x, page_size, layout, S, unused_entry=-1, check_oracle=T
 
 @pytest.mark.parametrize("layout", ["HND", "NHD"])
 @pytest.mark.parametrize("page_size", [8, 16, 32, 64, 256])
-@pytest.mark.parametrize("g,D", [(4, 128), (1, 64), (8, 64), (16, 128)])
+@pytest.mark.parametrize("g,D", [(4, 128), (1, 64), (1, 128), (8, 64), (16, 128)])
 def test_paged_equals_contiguous(layout, page_size, g, D):
     w = Workload("paged", B=4, Hq=2 * g, Hkv=2, D=D, Lmax=3000, ragged=False, sigma_k=3.0, nan_pad=True)
     x = make_inputs(w, 9, device="cuda", seqlens=[3000, 1, 1777, 0])
@@ -81,3 +81,28 @@ def test_paged_ragged_64k_full_size(layout, page_size):
     bs = [int(np.argmax(x.seqlens_host)), int(np.argmin(x.seqlens_host)), 7]
     ref_o, ref_l = oracle_rows(x, bs)
     compare(out_p[bs], lse_p[bs], ref_o, ref_l, "ragged_64k paged")
+
+
+@pytest.mark.parametrize("layout", ["HND", "NHD"])
+@pytest.mark.parametrize("page_size", [8, 16, 64])
+@pytest.mark.parametrize("g", [1, 4])
+def test_page_outside_the_pool_reads_zeros(layout, page_size, g):
+    """A block-table entry past the pool (or negative) on a used page reads a
+    page of zeros for K and V instead of faulting: against the oracle on the
+    same cache with those tokens set to zero."""
+    w = Workload("paged", B=2, Hq=2 * g, Hkv=2, D=128, Lmax=600, ragged=False, nan_pad=True)
+    x = make_inputs(w, 11, device="cuda", seqlens=[600, 333])
+    pg = make_paged(x, page_size, layout, seed=3)
+    num_pages = pg.k_pages.shape[0]
+    bad = {(0, 1): num_pages + 5, (1, 2): -3}   # (sequence, logical page) -> out-of-pool index
+    for (b, lp), idx in bad.items():
+        pg.block_table[b, lp] = idx
+    S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.Lmax)
+    out, lse = fd.decode_paged(x.q, pg.k_pages, pg.v_pages, pg.block_table, x.seqlens, x.scale, layout=layout,
+                               num_splits=S)
+    torch.cuda.synchronize()
+    for (b, lp) in bad:
+        x.k[b, :, lp * page_size:(lp + 1) * page_size] = 0
+        x.v[b, :, lp * page_size:(lp + 1) * page_size] = 0
+    ref_o, ref_l = oracle_rows(x)
+    compare(out, lse, ref_o, ref_l, f"out-of-pool pages, {page_size} {layout}")
