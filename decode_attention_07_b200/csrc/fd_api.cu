@@ -269,7 +269,7 @@ int debug_spoil_guess() {
 // ---------------------------------------------------------------- launches --
 template <int D, class Consumer, bool kFused, bool kPaged>
 int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p, cudaStream_t st) {
-    constexpr int smem = fd::SplitConfig<D, Consumer::G, Consumer::kElemBytes>::kSmemBytes;
+    constexpr int smem = fd::SplitConfig<D, Consumer::G, Consumer::kElemBytes, kPaged>::kSmemBytes;
     auto kern = fd::fd_split_kernel<D, Consumer, kFused, kPaged>;
     // the attribute is per function and device; set it once per device
     static std::once_flag once[kMaxDevices];
@@ -291,7 +291,7 @@ int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::Split
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = dim3(static_cast<unsigned>(p.P));
-    cfg.blockDim = dim3(fd::kSplitThreads);
+    cfg.blockDim = dim3(fd::split_threads<kPaged>());
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

@@ -10,12 +10,13 @@
 // running max / running sum below do. A final reduction rescales the splits
 // by their log-sum-exps (fd_merge.cuh).
 //
-// Block layout (352 threads, one block per SM):
+// Block layout (352 threads, 384 for paged caches; one block per SM):
 //   warp 8      producer: one lane streams K and V tiles (64 tokens x D bf16
 //               each) from HBM into a ring of shared-memory stages with 3-D
 //               TMA loads, 128-byte swizzled, mbarrier completion; with each
 //               group's first tile of a row segment it also bulk-copies that
-//               row's query heads into the stage.
+//               row's query heads into the stage. Paged caches: it brings K
+//               and the query heads, and warp 11 (one lane) brings V.
 //   warps 0..7  consumers in two groups of four. Group q takes the tiles with
 //               sequence number = q (mod 2), so each SM sub-partition runs two
 //               independent chains; warp w of a group owns tokens
@@ -61,6 +62,13 @@ constexpr int kFinisherWarps = 2;                 // warps 9, 10
 constexpr int kFinisherThreads = kFinisherWarps * 32;
 constexpr int kSplitThreads = kConsumerThreads + 32 + kFinisherThreads;
 constexpr int kWorkerThreads = kConsumerThreads + kFinisherThreads;   // all but the producer
+// Paged caches add a second producer, warp 11, that brings the V boxes while
+// warp 8 brings K and the query heads: a TMA copy costs its issuing thread a
+// fixed time, which dominates the small boxes of small pages, and copies from
+// two warps start in parallel.
+constexpr int kVProducerWarp = kProducerWarp + 1 + kFinisherWarps;
+template <bool kPaged>
+constexpr int split_threads() { return kSplitThreads + (kPaged ? 32 : 0); }
 constexpr int kPendingMax = 4;                    // rows or chunks a block completes (a run cuts at most 2
                                                   // rows; each completed chunk may complete its row)
 constexpr int kBarFinishers = 1, kBarWorkers = 2; // named barrier ids
@@ -136,7 +144,7 @@ __device__ __forceinline__ size_t out_row(const SplitParams &p, int b, int h, in
 }
 
 // E = bytes per cached element: 2 (bf16) or 1 (8-bit codes).
-template <int D, int G, int E = 2>
+template <int D, int G, int E = 2, bool kPaged = false>
 struct SplitConfig {
     static constexpr int kRowBytes = D * E;                                // one token of one head
     static constexpr int kBoxRowBytes = kRowBytes < 128 ? kRowBytes : 128; // a box row = one swizzle span
@@ -150,7 +158,7 @@ struct SplitConfig {
     static constexpr int kMergeFloats = kConsumerWarps * kWarpFloats;      // one merge buffer
     static constexpr int kCtrlBytes = 2048;                                // barriers, start info, queue, weights
     static constexpr int kPageBytes = kPageWindow * 4;                     // block-table window (paged)
-    static constexpr int kFixedBytes = 1024 + kCtrlBytes + kPageBytes;
+    static constexpr int kFixedBytes = 1024 + kCtrlBytes + (kPaged ? 2 : 1) * kPageBytes;   // one window per producer
     // 128 KiB of K/V tiles in flight (measured best for bf16: 4 stages at
     // D = 128), as many as fit next to one merge buffer, in whole pairs
     static constexpr int fit_stages(int s) {
@@ -751,11 +759,11 @@ struct HeadConsumer {
 
 // ------------------------------------------------------------------ kernel --
 template <int D, class Consumer, bool kFused, bool kPaged = false>
-__global__ void __launch_bounds__(kSplitThreads, 1)
+__global__ void __launch_bounds__(split_threads<kPaged>(), 1)
     fd_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const SplitParams p) {
     constexpr int G = Consumer::G;
-    using Cfg = SplitConfig<D, G, Consumer::kElemBytes>;
+    using Cfg = SplitConfig<D, G, Consumer::kElemBytes, kPaged>;
     constexpr int kTok = Consumer::kWarpTokens;          // tokens per consumer warp and tile
     constexpr int kSlices = kTileTokens / kTok;           // warps per consumer group
     constexpr int kGroupsC = kConsumerWarps / kSlices;    // groups taking turns on tiles
@@ -774,8 +782,8 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     uint64_t *empty = full + kStages;
     uint64_t *mfull = empty + kStages;                                     // merge buffer filled (8 warps)
     uint64_t *mempty = mfull + kBufs;                                      // merge buffer drained (finishers)
-    uint64_t *pbar = mempty + kBufs;                                       // block-table window landed
-    StartInfo *info = reinterpret_cast<StartInfo *>(pbar + 1);
+    uint64_t *pbar = mempty + kBufs;                                       // block-table windows landed (K, V)
+    StartInfo *info = reinterpret_cast<StartInfo *>(pbar + 2);
     StartInfo *guess = info + 1;                                           // the start as guessed before the wait
     float *weights = reinterpret_cast<float *>(guess + 1);                 // [G][8] merge weights, [G] lse
     constexpr int kWeightFloats = (G * kConsumerWarps + G + 3) / 4 * 4;
@@ -785,7 +793,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     static_assert(kStageFloats >= (G == 1 ? kTwoLevelSegs * (D + 1) + 4 : kStageBudgetFloats),
                   "a one-level row must fit the shared memory free at the end of the run");
     EndPlan *plan = reinterpret_cast<EndPlan *>(weights + kWeightFloats);  // what the end of the run merges
-    static_assert((2 * kStages + 2 * kBufs + 1) * 8 + 2 * sizeof(StartInfo) + kWeightFloats * 4 + sizeof(EndPlan) <=
+    static_assert((2 * kStages + 2 * kBufs + 2) * 8 + 2 * sizeof(StartInfo) + kWeightFloats * 4 + sizeof(EndPlan) <=
                       Cfg::kCtrlBytes,
                   "control block over its bytes");
     int32_t *page_win = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(merge) +
@@ -799,7 +807,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], kPaged ? 2 : 1);   // paged caches: the K and the V producer arrive
             mbar_init(&empty[s], kSlices);
         }
         for (int b = 0; b < kBufs; ++b) {
@@ -807,6 +815,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
             mbar_init(&mempty[b], kFinisherWarps);
         }
         mbar_init(pbar, 1);
+        mbar_init(pbar + 1, 1);
         fence_mbar_init();
     }
     if (warp == kProducerWarp && lane == 0) {   // kernel parameters, not inputs: safe before the wait
@@ -905,12 +914,17 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
     volatile int *abort = &info->abort;
     const uint32_t q_bytes = static_cast<uint32_t>(p.cols) * D * 2;   // q_len copies of g rows
 
-    if (warp == kProducerWarp) {
+    // paged caches: warp 8 brings K and the query heads, warp 11 brings V
+    const bool v_role = kPaged && warp == kVProducerWarp;
+    if (warp == kProducerWarp || v_role) {
         // ---------------------------------------------------- producer --
         if (lane != 0 || remaining <= 0) return;
         const uint64_t policy = l2_policy_evict_first();
         // paged caches: a window of the current sequence's block-table row in
-        // shared memory, fetched with a 1-D bulk copy when a page falls outside it
+        // shared memory, fetched with a 1-D bulk copy when a page falls outside
+        // it (one window and barrier per producer)
+        uint64_t *wbar = pbar + (v_role ? 1 : 0);
+        int32_t *win = page_win + (v_role ? kPageWindow : 0);
         int win_b = -1, win_lo = 0, win_hi = 0;
         uint32_t win_phase = 0;
         bool win_pending = false;   // a window copy issued and not yet seen complete
@@ -920,15 +934,15 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                 win_lo = lp & ~3;
                 win_hi = min(win_lo + kPageWindow, p.max_pages);
                 const uint32_t bytes = static_cast<uint32_t>(win_hi - win_lo) * 4u;
-                mbar_arrive_expect_tx(pbar, bytes);
+                mbar_arrive_expect_tx(wbar, bytes);
                 if (FD_DCHECK(b < p.B && win_lo >= 0 && win_lo < win_hi))
-                    bulk_load(page_win, p.block_table + static_cast<size_t>(b) * p.max_pages + win_lo, bytes, pbar);
+                    bulk_load(win, p.block_table + static_cast<size_t>(b) * p.max_pages + win_lo, bytes, wbar);
                 win_pending = true;
-                if (!wait_bounded(pbar, win_phase, abort)) return false;
+                if (!wait_bounded(wbar, win_phase, abort)) return false;
                 win_pending = false;
                 win_phase ^= 1u;
             }
-            *page = page_win[lp - win_lo];
+            *page = win[lp - win_lo];
             return true;
         };
         // without a restart the guessed tiles already issued are the real first
@@ -949,16 +963,17 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                 // once a wait anywhere in the block gave up, issue nothing more (a
                 // stage whose copy never completed must not be armed again)
                 if (*abort || !wait_bounded(&empty[stage], phase ^ 1u, abort)) {
-                    drain_copies<kStages>(full, seq, pbar, win_pending, win_phase);
+                    drain_copies<kStages>(full, seq, wbar, win_pending, win_phase);
                     return;
                 }
                 uint8_t *kt = ring + stage * Cfg::kStageBytes;
                 uint8_t *vt = kt + Cfg::kTileBytes;
-                const bool with_q = k < kGroupsC;   // each group's first tile of the segment
+                const bool with_q = k < kGroupsC && !v_role;   // each group's first tile of the segment
                 const uint32_t qb = with_q ? q_bytes : 0u;
 #ifdef FD_DEBUG
                 if (blockIdx.x == 0 && static_cast<int>(seq) == p.debug_withhold) {
-                    mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kTileBytes + qb);   // armed, never filled
+                    // armed, never filled
+                    mbar_arrive_expect_tx(&full[stage], (kPaged ? 1 : 2) * Cfg::kTileBytes + qb);
                     continue;
                 }
 #endif
@@ -984,15 +999,15 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                     int page1 = 0;   // the one page of a tile when page_size >= 64 (kept in a register)
                     if (psize >= kTileTokens) {
                         if (c.b == win_b && lp0 >= win_lo && lp0 < win_hi) {
-                            page1 = page_win[lp0 - win_lo];   // the common case: inside the window
+                            page1 = win[lp0 - win_lo];   // the common case: inside the window
                         } else if (!page_of(c.b, lp0, &page1)) {
-                            drain_copies<kStages>(full, seq, pbar, win_pending, win_phase);
+                            drain_copies<kStages>(full, seq, wbar, win_pending, win_phase);
                             return;
                         }
                     } else {
                         for (int j = 0; j < nsub; ++j)
                             if (!page_of(c.b, lp0 + j, &page[j])) {
-                                drain_copies<kStages>(full, seq, pbar, win_pending, win_phase);
+                                drain_copies<kStages>(full, seq, wbar, win_pending, win_phase);
                                 return;
                             }
                     }
@@ -1001,16 +1016,18 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                         // Coordinates {element, half, token, head, page} (head-major pages)
                         // or {element, half, head, token, page} (token-major pages).
                         const uint32_t page_bytes = static_cast<uint32_t>(rows) * D * 2;
-                        mbar_arrive_expect_tx(&full[stage], 2u * nsub * page_bytes + qb);
+                        mbar_arrive_expect_tx(&full[stage], nsub * page_bytes + qb);
                         const int cz = p.kv_nhd ? c.h : off, cw = p.kv_nhd ? off : c.h;
-                        for (int j = 0; j < nsub; ++j) {
-                            tma_load_5d(kt + j * page_bytes, &tm_k, &full[stage], 0, 0, cz, cw, page[j], policy);
-                            tma_load_5d(vt + j * page_bytes, &tm_v, &full[stage], 0, 0, cz, cw, page[j], policy);
-                        }
+                        const CUtensorMap *map = v_role ? &tm_v : &tm_k;
+                        uint8_t *dst = v_role ? vt : kt;
+                        for (int j = 0; j < nsub; ++j)
+                            tma_load_5d(dst + j * page_bytes, map, &full[stage], 0, 0, cz, cw, page[j], policy);
                     } else {
                         // a page's rows of one box column land at j * rows box rows
                         const uint32_t sub_bytes = static_cast<uint32_t>(rows) * Cfg::kBoxRowBytes;
-                        mbar_arrive_expect_tx(&full[stage], 2u * nsub * sub_bytes * Cfg::kBoxes + qb);
+                        mbar_arrive_expect_tx(&full[stage], nsub * sub_bytes * Cfg::kBoxes + qb);
+                        const CUtensorMap *map = v_role ? &tm_v : &tm_k;
+                        uint8_t *dstb = v_role ? vt : kt;
                         for (int j = 0; j < nsub; ++j) {
                             const int pgj = psize >= kTileTokens ? page1 : page[j];
 #pragma unroll
@@ -1023,12 +1040,10 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
                                 const bool inside = pgj >= 0 && pgj < p.num_pages;
                                 if (p.kv_nhd) {
                                     const int zz = inside ? pgj * (1 << p.page_shift) + off : -kTileTokens;
-                                    tma_load_3d(kt + dst, &tm_k, &full[stage], x, c.h, zz, policy);
-                                    tma_load_3d(vt + dst, &tm_v, &full[stage], x, c.h, zz, policy);
+                                    tma_load_3d(dstb + dst, map, &full[stage], x, c.h, zz, policy);
                                 } else {
                                     const int zz = inside ? pgj * p.Hkv + c.h : -1;
-                                    tma_load_3d(kt + dst, &tm_k, &full[stage], x, off, zz, policy);
-                                    tma_load_3d(vt + dst, &tm_v, &full[stage], x, off, zz, policy);
+                                    tma_load_3d(dstb + dst, map, &full[stage], x, off, zz, policy);
                                 }
                             }
                         }
@@ -1046,7 +1061,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1)
         }
         // after an abort the consumers no longer wait for the last stages: the
         // producer keeps the block alive until its copies have landed
-        if (*abort) drain_copies<kStages>(full, seq, pbar, win_pending, win_phase);
+        if (*abort) drain_copies<kStages>(full, seq, wbar, win_pending, win_phase);
         return;
     }
 
