@@ -158,6 +158,14 @@ def byte_counts(w, lens, S, q_len=1, elem_bytes=2):
                 segments=n_part, whole_rows=n_whole, multi_rows=multi_rows)
 
 
+def launch_bytes(w, lens_per_copy, S, q_len=1, elem_bytes=2):
+    """Algorithmic bytes of one launch when the timed calls alternate over
+    input copies with these lengths (ragged copies differ): the copies' mean
+    of byte_counts."""
+    per_copy = [byte_counts(w, lens, S, q_len, elem_bytes) for lens in lens_per_copy]
+    return {k: sum(c[k] for c in per_copy) / len(per_copy) for k in per_copy[0]}
+
+
 # ------------------------------------------------------------- the CPU arm --
 
 def oracle_sample(x, budget_s=12.0, nthreads=0, collect=None):
@@ -339,10 +347,7 @@ def run_fd(args, w, rank, world):
             g = torch.Generator(device=dev).manual_seed(rank_seed(args.seed, rank) + 77 + i)
             x.q = (torch.randn((w.B, Q, w.Hq, w.D), generator=g, device=dev) * w.sigma_q).to(torch.bfloat16)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if n_copies == 1 else None
-    # the timed calls alternate over the copies, whose lengths differ on ragged
-    # workloads: the bytes of one launch are the copies' mean
-    per_copy = [byte_counts(w, x.seqlens_host, S, Q, 1 if quant else 2) for x in xs]
-    counts = {k: sum(c[k] for c in per_copy) / n_copies for k in per_copy[0]}
+    counts = launch_bytes(w, [x.seqlens_host for x in xs], S, Q, 1 if quant else 2)
     kv_bytes = sum(x.kv_bytes() for x in xs) / n_copies
     if args.paged:
         # the same logical caches, scattered into shuffled page pools

@@ -61,3 +61,26 @@ def test_gpu_arm_line():
     p = d["parity"]
     assert p["max_abs_err_out"] <= p["tolerance"]["out_abs"] and p["max_rel_err_lse"] <= p["tolerance"]["lse_rel"]
     assert d["per_call"]["median_us"] > 0 and d["read_probe"]["gbs"] > 0
+
+
+def test_launch_bytes_average_the_rotated_copies():
+    """The timed calls alternate over input copies; on a ragged workload the
+    copies' lengths differ, so one launch's algorithmic bytes are their mean.
+    K/V bytes are counted inside the sequences only (2 bytes per bf16
+    element, K and V)."""
+    import numpy as np
+
+    import bench
+    from decode_attention_07_b200.configs import WORKLOADS
+
+    w = WORKLOADS["ragged_64k"]
+    a = np.array([1, 65536] + [4096] * (w.B - 2), dtype=np.int32)
+    b = np.array([777] * w.B, dtype=np.int32)
+    S = 148
+    kv = lambda lens: int(lens.astype(np.int64).sum()) * w.Hkv * w.D * 2 * 2
+    one = bench.launch_bytes(w, [a], S)
+    assert one == bench.byte_counts(w, a, S) and one["kv"] == kv(a)
+    two = bench.launch_bytes(w, [a, b], S)
+    assert two["kv"] == (kv(a) + kv(b)) / 2
+    assert two["total"] == (bench.byte_counts(w, a, S)["total"] + bench.byte_counts(w, b, S)["total"]) / 2
+    assert two["q"] == w.B * w.Hq * w.D * 2
