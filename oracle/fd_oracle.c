@@ -94,7 +94,11 @@ static double e4m3_to_double(uint8_t c) {
     if (e == 0)
         mag = ldexp(m / 8.0, -6);
     else
+#if FDO_MUTANT == 13
+        mag = ldexp(1.0 + m / 8.0, e - 8);         /* planted: exponent bias 8 */
+#else
         mag = ldexp(1.0 + m / 8.0, e - 7);
+#endif
 #endif
     return s ? -mag : mag;
 }
@@ -172,7 +176,11 @@ static void row_logits(const job_t *J, int b, int i, const uint16_t *qrow, int t
     for (int t = t0; t < t1; ++t) {
         const size_t krow = (((size_t)b * J->Hkv + j) * J->Lmax + t) * J->D;
         double dot = 0.0;
+#if FDO_MUTANT == 12
+        for (int d = 0; d < J->D - 1; ++d) dot += bf16_to_double(qrow[d]) * key_at(J, krow + d, j);   /* planted */
+#else
         for (int d = 0; d < J->D; ++d) dot += bf16_to_double(qrow[d]) * key_at(J, krow + d, j);
+#endif
 #if FDO_MUTANT == 1
         z[t - t0] = dot;                           /* planted: scale dropped */
 #else
@@ -200,7 +208,11 @@ static double row_softmax_sum(const job_t *J, int b, int i, int t0, int t1,
     for (int t = t0; t < t1; ++t) {
         const double w = exp(z[t - t0] - M);
         const size_t vrow = (((size_t)b * J->Hkv + j) * J->Lmax + t) * J->D;
+#if FDO_MUTANT == 14
+        for (int d = 0; d < J->D; ++d) o[d] += w * value_at(J, vrow + (J->D - 1 - d), j);   /* planted */
+#else
         for (int d = 0; d < J->D; ++d) o[d] += w * value_at(J, vrow + d, j);
+#endif
     }
 #if FDO_MUTANT != 6
     for (int d = 0; d < J->D; ++d) o[d] /= Z;       /* mutant 6 plants: no normalisation */

@@ -1,7 +1,7 @@
 """Each planted mistake in the oracle (FDO_MUTANT in fd_oracle.c) must be
 caught by at least one pin: this shows the pins constrain every step of the
 oracle (scale, group mapping, sequence length, log base, value operand,
-normalisation, split reduction, causal offset, dequantisation)."""
+normalisation, split reduction, causal offset, dequantisation, the dot product's terms, the value operand's index)."""
 import pytest
 
 import oracle
@@ -20,6 +20,9 @@ MUTANTS = {
     9: "E4M3 subnormal codes decoded as normals",
     10: "values dequantised with the key scale",
     11: "int8 codes read as unsigned",
+    12: "dot product drops the last head-dim term",
+    13: "E4M3 exponent bias 8 instead of 7",
+    14: "output dimension d reads value dimension D-1-d",
 }
 
 
