@@ -5,10 +5,15 @@ of the workload, inputs resident in HBM. Prints ONE JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl fd|reference]
 
-Multi-GPU (torchrun, one process per GPU): every rank decodes its own
-independent batch of the same shape (seed + rank); nothing is exchanged on the
-data path, so scaling is weak and value = sum over ranks of KV bytes / the
-slowest rank's device time.
+Multi-GPU, one process per GPU: under torchrun (WORLD_SIZE set, and equal to
+--gpus), or, with --gpus N > 1 and no WORLD_SIZE, bench.py starts the N ranks
+itself. Every rank decodes its own independent batch of the same shape (seed +
+rank); nothing is exchanged on the data path, so scaling is weak and value =
+sum over ranks of KV bytes / the slowest rank's device time.
+
+At one GPU on the headline workload the line also carries per_config: every
+other workload (and the 8-bit caches of the two long batch-1 ones) measured
+the same way in the same run.
 
 The reference arm (--impl reference) is the CPU oracle (fp64, host cores) on
 a bounded sample of the same workload.
@@ -288,91 +293,232 @@ def read_probe_gbs(dev, stream, nbytes=2 << 30, reps=10):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     gbs = nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    timed_out = probe_timed_out(int(sink.item()))
     del buf
     torch.cuda.empty_cache()
-    return gbs
+    return None if timed_out else gbs
 
 
-def per_call_stats(call_at, dev, stream, steps):
-    """Each call timed alone with CUDA events, L2 flushed before it by a
-    write of twice its size (outside the events): median, p10, p90 in us."""
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+def probe_timed_out(sink_word: int) -> bool:
+    """fd_read_probe folds data into the low 32 bits of its sink and sets the
+    upper half when a bounded wait gave up (a pass that stopped early would
+    report an inflated rate)."""
+    return ((sink_word >> 32) & 0x7FFFFFFF) != 0
+
+
+class L2Flush:
+    """Evicts the caller's data from L2 between isolated calls: a write of
+    twice L2's size, then a read of another buffer of twice its size, so L2
+    is left holding clean lines (a timed call that starts behind the write
+    alone would first pay for writing back ~L2 of dirty lines)."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self, i):
+        self.w.fill_(i & 255)
+        self.r.sum()
+
+
+def per_call_stats(call_at, dev, stream, steps, flush=None):
+    """Each call timed alone with CUDA events, L2 flushed before it (outside
+    the events, see L2Flush): median, p10, p90 in us."""
+    flush = flush or L2Flush(dev)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for i in range(steps):
-        flush.fill_(i & 255)
+        flush(i)
         ev[i][0].record(stream)
         call_at(i)
         ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     t = np.array([a.elapsed_time(b) * 1e3 for a, b in ev])
-    del flush
     return {"median_us": float(np.median(t)), "p10_us": float(np.percentile(t, 10)),
             "p90_us": float(np.percentile(t, 90)), "calls": steps,
-            "l2": "flushed before every call (write of 2x L2, outside the events)"}
+            "l2": "flushed before every call: write of 2x L2, then read of another 2x L2 (outside the events)"}
+
+
+class Workspace:
+    """One workload's inputs, outputs, workspace and prepared calls on this
+    rank: `calls[i]` enqueues one call on input copy i (two copies rotated
+    when a copy is larger than L2, so no call finds its predecessor's bytes
+    in L2; one copy otherwise, with L2 flushed before every timed call)."""
+
+    def __init__(self, w, kv, seed, dev, stream, q_len=1, paged=0, layout="HND"):
+        self.w, self.kv, self.dev, self.stream = w, kv, dev, stream
+        self.quant = kv != "bf16"
+        self.S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.Lmax)
+        S, Q = self.S, q_len
+
+        def draw(sd):
+            if self.quant:
+                from decode_attention_07_b200.inputs import make_quant
+                return make_quant(w, kv, sd, device=dev)
+            return make_inputs(w, sd, device=dev)
+
+        xs = [draw(seed)]
+        kv_per_copy = xs[0].kv_bytes()
+        self.n_copies = 2 if kv_per_copy >= L2_BYTES else 1
+        self.l2_note = (f"inputs larger than L2: 2 input copies of {kv_per_copy / 1e6:.0f} MB rotated"
+                        if self.n_copies == 2 else
+                        "L2 flushed before every timed call (write of 2x L2 then read of 2x L2, outside the events)")
+        for c in range(1, self.n_copies):
+            xs.append(draw(seed + 1000 * c))
+        nbytes = fd.fd_workspace_bytes(w.B, w.Hq * Q, w.Hkv, w.D, w.Lmax, S)
+        self.ws = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=dev)   # row counters start at zero
+        oshape = (w.B, w.Hq) if Q == 1 else (w.B, Q, w.Hq)
+        out = torch.empty(oshape + (w.D,), dtype=torch.float32, device=dev)
+        lse = torch.empty(oshape, dtype=torch.float32, device=dev)
+        self.out, self.lse = out, lse
+        if Q > 1:
+            # q_len new tokens per sequence: queries [B, q_len, Hq, D] drawn like q
+            for i, x in enumerate(xs):
+                g = torch.Generator(device=dev).manual_seed(seed + 77 + i)
+                x.q = (torch.randn((w.B, Q, w.Hq, w.D), generator=g, device=dev) * w.sigma_q).to(torch.bfloat16)
+        self.counts = launch_bytes(w, [x.seqlens_host for x in xs], S, Q, 1 if self.quant else 2)
+        self.kv_bytes = sum(x.kv_bytes() for x in xs) / self.n_copies
+        ws = self.ws
+        if paged:
+            # the same logical caches, scattered into shuffled page pools
+            from decode_attention_07_b200.inputs import make_paged
+            pgs = [make_paged(x, paged, layout, seed=7 + i) for i, x in enumerate(xs)]
+            for x in xs:   # the contiguous copies are not used by the paged calls
+                if self.quant:
+                    x.k8 = x.v8 = None
+                else:
+                    x.k = x.v = None
+            torch.cuda.empty_cache()
+            if self.quant:
+                self.calls = [fd.prepare_decode_quant_paged(x.q, pg.k_pages, pg.v_pages, x.k_scale, x.v_scale, kv,
+                                                            pg.block_table, x.seqlens, x.scale, out, lse, ws, layout,
+                                                            S, stream) for x, pg in zip(xs, pgs)]
+            else:
+                self.calls = [fd.prepare_decode_paged(x.q, pg.k_pages, pg.v_pages, pg.block_table, x.seqlens,
+                                                      x.scale, out, lse, ws, layout, S, stream)
+                              for x, pg in zip(xs, pgs)]
+            self.pages = pgs
+        elif self.quant:
+            self.calls = [fd.prepare_decode_quant(x.q, x.k8, x.v8, x.k_scale, x.v_scale, kv, x.seqlens, x.scale, out,
+                                                  lse, ws, S, stream) for x in xs]
+        elif Q > 1:
+            self.calls = [fd.prepare_decode_multi(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream)
+                          for x in xs]
+        else:
+            self.calls = [fd.prepare_decode(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream) for x in xs]
+        self.xs = xs
+        self.flush = L2Flush(dev) if self.n_copies == 1 else None
+
+    def call(self, i):
+        self.calls[i % self.n_copies]()
+
+    def timed(self, steps):
+        """Device milliseconds of `steps` calls: back to back over the rotated
+        copies (one event pair), or, for a workload that fits in L2, call by
+        call with L2 flushed before each (flush outside the events)."""
+        st = self.stream
+        if self.flush is None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            for i in range(steps):
+                self.call(i)
+            e1.record(st)
+            torch.cuda.synchronize(self.dev)
+            return e0.elapsed_time(e1)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            self.flush(i)
+            ev[i][0].record(st)
+            self.call(0)
+            ev[i][1].record(st)
+        torch.cuda.synchronize(self.dev)
+        return sum(a.elapsed_time(b) for a, b in ev)
+
+    def parity_rows(self):
+        """(b, kv head) rows checked against the oracle: the first and the
+        last sequence, each with its last kv head (empty rows skipped)."""
+        w = self.w
+        rows = []
+        for b in sorted({0, w.B - 1}):
+            if int(min(max(self.xs[0].seqlens_host[b], 0), w.Lmax)) > 0:
+                rows.append((b, w.Hkv - 1))
+        return rows
+
+    def parity(self, rows=None):
+        """One call on input copy 0, then the oracle on `rows`: max-abs error
+        on out, relative error on lse (floored at 1)."""
+        import oracle
+        w, x = self.w, self.xs[0]
+        orc = oracle.default()
+        self.calls[0]()
+        torch.cuda.synchronize(self.dev)
+        o_gpu, l_gpu = self.out.double().cpu().numpy(), self.lse.double().cpu().numpy()
+        err_o, err_l, n = 0.0, 0.0, 0
+        for b, j in rows if rows is not None else self.parity_rows():
+            L = int(min(max(x.seqlens_host[b], 0), w.Lmax))
+            qh = bf16_bits(x.q[b:b + 1, j * w.g:(j + 1) * w.g])
+            if self.quant:
+                o, lo = orc.attention_quant(qh, x.k8[b:b + 1, j:j + 1, :L].cpu().numpy(),
+                                            x.v8[b:b + 1, j:j + 1, :L].cpu().numpy(), x.k_scale[j:j + 1].cpu().numpy(),
+                                            x.v_scale[j:j + 1].cpu().numpy(), np.array([L], np.int32), x.scale,
+                                            x.kv_type)
+            else:
+                o, lo = orc.attention(qh, bf16_bits(x.k[b:b + 1, j:j + 1, :L]), bf16_bits(x.v[b:b + 1, j:j + 1, :L]),
+                                      np.array([L], np.int32), x.scale)
+            og, lg = o_gpu[b, j * w.g:(j + 1) * w.g], l_gpu[b, j * w.g:(j + 1) * w.g]
+            err_o = max(err_o, float(np.abs(og - o[0]).max()))
+            fin = np.isfinite(lo[0])
+            if fin.any():
+                err_l = max(err_l, float((np.abs(lg[fin] - lo[0][fin]) / np.maximum(1.0, np.abs(lo[0][fin]))).max()))
+            n += w.g
+        return {"max_abs_err_out": err_o, "max_rel_err_lse": err_l, "rows": n,
+                "tolerance": {"out_abs": 2e-3, "lse_rel": 1e-4},
+                "against": "oracle (fp64): the first and last sequence, last kv head, all its query heads"}
+
+
+def config_entry(args, w, kv, dev, stream, peak):
+    """One workload measured like the headline, for the line's per_config
+    object: back-to-back and isolated us per call, KV and algorithmic
+    bandwidth, roofline fraction, and oracle parity on sampled rows."""
+    wk = Workspace(w, kv, args.seed, dev, stream)
+    for i in range(max(3, args.warmup)):
+        wk.call(i)
+    torch.cuda.synchronize(dev)
+    ms = wk.timed(args.steps)
+    us = ms * 1e3 / args.steps
+    iso = per_call_stats(wk.call, dev, stream, max(10, min(args.steps, 20)))
+    achieved = wk.counts["total"] / (us * 1e-6) / 1e9
+    key = w.name + (f":{kv}" if kv != "bf16" else "")
+    entry = {
+        "workload": w.name, "kv_cache": kv, "num_splits": wk.S, "l2": wk.l2_note,
+        "timing": "back to back over rotated copies" if wk.flush is None else "call by call, L2 flushed before each",
+        "us_per_call": us, "us_per_call_isolated": iso,
+        "kv_gbs": wk.kv_bytes / (us * 1e-6) / 1e9,
+        "pct_of_nominal_hbm_kv": 100.0 * wk.kv_bytes / (us * 1e-6) / 1e9 / NOMINAL_HBM_GBS,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS, "bytes_per_launch": wk.counts["total"],
+                     "traffic": measured_traffic(key)},
+        "parity": wk.parity(),
+        "steps": args.steps,
+    }
+    del wk
+    torch.cuda.empty_cache()
+    return key, entry
+
+
+# workloads measured beside the headline in the per_config object (name, cache type)
+PER_CONFIG = [("tiny_mha", "bf16"), ("gqa_128k", "bf16"), ("batch_4k", "bf16"), ("ragged_64k", "bf16"),
+              ("mha_16k", "e4m3"), ("gqa_128k", "e4m3")]
 
 
 def run_fd(args, w, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
-    S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.Lmax)
     quant = args.kv != "bf16"
-
-    def draw(seed):
-        if quant:
-            from decode_attention_07_b200.inputs import make_quant
-            return make_quant(w, args.kv, seed, device=dev)
-        return make_inputs(w, seed, device=dev)
-
-    xs = [draw(rank_seed(args.seed, rank))]
-    kv_per_copy = xs[0].kv_bytes()
-    if kv_per_copy >= L2_BYTES:
-        # rotate input copies so every call streams bytes that are not in L2
-        n_copies = 2
-        l2_note = f"inputs larger than L2: {n_copies} input copies of {kv_per_copy / 1e6:.0f} MB rotated"
-    else:
-        n_copies = 1
-        l2_note = "L2 flushed before every timed call (256 MiB write outside the timed events)"
-    for c in range(1, n_copies):
-        xs.append(draw(rank_seed(args.seed, rank) + 1000 * c))
     Q = args.q_len
-    nbytes = fd.fd_workspace_bytes(w.B, w.Hq * Q, w.Hkv, w.D, w.Lmax, S)
-    ws = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=dev)      # row counters start at zero
-    oshape = (w.B, w.Hq) if Q == 1 else (w.B, Q, w.Hq)
-    out = torch.empty(oshape + (w.D,), dtype=torch.float32, device=dev)
-    lse = torch.empty(oshape, dtype=torch.float32, device=dev)
-    if Q > 1:
-        # q_len new tokens per sequence: queries [B, q_len, Hq, D] drawn like q
-        for i, x in enumerate(xs):
-            g = torch.Generator(device=dev).manual_seed(rank_seed(args.seed, rank) + 77 + i)
-            x.q = (torch.randn((w.B, Q, w.Hq, w.D), generator=g, device=dev) * w.sigma_q).to(torch.bfloat16)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if n_copies == 1 else None
-    counts = launch_bytes(w, [x.seqlens_host for x in xs], S, Q, 1 if quant else 2)
-    kv_bytes = sum(x.kv_bytes() for x in xs) / n_copies
-    if args.paged:
-        # the same logical caches, scattered into shuffled page pools
-        from decode_attention_07_b200.inputs import make_paged
-        pgs = [make_paged(x, args.paged, args.layout, seed=7 + i) for i, x in enumerate(xs)]
-        for x in xs:   # the contiguous copies are not used by the paged calls
-            if quant:
-                x.k8 = x.v8 = None
-            else:
-                x.k = x.v = None
-        torch.cuda.empty_cache()
-        if quant:
-            calls = [fd.prepare_decode_quant_paged(x.q, pg.k_pages, pg.v_pages, x.k_scale, x.v_scale, args.kv,
-                                                   pg.block_table, x.seqlens, x.scale, out, lse, ws, args.layout, S,
-                                                   stream) for x, pg in zip(xs, pgs)]
-        else:
-            calls = [fd.prepare_decode_paged(x.q, pg.k_pages, pg.v_pages, pg.block_table, x.seqlens, x.scale, out,
-                                             lse, ws, args.layout, S, stream) for x, pg in zip(xs, pgs)]
-    elif quant:
-        calls = [fd.prepare_decode_quant(x.q, x.k8, x.v8, x.k_scale, x.v_scale, args.kv, x.seqlens, x.scale, out, lse,
-                                         ws, S, stream) for x in xs]
-    elif Q > 1:
-        calls = [fd.prepare_decode_multi(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream) for x in xs]
-    else:
-        calls = [fd.prepare_decode(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream) for x in xs]
+    wk = Workspace(w, args.kv, rank_seed(args.seed, rank), dev, stream, Q, args.paged, args.layout)
+    S, n_copies, xs, out, lse, ws = wk.S, wk.n_copies, wk.xs, wk.out, wk.lse, wk.ws
+    counts, kv_bytes, calls = wk.counts, wk.kv_bytes, wk.calls
 
     def barrier():
         if world > 1:
@@ -380,62 +526,59 @@ def run_fd(args, w, rank, world):
 
     probe = read_probe_gbs(dev, stream) if rank == 0 else None
     for i in range(max(3, args.warmup)):
-        calls[i % n_copies]()
+        wk.call(i)
     torch.cuda.synchronize(dev)
 
-    # ---- main timed region: K calls back to back, one event pair ---------
-    # (the small workload, whose inputs fit in L2, is instead flushed before
-    # each call and timed call by call, flush outside the events)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps if flush is not None else 1)]
+    # ---- main timed region: K calls back to back (or, for a workload that
+    # fits in L2, call by call with L2 flushed outside the events) ---------
     barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clocks:
         t_wall = time.perf_counter()
-        if flush is None:
-            ev[0][0].record(stream)
-            for i in range(args.steps):
-                calls[i % n_copies]()
-            ev[0][1].record(stream)
-        else:
-            for i in range(args.steps):
-                flush.fill_(i & 255)
-                ev[i][0].record(stream)
-                calls[0]()
-                ev[i][1].record(stream)
-        torch.cuda.synchronize(dev)
+        ms_local = wk.timed(args.steps)
         # keep the sampler on the same work for >= 1.5 s so clocks are seen under load
         t_min = time.perf_counter() + (0.0 if args.no_clock_window else 1.5)
         j = 0
         while time.perf_counter() < t_min:
             for _ in range(50):
-                calls[j % n_copies]()
+                wk.call(j)
                 j += 1
             torch.cuda.synchronize(dev)
         wall = time.perf_counter() - t_wall
     barrier()
-    ms_max = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev)
+    ms_max = max_over_ranks(ms_local, dev)
     us_per_call = ms_max * 1e3 / args.steps
     gbs = whole_job_gbs(world, kv_bytes, args.steps, ms_max)
 
-    per_call = per_call_stats(lambda i: calls[i % n_copies](), dev, stream, max(10, min(args.steps, 50)))
+    per_call = per_call_stats(wk.call, dev, stream, max(10, min(args.steps, 50)))
 
     # ---- the two stages as separate kernels (for the per-stage split) ------
-    ev_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-             torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps if not args.paged and Q == 1 and not quant else 0)]
-    for i in range(len(ev_s)):
-        x = xs[i % n_copies]
-        if flush is not None:
-            flush.fill_(i & 255)
-        ev_s[i][0].record(stream)
-        fd.fd_split(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream)
-        ev_s[i][1].record(stream)
-        fd.fd_combine(w.B, w.Hq, w.Hkv, w.D, w.Lmax, x.seqlens, out, lse, ws, S, stream)
-        ev_s[i][2].record(stream)
-    torch.cuda.synchronize(dev)
-    split_us = 1e3 * sum(a.elapsed_time(b) for a, b, _ in ev_s) / max(1, len(ev_s)) if ev_s else None
-    combine_us = 1e3 * sum(b.elapsed_time(c) for _, b, c in ev_s) / max(1, len(ev_s)) if ev_s else None
+    # Each stage is bracketed by its own events with a host sync between the
+    # two, so the combine is timed alone (not overlapped with the split's
+    # tail by its programmatic dependent launch); L2 is flushed before each
+    # split, so it starts cold as an isolated call does.
+    stages = None
+    if not args.paged and Q == 1 and not quant:
+        flush = L2Flush(dev)
+        split_t, comb_t = [], []
+        for i in range(max(5, min(args.steps, 20))):
+            x = xs[i % n_copies]
+            flush(i)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e[0].record(stream)
+            fd.fd_split(x.q, x.k, x.v, x.seqlens, x.scale, out, lse, ws, S, stream)
+            e[1].record(stream)
+            torch.cuda.synchronize(dev)
+            e[2].record(stream)
+            fd.fd_combine(w.B, w.Hq, w.Hkv, w.D, w.Lmax, x.seqlens, out, lse, ws, S, stream)
+            e[3].record(stream)
+            torch.cuda.synchronize(dev)
+            split_t.append(e[0].elapsed_time(e[1]) * 1e3)
+            comb_t.append(e[2].elapsed_time(e[3]) * 1e3)
+        del flush
+        stages = {"split_us": float(np.median(split_t)), "combine_us": float(np.median(comb_t)),
+                  "how": "medians; each stage alone between its own events, a host sync between them, "
+                         "L2 flushed before the split"}
 
     # ---- end to end: host buffers in, host buffers out ---------------------
     e2e = None
@@ -483,6 +626,7 @@ def run_fd(args, w, rank, world):
         e2e = {"value": whole_job_gbs(world, x.kv_bytes(), e_steps, ems), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
                "us_per_call": ems * 1e3 / e_steps}
+        del dq, dk, dv, dsq
 
     status = fd.fd_device_status(stream)
     if status != 0:
@@ -496,22 +640,24 @@ def run_fd(args, w, rank, world):
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_max / args.steps, "us_per_call": us_per_call,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": args.kv, "data": "synthetic",
-        "config": dict(config_dict(w, S, l2_note), **({"kv_cache": args.kv} if quant else {}),
+        "config": dict(config_dict(w, S, wk.l2_note), **({"kv_cache": args.kv} if quant else {}),
                        **({"paged": {"page_size": args.paged, "layout": args.layout}} if args.paged else {}),
                        **({"q_len": Q} if Q > 1 else {})),
         "pct_of_nominal_hbm": 100.0 * gbs / world / NOMINAL_HBM_GBS,
         "pct_of_measured_copy": 100.0 * gbs / world / peak,
-        "read_probe": {"gbs": probe, "bytes": 2 << 30, "kernel": "fd_read_probe (bulk copies, 1 block per SM, 128 KiB in flight)"},
+        "read_probe": {"gbs": probe, "bytes": 2 << 30,
+                       "kernel": "fd_read_probe (bulk copies, 1 block per SM, 128 KiB in flight)"},
         "pct_of_read_probe": 100.0 * gbs / world / probe if probe else None,
         "per_call": per_call,
         "call_bytes_gbs": world * counts["total"] * args.steps / (ms_max * 1e-3) / 1e9,
-        "roofline": {"kernel": "fd_split_kernel (fused combine)" + (f", {args.kv} cache" if quant else ""), "bound": "hbm", "achieved": kernel_gbs,
+        "roofline": {"kernel": "fd_split_kernel (fused combine)" + (f", {args.kv} cache" if quant else ""),
+                     "bound": "hbm", "achieved": kernel_gbs,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": kernel_gbs / peak,
                      "traffic": None if args.paged or Q > 1 else measured_traffic(w.name + (f":{args.kv}" if quant else "")),
                      "bytes_per_launch": counts["total"],
                      "us_per_launch": us_per_call,
                      "frac_of_nominal_8tbs": kernel_gbs / NOMINAL_HBM_GBS},
-        "stages_alone": {"split_us": split_us, "combine_us": combine_us},
+        "stages_alone": stages,
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),
         "e2e": e2e,
@@ -539,8 +685,38 @@ def run_fd(args, w, rank, world):
                                 "sample": desc, "seconds": s,
                                 "single_thread": {"value": b1 / s1 / 1e9, "unit": "GB/s", "cores": 1,
                                                   "sample": desc1, "seconds": s1}}
+    if world == 1 and not args.no_per_config and not args.paged and Q == 1 and not quant and w.name == HEADLINE:
+        del wk, xs, calls, out, lse, ws
+        torch.cuda.empty_cache()
+        per = {}
+        for name, kv in PER_CONFIG:
+            key, entry = config_entry(args, WORKLOADS[name], kv, dev, stream, peak)
+            per[key] = entry
+            line["gpu_launches"] += args.steps
+        line["per_config"] = per
+        if fd.fd_device_status(stream) != 0:
+            raise RuntimeError("device status after the per-config runs")
+    if world == 1 and rank == 0:
+        line["host_cost"] = host_cost(w)
     print(json.dumps(line), flush=True)
     return 0
+
+
+def host_cost(w, calls=200):
+    """Host microseconds per call of fd_decode / fd_decode_splits / fd_plan
+    through the C ABI, timed by the C++ program fd_host_bench (no Python on
+    the path), on this workload's shape; an empty kernel's launch beside them."""
+    from decode_attention_07_b200 import build as lib_build
+    exe = lib_build.HOST_BENCH
+    if not os.path.exists(exe):
+        return {"unavailable": "fd_host_bench is not built (python -c 'import __graft_entry__ as g; g.build()')"}
+    r = subprocess.run([exe, str(w.B), str(w.Hq), str(w.Hkv), str(w.D), str(w.Lmax), str(calls)],
+                       capture_output=True, text=True, timeout=300)
+    if r.returncode != 0:
+        return {"unavailable": f"fd_host_bench exited {r.returncode}: {r.stderr.strip()[-200:]}"}
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    d["how"] = "C++ through the C ABI, steady clock around CALLS back-to-back enqueues, tensor maps cached"
+    return d
 
 
 def run_cp(args, w, rank, world):
@@ -635,6 +811,57 @@ def run_cp(args, w, rank, world):
     return 0
 
 
+def launch_ranks(n: int, argv) -> int:
+    """`--gpus N` outside torchrun: start N copies of this script, one per
+    GPU, with RANK / LOCAL_RANK / WORLD_SIZE / MASTER_ADDR / MASTER_PORT set
+    as torchrun would, and wait for all of them. Rank 0's stdout is ours;
+    the others' is discarded (they print nothing). If one rank fails, the
+    others are ended (by their own PIDs) and the first failure is returned."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    procs = []
+    for r in range(n):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE=str(n), LOCAL_WORLD_SIZE=str(n),
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        procs.append(subprocess.Popen([sys.executable, os.path.abspath(__file__), *argv], env=env,
+                                      stdout=None if r == 0 else subprocess.DEVNULL))
+    rc = 0
+    pending = list(procs)
+    while pending:
+        for pr in list(pending):
+            code = pr.poll()
+            if code is None:
+                continue
+            pending.remove(pr)
+            if code != 0 and rc == 0:
+                rc = code
+                for other in pending:
+                    other.terminate()
+        time.sleep(0.05)
+    return rc
+
+
+def check_launch(world: int, rank: int) -> int:
+    """`--check-launch`: the multi-rank plumbing alone, without a GPU
+    workload. Every rank joins the process group (NCCL with GPUs, gloo
+    without), the ranks count themselves with an all-reduce and gather their
+    PIDs; rank 0 prints one JSON line."""
+    t = torch.ones(1, dtype=torch.float64)
+    pids = [os.getpid()]
+    if world > 1:
+        if torch.cuda.is_available():
+            t = t.cuda()
+        torch.distributed.all_reduce(t)
+        pids = [None] * world
+        torch.distributed.all_gather_object(pids, os.getpid())
+    if rank == 0:
+        print(json.dumps({"check_launch": True, "n_gpus": world, "ranks_joined": int(t.item()), "pids": pids,
+                          "backend": torch.distributed.get_backend() if world > 1 else None}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -657,7 +884,18 @@ def main():
                     help="new tokens per sequence, each a query seeing the cache up to itself (fd_decode_multi)")
     ap.add_argument("--no-clock-window", action="store_true",
                     help="do not extend clock sampling past the timed region (for profiler runs)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="report the headline workload only (no per_config object)")
+    ap.add_argument("--check-launch", action="store_true",
+                    help="only start the ranks, join the process group and report them (no workload)")
     args = ap.parse_args()
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" in os.environ:
+        if int(os.environ["WORLD_SIZE"]) != args.gpus:
+            ap.error(f"WORLD_SIZE={os.environ['WORLD_SIZE']} but --gpus {args.gpus}: launch one rank per GPU")
+    elif args.gpus > 1:
+        return launch_ranks(args.gpus, sys.argv[1:])
     if args.paged and args.q_len != 1:
         ap.error("--paged takes one query per sequence")
     if args.cp and (args.paged or args.kv != "bf16" or args.q_len != 1):
@@ -665,11 +903,18 @@ def main():
     w = WORKLOADS[args.config]
     world = int(os.environ.get("WORLD_SIZE", 1))
     rank = int(os.environ.get("RANK", 0))
-    if world > 1 and args.impl == "fd":
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+    if world > 1 and (args.impl == "fd" or args.check_launch):
         import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        elif args.check_launch:   # CPU-only check of the launcher
+            torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+        else:
+            raise RuntimeError("the GPU arm needs CUDA devices")
     try:
+        if args.check_launch:
+            return check_launch(world, rank)
         if args.impl == "reference":
             return run_reference(args, w, rank, world)
         if args.cp:

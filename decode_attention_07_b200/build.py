@@ -9,6 +9,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libfdecode.so")
 DEBUG_LIBRARY = os.path.join(PKG, "libfdecode_debug.so")   # -DFD_DEBUG: device-side bounds checks
+HOST_BENCH = os.path.join(PKG, "fd_host_bench")   # host time per call through the C ABI (bench.py runs it)
 SOURCES = [os.path.join(CSRC, "fd_api.cu"), os.path.join(CSRC, "fd_probe.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + \
     [os.path.join(INCLUDE, "fd.h")]
@@ -33,6 +34,19 @@ def up_to_date(out: str) -> bool:
         return False
     t = os.path.getmtime(out)
     return all(os.path.getmtime(d) <= t for d in DEPS)
+
+
+def build_host_bench(force: bool = False) -> str:
+    """The C++ program that times fd_decode's host side; linked against the
+    in-tree libfdecode.so (found next to it at run time)."""
+    src = os.path.join(CSRC, "fd_host_bench.cu")
+    if not force and os.path.exists(HOST_BENCH) and os.path.getmtime(HOST_BENCH) >= max(
+            os.path.getmtime(src), os.path.getmtime(LIBRARY)):
+        return HOST_BENCH
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O2", "-std=c++17", "-I", INCLUDE, "-o",
+           HOST_BENCH, src, "-L", PKG, "-lfdecode", "-Xlinker", "-rpath,$ORIGIN"]
+    subprocess.run(cmd, check=True)
+    return HOST_BENCH
 
 
 def build(force: bool = False, verbose_ptxas: bool = False, out: str = None, debug: bool = False) -> str:

@@ -128,23 +128,83 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+// Encoded tensor maps, cached per device. A map holds only the base address,
+// the shape, the strides and the box, so a map encoded once for a buffer
+// stays valid for every later call on that buffer (and for a new buffer
+// that happens to reuse the address with the same shape). A decode loop that
+// reuses its caches thus encodes each map once instead of once per call.
+// Entries are replaced round-robin when the cache is full.
+struct MapKey {
+    int dtype, rank, swizzle;
+    const void *base;
+    cuuint64_t dims[5], strides[4];
+    cuuint32_t box[5];
+};
+struct MapEntry {
+    MapKey key;
+    CUtensorMap map;
+};
+constexpr int kMapCacheEntries = 32;
+struct MapCache {
+    MapEntry e[kMapCacheEntries];
+    int size = 0, next = 0;
+};
+MapCache g_map_cache[kMaxDevices];
+std::mutex g_map_mutex;
+
+// cuTensorMapEncodeTiled with element strides 1, no interleave, 256-byte L2
+// promotion and no fill, through the cache.
+int encode_tiled(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base, const cuuint64_t *dims,
+                 const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapSwizzle swz) {
+    int dev;
+    if (current_device(&dev) != FD_OK) return FD_ERR_DEVICE;
+    MapKey k;
+    std::memset(&k, 0, sizeof k);   // padding included: keys are compared bytewise
+    k.dtype = static_cast<int>(dtype);
+    k.rank = rank;
+    k.swizzle = static_cast<int>(swz);
+    k.base = base;
+    for (int i = 0; i < rank; ++i) {
+        k.dims[i] = dims[i];
+        k.box[i] = box[i];
+        if (i + 1 < rank) k.strides[i] = strides[i];
+    }
+    {
+        std::lock_guard<std::mutex> lock(g_map_mutex);
+        MapCache &c = g_map_cache[dev];
+        for (int i = 0; i < c.size; ++i)
+            if (std::memcmp(&c.e[i].key, &k, sizeof k) == 0) {
+                *map = c.e[i].map;
+                return FD_OK;
+            }
+    }
+    auto fn = encode_fn();
+    if (!fn) return FD_ERR_LAUNCH;
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    const CUresult r = fn(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return FD_ERR_LAUNCH;
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    MapCache &c = g_map_cache[dev];
+    const int slot = c.size < kMapCacheEntries ? c.size++ : (c.next++ % kMapCacheEntries);
+    c.e[slot].key = k;
+    c.e[slot].map = *map;
+    return FD_OK;
+}
+
 // K or V cache [B*Hkv rows][Lmax][D] as a 3-D tensor (D innermost). bf16:
 // box = 64 head-dim elements (128 bytes, 128-byte swizzle) x 64 tokens x 1
 // row. 8-bit codes (one_byte): box = all D codes of a token (128 bytes with
 // the 128-byte swizzle for D = 128, 64 bytes with the 64-byte one for D = 64).
 int encode_cache_map(CUtensorMap *map, const void *base, int D, int Lmax, long long rows, bool one_byte = false) {
-    auto fn = encode_fn();
-    if (!fn) return FD_ERR_LAUNCH;
     const cuuint64_t e = one_byte ? 1 : 2;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Lmax), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * e, static_cast<cuuint64_t>(Lmax) * D * e};
     cuuint32_t box[3] = {one_byte ? static_cast<cuuint32_t>(D) : 64u, static_cast<cuuint32_t>(fd::kTileTokens), 1};
-    cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapSwizzle swz = one_byte && D == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-    CUresult r = fn(map, one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? FD_OK : FD_ERR_LAUNCH;
+    return encode_tiled(map, one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims,
+                        strides, box, swz);
 }
 
 // Paged K or V pool as a 3-D tensor, head-dim innermost. Head-major pages
@@ -158,8 +218,6 @@ int encode_cache_map(CUtensorMap *map, const void *base, int D, int Lmax, long l
 // codes of a token (64-byte swizzle for D = 64).
 int encode_paged_map(CUtensorMap *map, const void *base, int D, int page_size, int Hkv, long long num_pages,
                      bool nhd, bool one_byte = false) {
-    auto fn = encode_fn();
-    if (!fn) return FD_ERR_LAUNCH;
     const cuuint64_t e = one_byte ? 1 : 2;   // 8-bit codes or bf16
     const cuuint32_t rows = static_cast<cuuint32_t>(page_size < fd::kTileTokens ? page_size : fd::kTileTokens);
     const cuuint64_t row = static_cast<cuuint64_t>(D) * e;   // bytes of one token of one head
@@ -182,12 +240,9 @@ int encode_paged_map(CUtensorMap *map, const void *base, int D, int page_size, i
         box[1] = rows;
         box[2] = 1;
     }
-    cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapSwizzle swz = one_byte && D == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-    CUresult r = fn(map, one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? FD_OK : FD_ERR_LAUNCH;
+    return encode_tiled(map, one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims,
+                        strides, box, swz);
 }
 
 // Small pages at D = 128 (page_size < 64): each 256-byte token row viewed as
@@ -196,8 +251,6 @@ int encode_paged_map(CUtensorMap *map, const void *base, int D, int page_size, i
 // {64, 2, page_size, Hkv, num_pages}, box {64, 2, page_size, 1, 1}; token-major:
 // {64, 2, Hkv, page_size, num_pages}, box {64, 2, 1, page_size, 1}.
 int encode_paged_map_rows(CUtensorMap *map, const void *base, int page_size, int Hkv, long long num_pages, bool nhd) {
-    auto fn = encode_fn();
-    if (!fn) return FD_ERR_LAUNCH;
     const cuuint64_t row = 256;   // bytes of one token of one head (D = 128, bf16)
     cuuint64_t dims[5], strides[4];
     cuuint32_t box[5];
@@ -224,11 +277,7 @@ int encode_paged_map_rows(CUtensorMap *map, const void *base, int page_size, int
         box[3] = 1;
     }
     strides[3] = static_cast<cuuint64_t>(page_size) * Hkv * row;
-    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? FD_OK : FD_ERR_LAUNCH;
+    return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // Host-side failure injection for tests: with FD_TEST_FAIL_LAUNCH set in the
@@ -442,6 +491,8 @@ int run_split(const Problem &pr, bool fused, int q_len = 1) {
     p.kv_nhd = 0;
     p.num_pages = 0;
     p.k_scale = p.v_scale = nullptr;
+    p.k_base = pr.k;
+    p.v_base = pr.v;
     p.debug_withhold = debug_withhold();
     p.debug_spoil_guess = debug_spoil_guess();
     // with max_len == 0 every block finds zero tiles and only writes empty rows;
@@ -500,6 +551,7 @@ int run_split_paged(const Problem &pr, const PagedLayout &pl, int q_len = 1, int
     p.num_pages = pl.num_pages;
     p.k_scale = k_scale;
     p.v_scale = v_scale;
+    p.k_base = p.v_base = nullptr;   // paged pools: no contiguous span to prefetch
     p.debug_withhold = debug_withhold();
     p.debug_spoil_guess = debug_spoil_guess();
     if (quant)
@@ -550,6 +602,8 @@ int run_split_quant(const Problem &pr, int q_len, int kv_type, const float *k_sc
     p.num_pages = 0;
     p.k_scale = k_scale;
     p.v_scale = v_scale;
+    p.k_base = pr.k;
+    p.v_base = pr.v;
     p.debug_withhold = debug_withhold();
     p.debug_spoil_guess = debug_spoil_guess();
     return kv_type == FD_KV_E4M3 ? launch_split_quant<true>(pr.D, p.cols, tk, tv, p, pr.stream)
@@ -608,20 +662,24 @@ Problem make_problem(int B, int Hq, int Hkv, int D, int max_len, const uint16_t 
 static __device__ __align__(256) unsigned char g_fd_static_scratch[FD_STATIC_SCRATCH_BYTES];
 
 void *g_static_scratch_ptr[kMaxDevices];
-cudaError_t g_static_scratch_err[kMaxDevices];
-std::once_flag g_static_scratch_once[kMaxDevices];
+std::mutex g_static_scratch_mutex;
 
-// Device address of this device's fixed scratch buffer (looked up on first use).
+// Device address of this device's fixed scratch buffer, looked up on first
+// use. Only a successful lookup is kept: a lookup that fails (for instance
+// under stream capture, where loading the module may be refused) returns
+// FD_ERR_LAUNCH and is tried again by the next call.
 int static_scratch(void **ptr) {
     int dev;
     int rc = current_device(&dev);
     if (rc != FD_OK) return rc;
-    std::call_once(g_static_scratch_once[dev], [dev] {
-        g_static_scratch_err[dev] = cudaGetSymbolAddress(&g_static_scratch_ptr[dev], g_fd_static_scratch);
-    });
-    if (g_static_scratch_err[dev] != cudaSuccess || g_static_scratch_ptr[dev] == nullptr) {
-        cudaGetLastError();
-        return FD_ERR_LAUNCH;
+    std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+    if (g_static_scratch_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_fd_static_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return FD_ERR_LAUNCH;
+        }
+        g_static_scratch_ptr[dev] = p;
     }
     *ptr = g_static_scratch_ptr[dev];
     return FD_OK;

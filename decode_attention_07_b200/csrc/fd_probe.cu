@@ -80,9 +80,10 @@ __global__ void __launch_bounds__(32, 1) fd_read_probe_kernel(const uint8_t *buf
     for (size_t k = 0; k < mine; ++k) {
         const int s = static_cast<int>(k % kProbeStages);
         if (!wait_phase(&bar[s], static_cast<uint32_t>((k / kProbeStages) & 1))) {
-            // give up, but leave only once the copies already issued have landed
-            // (each of those waits bounded too)
+            // give up, but leave only once the copies already issued have landed,
+            // chunk k's own included (each of those waits bounded too)
             atomicExch(timed_out, 1);
+            wait_phase(&bar[s], static_cast<uint32_t>((k / kProbeStages) & 1));
             for (size_t j = k + 1; j < mine && j < k + kProbeStages; ++j)
                 wait_phase(&bar[j % kProbeStages], static_cast<uint32_t>((j / kProbeStages) & 1));
             return;

@@ -121,10 +121,44 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int x
                  : "memory");
 }
 
+// Ask for `bytes` contiguous bytes at `src` to be brought into L2 (1-D bulk
+// prefetch: one instruction for a whole contiguous span, where a tiled
+// prefetch takes one per box). 16-byte aligned address, size a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
+}
+
+// ------------------------------------------------ packed / mixed fp32 math --
+// c + a.lo * b.lo, then + a.hi * b.hi: two fused multiply-adds of bf16 pairs
+// into an fp32 sum (each product exact, each step rounded once) -- the same
+// result as converting both operands to fp32 and using fmaf twice, without
+// the conversions.
+__device__ __forceinline__ float fma2_bf16(uint32_t a, uint32_t b, float c) {
+    float d;
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t.reg .f32 t;\n\t"
+        "mov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 t, al, bl, %3;\n\tfma.rn.f32.bf16 %0, ah, bh, t;\n\t}"
+        : "=f"(d)
+        : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+
+// (c0, c1) += a * (lo(w), hi(w)) for a bf16 pair w: two fp32 fused
+// multiply-adds in one packed instruction, each rounded as fmaf would.
+__device__ __forceinline__ void fma_f32x2_bf16(float &c0, float &c1, float a, uint32_t w) {
+    asm("{\n\t.reg .b64 x, y, c;\n\t.reg .b32 lo, hi;\n\t"
+        "shl.b32 lo, %3, 16;\n\tand.b32 hi, %3, 0xffff0000;\n\t"
+        "mov.b64 x, {%2, %2};\n\tmov.b64 y, {lo, hi};\n\tmov.b64 c, {%0, %1};\n\t"
+        "fma.rn.f32x2 c, x, y, c;\n\tmov.b64 {%0, %1}, c;\n\t}"
+        : "+f"(c0), "+f"(c1)
+        : "f"(a), "r"(w));
 }
 
 // --------------------------------------------------------- tensor-core ops --

@@ -106,6 +106,9 @@ struct SplitParams {
     // 8-bit caches only: value of a cached element = scale[kv head] * decode(code)
     const float *k_scale;     // [Hkv]
     const float *v_scale;     // [Hkv]
+    // contiguous caches only: the K and V arrays, for the bulk L2 prefetch before the dependency wait
+    const void *k_base;
+    const void *v_base;
     int debug_withhold;       // debug builds: block 0 issues no copy for this tile (a wait then runs out); -1: off
     int debug_spoil_guess;    // debug builds: make every block's pre-wait guess of its start wrong
 };
@@ -217,6 +220,20 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
     }
 }
 
+// Wait for warp 0 to publish the block's real start (phase 0 of `bar`). If
+// the bounded wait gives up, the device error word is set; the block then
+// goes on with whatever the start record holds and the call is reported as
+// failed by fd_device_status.
+__device__ __forceinline__ void wait_start(uint64_t *bar) {
+    if (mbar_try_wait(bar, 0)) return;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, 0))
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            atomicExch(&g_fd_error_word, -10 /* FD_ERR_TIMEOUT */);
+            return;
+        }
+}
+
 // After a wait gave up: wait once more, bounded and regardless of the abort
 // flag, for a phase whose copies were issued, so that no copy still lands in
 // this block's shared memory after it exits.
@@ -237,6 +254,19 @@ __device__ __forceinline__ void drain_copies(uint64_t *full, uint32_t issued, ui
         drain_phase(&full[s], (n - 1) & 1u);
     }
     if (window_pending) drain_phase(pbar, win_phase);
+}
+
+// Contiguous caches: ask L2 for tiles [t0, t1) of row z of K and of V, as
+// one bulk prefetch each (clipped to the row's Lmax tokens; nothing past the
+// row is touched).
+template <int kRowBytes>
+__device__ __forceinline__ void prefetch_row_span(const SplitParams &p, int z, int t0, int t1) {
+    const int tok0 = t0 * kTileTokens, tok1 = min(t1 * kTileTokens, p.Lmax);
+    if (tok1 <= tok0) return;
+    const size_t off = (static_cast<size_t>(z) * p.Lmax + tok0) * kRowBytes;
+    const uint32_t bytes = static_cast<uint32_t>(tok1 - tok0) * kRowBytes;
+    bulk_prefetch_l2(static_cast<const uint8_t *>(p.k_base) + off, bytes);
+    bulk_prefetch_l2(static_cast<const uint8_t *>(p.v_base) + off, bytes);
 }
 
 __device__ __forceinline__ int row_tiles(const int32_t *seqlens, int b, int Lmax) {
@@ -620,17 +650,22 @@ struct GroupConsumer {
 };
 
 // ------------------------------------------------ one-head (MHA) consumer --
-template <int D, bool kInter = false>
+// kTok tokens of each tile per warp: 16 (four warps per group, two groups) or
+// 32 (two warps per group, four groups), the 32 as two 16-token halves whose
+// dependency chains interleave and which share one rescale of the state.
+template <int D, bool kInter = false, int kTok = 16>
 struct HeadConsumer {
     static constexpr int G = 1;
     static constexpr int kElemBytes = 2;
-    static constexpr int kWarpTokens = 16;
+    static constexpr int kWarpTokens = kTok;
     static constexpr bool kInterleaved = kInter;
     static constexpr int LPT = D / 8;          // lanes per token (16 bytes = 8 bf16 each)
     static constexpr int TPI = 32 / LPT;       // tokens per warp-wide load
-    static constexpr int ITER = kWarpTokens / TPI;
+    static constexpr int ITER = 16 / TPI;      // warp-wide loads per 16-token half
+    static constexpr int NSUB = kTok / 16;     // 16-token halves
+    static_assert(kTok == 16 || kTok == 32, "16 or 32 tokens per warp");
 
-    float qv[8];                               // q[d0 .. d0+7] of this lane's 16-byte chunk
+    uint4 qw;                                  // q[d0 .. d0+7] of this lane's 16-byte chunk (bf16 pairs)
     float m, l;                                // running max (base 2, warp-uniform) / lane partial sum
     float acc[8];                              // sum of p * v over this lane's tokens, chunk d0..d0+7
 
@@ -648,11 +683,7 @@ struct HeadConsumer {
     __device__ __forceinline__ void load_q(const uint8_t *qs, int) {
         const int lane = threadIdx.x & 31;
         const int d0 = 8 * (lane % LPT);
-        const uint4 w = *reinterpret_cast<const uint4 *>(qs + d0 * 2);
-        qv[0] = bf16lo_to_f32(w.x); qv[1] = bf16hi_to_f32(w.x);
-        qv[2] = bf16lo_to_f32(w.y); qv[3] = bf16hi_to_f32(w.y);
-        qv[4] = bf16lo_to_f32(w.z); qv[5] = bf16hi_to_f32(w.z);
-        qv[6] = bf16lo_to_f32(w.w); qv[7] = bf16hi_to_f32(w.w);
+        qw = *reinterpret_cast<const uint4 *>(qs + d0 * 2);
     }
 
     static __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -671,70 +702,104 @@ struct HeadConsumer {
         const int d0 = 8 * chunk;
         const int dhalf = d0 >> 6, j = (d0 & 63) >> 3;   // 64-element half of the head dims, chunk in it
 
-        // partial dots over this lane's 8 dims for tokens TPI*it + half
-        float pd[ITER];
+        // partial dots over this lane's 8 dims for tokens 16*s + TPI*it + half
+        float pd[NSUB][ITER];
 #pragma unroll
-        for (int it = 0; it < ITER; ++it) {
-            const int r = kWarpTokens * slice + TPI * it + half;
-            const uint4 w = lds128(k_smem + tile_offset<kInter>(r, dhalf, j));
-            float a = qv[0] * bf16lo_to_f32(w.x);
-            a = fmaf(qv[1], bf16hi_to_f32(w.x), a);
-            a = fmaf(qv[2], bf16lo_to_f32(w.y), a);
-            a = fmaf(qv[3], bf16hi_to_f32(w.y), a);
-            a = fmaf(qv[4], bf16lo_to_f32(w.z), a);
-            a = fmaf(qv[5], bf16hi_to_f32(w.z), a);
-            a = fmaf(qv[6], bf16lo_to_f32(w.w), a);
-            a = fmaf(qv[7], bf16hi_to_f32(w.w), a);
-            pd[it] = a;
-        }
+        for (int s = 0; s < NSUB; ++s)
+#pragma unroll
+            for (int it = 0; it < ITER; ++it) {
+                const int r = kWarpTokens * slice + 16 * s + TPI * it + half;
+                const uint4 w = lds128(k_smem + tile_offset<kInter>(r, dhalf, j));
+                // q . k over the 8 dims in order, products exact, fp32 sums (-0 start: the
+                // first step is the exact product, as a multiply would give)
+                float a = fma2_bf16(qw.x, w.x, -0.f);
+                a = fma2_bf16(qw.y, w.y, a);
+                a = fma2_bf16(qw.z, w.z, a);
+                a = fma2_bf16(qw.w, w.w, a);
+                pd[s][it] = a;
+            }
         // reduce across the LPT lanes of each token while spreading tokens
         // over lanes: after the halving steps lane keeps token index
-        // (lane % LPT) / 2; the last step leaves the full dot in both lanes
-        // of each pair.
+        // (lane % LPT) / 2 of each half; the last step leaves the full dot in
+        // both lanes of each pair.
 #pragma unroll
         for (int n = ITER; n > 1; n >>= 1) {
             const bool up = (lane & n) != 0;
 #pragma unroll
-            for (int k = 0; k < n / 2; ++k) {
-                const float send = up ? pd[k] : pd[k + n / 2];
-                const float keep = up ? pd[k + n / 2] : pd[k];
-                pd[k] = keep + __shfl_xor_sync(0xffffffffu, send, n);
-            }
+            for (int k = 0; k < n / 2; ++k)
+#pragma unroll
+                for (int s = 0; s < NSUB; ++s) {
+                    const float send = up ? pd[s][k] : pd[s][k + n / 2];
+                    const float keep = up ? pd[s][k + n / 2] : pd[s][k];
+                    pd[s][k] = keep + __shfl_xor_sync(0xffffffffu, send, n);
+                }
         }
-        float x = pd[0] + __shfl_xor_sync(0xffffffffu, pd[0], 1);
         const int my_it = chunk >> 1;
-        x *= scale_log2e;
-        if (TPI * my_it + half >= valid) x = -INFINITY;
-
-        float mx = x;   // both lanes of a pair hold the same value: skip the xor-1 step
+        float x[NSUB];
+        float mx = -INFINITY;   // both lanes of a pair hold the same value: skip the xor-1 step below
+#pragma unroll
+        for (int s = 0; s < NSUB; ++s) {
+            x[s] = (pd[s][0] + __shfl_xor_sync(0xffffffffu, pd[s][0], 1)) * scale_log2e;
+            if (16 * s + TPI * my_it + half >= valid) x[s] = -INFINITY;
+            mx = fmaxf(mx, x[s]);
+        }
 #pragma unroll
         for (int sh = 2; sh < 32; sh <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, sh));
         const float mn = fmaxf(m, mx);
         const float mu = mn == -INFINITY ? 0.f : mn;
         const float alpha = ex2(m - mu);
-        const float pv = ex2(x - mu);
-        l = fmaf(l, alpha, (lane & 1) ? 0.f : pv);
+        float pv[NSUB], psum = 0.f;
+#pragma unroll
+        for (int s = 0; s < NSUB; ++s) {
+            pv[s] = ex2(x[s] - mu);
+            psum += pv[s];
+        }
+        l = fmaf(l, alpha, (lane & 1) ? 0.f : psum);
         m = mn;
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc[k] *= alpha;
 
+        if (16 * NSUB <= valid) {
+            // every token of the warp's slice is inside the row: no per-token
+            // test, so all weights and value rows are fetched before the first
+            // multiply-add (a test per token keeps each load behind the last)
+            float pt[NSUB][ITER];
+            uint4 vw[NSUB][ITER];
 #pragma unroll
-        for (int it = 0; it < ITER; ++it) {
-            const float pt = __shfl_sync(0xffffffffu, pv, half * LPT + 2 * it);
-            const int t = TPI * it + half;
-            if (t < valid) {
-                const int r = kWarpTokens * slice + t;
-                const uint4 w = lds128(v_smem + tile_offset<kInter>(r, dhalf, j));
-                acc[0] = fmaf(pt, bf16lo_to_f32(w.x), acc[0]);
-                acc[1] = fmaf(pt, bf16hi_to_f32(w.x), acc[1]);
-                acc[2] = fmaf(pt, bf16lo_to_f32(w.y), acc[2]);
-                acc[3] = fmaf(pt, bf16hi_to_f32(w.y), acc[3]);
-                acc[4] = fmaf(pt, bf16lo_to_f32(w.z), acc[4]);
-                acc[5] = fmaf(pt, bf16hi_to_f32(w.z), acc[5]);
-                acc[6] = fmaf(pt, bf16lo_to_f32(w.w), acc[6]);
-                acc[7] = fmaf(pt, bf16hi_to_f32(w.w), acc[7]);
-            }
+            for (int s = 0; s < NSUB; ++s)
+#pragma unroll
+                for (int it = 0; it < ITER; ++it) {
+                    pt[s][it] = __shfl_sync(0xffffffffu, pv[s], half * LPT + 2 * it);
+                    vw[s][it] = lds128(v_smem + tile_offset<kInter>(kWarpTokens * slice + 16 * s + TPI * it + half,
+                                                                     dhalf, j));
+                }
+#pragma unroll
+            for (int s = 0; s < NSUB; ++s)
+#pragma unroll
+                for (int it = 0; it < ITER; ++it) {
+                    fma_f32x2_bf16(acc[0], acc[1], pt[s][it], vw[s][it].x);
+                    fma_f32x2_bf16(acc[2], acc[3], pt[s][it], vw[s][it].y);
+                    fma_f32x2_bf16(acc[4], acc[5], pt[s][it], vw[s][it].z);
+                    fma_f32x2_bf16(acc[6], acc[7], pt[s][it], vw[s][it].w);
+                }
+            return;
         }
+        // the row ends inside the slice: rows past it may hold anything (NaN) and are skipped
+#pragma unroll
+        for (int s = 0; s < NSUB; ++s)
+#pragma unroll
+            for (int it = 0; it < ITER; ++it) {
+                const float pt = __shfl_sync(0xffffffffu, pv[s], half * LPT + 2 * it);
+                const int t = 16 * s + TPI * it + half;
+                if (t < valid) {
+                    const int r = kWarpTokens * slice + t;
+                    const uint4 w = lds128(v_smem + tile_offset<kInter>(r, dhalf, j));
+                    fma_f32x2_bf16(acc[0], acc[1], pt, w.x);
+                    fma_f32x2_bf16(acc[2], acc[3], pt, w.y);
+                    fma_f32x2_bf16(acc[4], acc[5], pt, w.z);
+                    fma_f32x2_bf16(acc[6], acc[7], pt, w.w);
+                }
+            }
     }
 
     __device__ __forceinline__ void to_smem(float *wb) {
@@ -783,7 +848,8 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
     uint64_t *mfull = empty + kStages;                                     // merge buffer filled (8 warps)
     uint64_t *mempty = mfull + kBufs;                                      // merge buffer drained (finishers)
     uint64_t *pbar = mempty + kBufs;                                       // block-table windows landed (K, V)
-    StartInfo *info = reinterpret_cast<StartInfo *>(pbar + 2);
+    uint64_t *startbar = pbar + 2;                                         // warp 0 has worked out the real start
+    StartInfo *info = reinterpret_cast<StartInfo *>(startbar + 1);
     StartInfo *guess = info + 1;                                           // the start as guessed before the wait
     float *weights = reinterpret_cast<float *>(guess + 1);                 // [G][8] merge weights, [G] lse
     constexpr int kWeightFloats = (G * kConsumerWarps + G + 3) / 4 * 4;
@@ -793,7 +859,7 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
     static_assert(kStageFloats >= (G == 1 ? kTwoLevelSegs * (D + 1) + 4 : kStageBudgetFloats),
                   "a one-level row must fit the shared memory free at the end of the run");
     EndPlan *plan = reinterpret_cast<EndPlan *>(weights + kWeightFloats);  // what the end of the run merges
-    static_assert((2 * kStages + 2 * kBufs + 2) * 8 + 2 * sizeof(StartInfo) + kWeightFloats * 4 + sizeof(EndPlan) <=
+    static_assert((2 * kStages + 2 * kBufs + 3) * 8 + 2 * sizeof(StartInfo) + kWeightFloats * 4 + sizeof(EndPlan) <=
                       Cfg::kCtrlBytes,
                   "control block over its bytes");
     int32_t *page_win = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(merge) +
@@ -816,6 +882,7 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
         }
         mbar_init(pbar, 1);
         mbar_init(pbar + 1, 1);
+        mbar_init(startbar, 1);
         fence_mbar_init();
     }
     if (warp == kProducerWarp && lane == 0) {   // kernel parameters, not inputs: safe before the wait
@@ -825,22 +892,21 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
     // While the previous grid drains (HBM mostly idle), guess this block's
     // first tiles from seqlens as read now and pull them into L2. L2 is the
     // point of coherence, so a stale guess only wastes bandwidth; everything
-    // below is recomputed from the real inputs after the wait.
+    // below is recomputed from the real inputs after the wait. The guessed
+    // tiles of a contiguous cache are one span of K and one of V (inside the
+    // first row), asked for with two bulk prefetches: a tiled prefetch per
+    // box costs its issuing thread about as much as a copy, and a block placed
+    // late on its SM would otherwise reach the wait late.
     if (!kPaged && warp == 0) {
         find_start<true>(p, guess);
 #ifdef FD_DEBUG
         if (lane == 0 && p.debug_spoil_guess) guess->tile = guess->tile > 0 ? guess->tile - 1 : guess->tile + 1;
 #endif
         __syncwarp();
-        if (lane < 2 * kPrefetchTiles && guess->count > 0) {
-            const int t = lane >> 1;
-            const int tile = guess->tile + t;
-            if (t < guess->count && tile < guess->n) {
-                const CUtensorMap *map = (lane & 1) ? &tm_v : &tm_k;
-                const int z = guess->b * p.Hkv + guess->h;
-                for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-                    tma_prefetch_l2_3d(map, Cfg::kBoxCols * bx, tile * kTileTokens, z);
-            }
+        if (lane == 0 && guess->count > 0) {
+            const int nt = static_cast<int>(min(static_cast<long long>(kPrefetchTiles),
+                                                min(static_cast<long long>(guess->n - guess->tile), guess->count)));
+            prefetch_row_span<Cfg::kRowBytes>(p, guess->b * p.Hkv + guess->h, guess->tile, guess->tile + nt);
         }
         __syncwarp();
     }
@@ -848,21 +914,27 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
     // Launched as a programmatic dependent of the previous kernel on the
     // stream: everything above overlaps its tail; inputs are read only after it.
     grid_dependency_wait();
-    // The producer starts on the guessed first tiles (up to one ring's worth,
+    // The first tiles are issued from the guess (up to one ring's worth,
     // inside the first row) while warp 0 works out the real start from the
-    // inputs as they are now. When the two differ (the lengths changed under
-    // the guess), the ring restarts one phase on (below).
-    uint32_t n_spec = 0;
-    if (!kPaged && warp == kProducerWarp && lane == 0 && guess->count > 0) {
-        n_spec = static_cast<uint32_t>(min(static_cast<long long>(kStages),
-                                           min(static_cast<long long>(guess->n - guess->tile), guess->count)));
+    // inputs as they are now: even tiles by the producer, odd ones by
+    // finisher warp 9 (idle until the first segment ends), so the two consumer
+    // groups' first tiles start at once. When the guess and the real start
+    // differ (the lengths changed under the guess), the ring restarts one
+    // phase on (below).
+    const uint32_t n_spec = !kPaged && guess->count > 0
+                                ? static_cast<uint32_t>(min(static_cast<long long>(kStages),
+                                                            min(static_cast<long long>(guess->n - guess->tile),
+                                                                guess->count)))
+                                : 0u;
+    if constexpr (!kPaged) if (lane == 0 && (warp == kProducerWarp || warp == kProducerWarp + 1) && n_spec > 0) {
         const uint64_t policy = l2_policy_evict_first();
         const int z = guess->b * p.Hkv + guess->h;
         const uint16_t *q_row =
             p.q + (static_cast<size_t>(guess->b) * p.q_len * p.Hq + static_cast<size_t>(guess->h) * p.g) * D;
         const uint32_t q_run = static_cast<uint32_t>(p.g) * D * 2;
         const uint32_t q_bytes = static_cast<uint32_t>(p.cols) * D * 2;
-        for (uint32_t t = 0; t < n_spec; ++t) {   // tile t of the first segment into stage t, phase 0
+        // tile t of the first segment into stage t, phase 0
+        for (uint32_t t = warp == kProducerWarp ? 0u : 1u; t < n_spec; t += 2) {
             uint8_t *kt = ring + t * Cfg::kStageBytes;
             uint8_t *vt = kt + Cfg::kTileBytes;
             const bool with_q = static_cast<int>(t) < kGroupsC;
@@ -882,14 +954,20 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
                               &full[t]);
         }
     }
+    // Warp 0 publishes the real start through an mbarrier rather than a block
+    // barrier, so the consumers start on the first tiles while the producer is
+    // still issuing.
     if (warp == 0) {
         find_start<false>(p, info);
-        if (lane == 0 && !kPaged && guess->count > 0)
-            info->restart = !(info->count == guess->count && info->N == guess->N && info->first == guess->first &&
-                              info->b == guess->b && info->h == guess->h && info->tile == guess->tile &&
-                              info->n == guess->n);
+        if (lane == 0) {
+            if (!kPaged && guess->count > 0)
+                info->restart = !(info->count == guess->count && info->N == guess->N && info->first == guess->first &&
+                                  info->b == guess->b && info->h == guess->h && info->tile == guess->tile &&
+                                  info->n == guess->n);
+            mbar_arrive(startbar);
+        }
     }
-    __syncthreads();
+    wait_start(startbar);
     // After a wrong guess (the same decision in every thread): the producer lets
     // the guessed copies land (bounded), completes phase 0 of every stage with
     // nothing else in it, and everyone goes on from sequence number kStages
@@ -899,7 +977,7 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
     if (restart) {
         if (warp == kProducerWarp && lane == 0)
             for (int s2 = 0; s2 < kStages; ++s2) {
-                if (static_cast<uint32_t>(s2) < n_spec)
+                if (!kPaged && static_cast<int>(n_spec) > s2)
                     drain_phase(&full[s2], 0);
                 else
                     mbar_arrive(&full[s2]);

@@ -306,7 +306,9 @@ FD_API int fd_segments(int B, int Hkv, int max_len, const int32_t *seqlens_host,
  * cudaFree, no allocating library call.
  * The first call on each device looks up the buffer's device address
  * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture. Every call clears the buffer's per-row counters
+ * before any stream capture. If that lookup fails the call returns
+ * FD_ERR_LAUNCH, nothing is remembered, and the next call tries again; the
+ * address is kept once a lookup succeeds. Every call clears the buffer's per-row counters
  * (cudaMemsetAsync on `stream`) and then reuses it, so the buffer keeps the
  * last call's segments. All calls on one device share the one buffer: two
  * calls that can overlap on the GPU (different streams, no ordering between

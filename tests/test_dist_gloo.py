@@ -101,3 +101,44 @@ def test_token_ranges_tile_the_cache():
             assert rs[0][0] == 0 and rs[-1][1] == Lmax
             assert all(rs[i][1] == rs[i + 1][0] for i in range(world - 1))
             assert max(h - l for l, h in rs) - min(h - l for l, h in rs) <= 1
+
+
+# ------------------------------------------------ bench.py --gpus N launcher --
+
+def _bench(args, env_extra, timeout=300):
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", **env_extra)   # the CPU path: gloo
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        if k not in env_extra:
+            env.pop(k, None)
+    r = subprocess.run([sys.executable, "bench.py", *args], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=timeout)
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    return r, [json.loads(ln) for ln in lines]
+
+
+def test_bench_gpus_flag_starts_one_process_per_rank():
+    """`bench.py --gpus 2` outside torchrun starts two ranks itself; both
+    join one process group and rank 0 alone prints the line."""
+    r, lines = _bench(["--gpus", "2", "--check-launch"], {})
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert len(lines) == 1
+    d = lines[0]
+    assert d["n_gpus"] == 2 and d["ranks_joined"] == 2 and d["backend"] == "gloo"
+    assert len(set(d["pids"])) == 2 and os.getpid() not in d["pids"]
+
+
+def test_bench_rejects_a_world_size_that_differs_from_gpus():
+    r, lines = _bench(["--gpus", "2", "--check-launch"], {"WORLD_SIZE": "3", "RANK": "0"})
+    assert r.returncode != 0 and not lines
+    assert "WORLD_SIZE=3 but --gpus 2" in r.stderr
+
+
+def test_bench_single_rank_needs_no_process_group():
+    r, lines = _bench(["--check-launch"], {})
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert lines == [{"check_launch": True, "n_gpus": 1, "ranks_joined": 1, "pids": lines[0]["pids"],
+                      "backend": None}]

@@ -8,7 +8,10 @@ argument and uses the library's fixed device scratch buffer instead.
 Each check calls the entry point through the C ABI twice in a row, with
 different inputs, and compares both results with fd_decode (the entry point
 that takes a caller-allocated workspace) on the same inputs, within the
-parity tolerances used everywhere else. This file is collected last, so a
+parity tolerances used everywhere else. Two more checks compare it with the
+CPU oracle directly, so its parity does not rest on fd_decode alone: one on
+a problem cut into many segments, one on a problem the planner leaves
+unsplit (no scratch is needed, so the fixed buffer is never touched). This file is collected last, so a
 run that stops at the first failure has already run every other test; it
 passes on its own in a fresh process as well as after the other tests.
 """
@@ -20,7 +23,7 @@ import torch
 
 import decode_attention_07_b200 as fd
 from decode_attention_07_b200.configs import WORKLOADS, Workload
-from decode_attention_07_b200.inputs import make_inputs
+from decode_attention_07_b200.inputs import bf16_bits, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -83,6 +86,32 @@ def test_two_calls_match_the_workspace_entry_point(name):
         ref_out, ref_lse = fd.decode(x.q, x.k, x.v, x.seqlens, x.scale)
         torch.cuda.synchronize()
         assert_close(out, lse, ref_out, ref_lse, f"{name}, call {call + 1}")
+
+
+ORACLE_CASES = {
+    # B = 3, L up to 3000: many segments per row, NaN padding, an empty row
+    "split": [(Workload("orc", B=3, Hq=8, Hkv=2, D=128, Lmax=3000, ragged=False, sigma_k=3.0, nan_pad=True),
+               5, [3000, 700, 0]),
+              (Workload("orc", B=3, Hq=8, Hkv=2, D=128, Lmax=3000, ragged=False, sigma_k=3.0, nan_pad=True),
+               6, [1, 2999, 1500])],
+    # 4 tiles in all: the planner picks one split and no scratch is needed
+    "unsplit": [(Workload("one", B=1, Hq=4, Hkv=1, D=128, Lmax=200, ragged=False), 7, None),
+                (Workload("one", B=1, Hq=4, Hkv=1, D=128, Lmax=200, ragged=False), 8, [131])],
+}
+
+
+@pytest.mark.parametrize("name", list(ORACLE_CASES))
+def test_two_calls_match_the_oracle(name, orc):
+    for call, (w, seed, lens) in enumerate(ORACLE_CASES[name]):
+        S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.Lmax)
+        assert (S == 1) == (name == "unsplit")
+        x = make_inputs(w, seed, device="cuda", seqlens=lens)
+        out = torch.full((w.B, w.Hq, w.D), 99.0, device="cuda")
+        lse = torch.full((w.B, w.Hq), 99.0, device="cuda")
+        assert static_call(x, out, lse) == 0
+        torch.cuda.synchronize()
+        ref_out, ref_lse = orc.attention(bf16_bits(x.q), bf16_bits(x.k), bf16_bits(x.v), x.seqlens_host, x.scale)
+        assert_close(out, lse, torch.from_numpy(ref_out), torch.from_numpy(ref_lse), f"{name}, call {call + 1}")
 
 
 def test_rejects_problems_beyond_the_fixed_buffer():
