@@ -207,6 +207,17 @@ int encode_cache_map(CUtensorMap *map, const void *base, int D, int Lmax, long l
                         strides, box, swz);
 }
 
+// bf16 cache at D = 128 for the one-head consumer: each 256-byte token row
+// seen as two 128-byte halves, {64 elements, 2 halves, Lmax tokens, rows},
+// box {64, 2, 64, 1}: one copy brings a whole 64-token tile of one row as
+// [token][half][128 B] with the 128-byte swizzle.
+int encode_cache_map_rows(CUtensorMap *map, const void *base, int Lmax, long long rows) {
+    cuuint64_t dims[4] = {64, 2, static_cast<cuuint64_t>(Lmax), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[3] = {128, 256, static_cast<cuuint64_t>(Lmax) * 256};
+    cuuint32_t box[4] = {64, 2, static_cast<cuuint32_t>(fd::kTileTokens), 1};
+    return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // Paged K or V pool as a 3-D tensor, head-dim innermost. Head-major pages
 // [num_pages][Hkv][page_size][D]: the token rows of one (page, head) are
 // contiguous, so {D, page_size, num_pages * Hkv}, box {64, rows, 1}, row
@@ -463,9 +474,16 @@ int run_split(const Problem &pr, bool fused, int q_len = 1) {
     std::memset(&tk, 0, sizeof tk);
     std::memset(&tv, 0, sizeof tv);
     const long long rows = static_cast<long long>(pr.B) * pr.Hkv;
+    // one head per kv head at D = 128: one copy per K or V tile (see encode_cache_map_rows)
+    const bool rows_map = pr.D == 128 && pr.Hq / pr.Hkv * q_len == 1;
     if (pr.max_len > 0) {
-        if ((rc = encode_cache_map(&tk, pr.k, pr.D, pr.max_len, rows)) != FD_OK) return rc;
-        if ((rc = encode_cache_map(&tv, pr.v, pr.D, pr.max_len, rows)) != FD_OK) return rc;
+        if (rows_map) {
+            if ((rc = encode_cache_map_rows(&tk, pr.k, pr.max_len, rows)) != FD_OK) return rc;
+            if ((rc = encode_cache_map_rows(&tv, pr.v, pr.max_len, rows)) != FD_OK) return rc;
+        } else {
+            if ((rc = encode_cache_map(&tk, pr.k, pr.D, pr.max_len, rows)) != FD_OK) return rc;
+            if ((rc = encode_cache_map(&tv, pr.v, pr.D, pr.max_len, rows)) != FD_OK) return rc;
+        }
     } else if (!fused) {
         return FD_OK;   // no tokens anywhere: the combine writes every row
     }
@@ -497,6 +515,9 @@ int run_split(const Problem &pr, bool fused, int q_len = 1) {
     p.debug_spoil_guess = debug_spoil_guess();
     // with max_len == 0 every block finds zero tiles and only writes empty rows;
     // the (unused) tensor maps stay zeroed
+    if (rows_map)
+        return fused ? launch_split_t<128, fd::HeadConsumer<128, true>, true, false>(tk, tv, p, pr.stream)
+                     : launch_split_t<128, fd::HeadConsumer<128, true>, false, false>(tk, tv, p, pr.stream);
     return fused ? launch_split<true>(pr.D, p.cols, tk, tv, p, pr.stream)
                  : launch_split<false>(pr.D, p.cols, tk, tv, p, pr.stream);
 }

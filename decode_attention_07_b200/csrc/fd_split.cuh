@@ -284,6 +284,27 @@ __device__ __forceinline__ int tiles_at(const int32_t *seqlens, int b, int Lmax)
     return kL2Only ? row_tiles_l2(seqlens, b, Lmax) : row_tiles(seqlens, b, Lmax);
 }
 
+// One K and one V tile of a contiguous cache (tokens y .. y+63 of row z)
+// into the stage. Default layout: one 3-D box per 64 head-dim elements.
+// Interleaved layout (bf16, D = 128): one 4-D box {64 elements, 2 halves,
+// 64 tokens, 1 row} per tile, [token][half][128 B] in shared memory, so the
+// producer issues two copies per tile instead of four (every copy costs its
+// issuing thread a fixed time, taken from the warps sharing its scheduler).
+template <class Cfg, bool kInter>
+__device__ __forceinline__ void load_tile(uint8_t *kt, uint8_t *vt, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
+                                          uint64_t *bar, int y, int z, uint64_t policy) {
+    if constexpr (kInter) {
+        tma_load_4d(kt, tm_k, bar, 0, 0, y, z, policy);
+        tma_load_4d(vt, tm_v, bar, 0, 0, y, z, policy);
+    } else {
+#pragma unroll
+        for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+            tma_load_3d(kt + bx * Cfg::kBoxBytes, tm_k, bar, Cfg::kBoxCols * bx, y, z, policy);
+            tma_load_3d(vt + bx * Cfg::kBoxBytes, tm_v, bar, Cfg::kBoxCols * bx, y, z, policy);
+        }
+    }
+}
+
 // Next row with at least one tile (only called while tiles remain).
 __device__ __forceinline__ void next_row(Cursor &c, const SplitParams &p) {
     c.first += c.n;
@@ -943,11 +964,7 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
 #ifdef FD_DEBUG
             if (blockIdx.x == 0 && static_cast<int>(t) == p.debug_withhold) continue;   // armed, never filled
 #endif
-#pragma unroll
-            for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-                tma_load_3d(kt + bx * Cfg::kBoxBytes, &tm_k, &full[t], Cfg::kBoxCols * bx, y, z, policy);
-                tma_load_3d(vt + bx * Cfg::kBoxBytes, &tm_v, &full[t], Cfg::kBoxCols * bx, y, z, policy);
-            }
+            load_tile<Cfg, Consumer::kInterleaved>(kt, vt, &tm_k, &tm_v, &full[t], y, z, policy);
             if (with_q)
                 for (int j = 0; j < p.q_len; ++j)
                     bulk_load(vt + Cfg::kTileBytes + j * q_run, q_row + static_cast<size_t>(j) * p.Hq * D, q_run,
@@ -1058,11 +1075,7 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
                 const int y = (c.tile + k) * kTileTokens;
                 if (!kPaged) {
                     mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kTileBytes + qb);
-#pragma unroll
-                    for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-                        tma_load_3d(kt + bx * Cfg::kBoxBytes, &tm_k, &full[stage], Cfg::kBoxCols * bx, y, z, policy);
-                        tma_load_3d(vt + bx * Cfg::kBoxBytes, &tm_v, &full[stage], Cfg::kBoxCols * bx, y, z, policy);
-                    }
+                    load_tile<Cfg, Consumer::kInterleaved>(kt, vt, &tm_k, &tm_v, &full[stage], y, z, policy);
                 } else {
                     // the tile's tokens [y, y + 64) span one page (page_size >= 64) or
                     // 64 / page_size pages; pages past the sequence's end are not loaded
