@@ -327,6 +327,7 @@ struct QuantConsumer {
     // dims back in order and the value scale applied, then m[G] (base 2,
     // without the 2^kPScale factor), l[G].
     __device__ __forceinline__ void to_smem(float *wb) {
+        constexpr int S = merge_head_stride<D>();
         const int lane = threadIdx.x & 31;
         const int r0 = lane >> 2, cc = lane & 3;
         const int dlo = 2 * r0;   // head dim of accumulator row r0 within its chunk (row r0 + 8: dlo + 1)
@@ -337,19 +338,19 @@ struct QuantConsumer {
 #pragma unroll
                 for (int sh = 4; sh < 32; sh <<= 1) l[nt][e] += __shfl_xor_sync(0xffffffffu, l[nt][e], sh);
             const int ha = nt * 8 + 2 * cc, hb = ha + 1;
+            // dims d0 and d0 + 1 of one head as one 8-byte store; with the padded
+            // head stride the 16 lanes of each half warp fill all 32 banks
 #pragma unroll
             for (int c = 0; c < KC; ++c) {
-                const int d0 = 16 * c + dlo, d1 = d0 + 1;
-                wb[ha * D + d0] = o[nt][c][0] * vmul;
-                wb[hb * D + d0] = o[nt][c][1] * vmul;
-                wb[ha * D + d1] = o[nt][c][2] * vmul;
-                wb[hb * D + d1] = o[nt][c][3] * vmul;
+                const int d0 = 16 * c + dlo;
+                *reinterpret_cast<float2 *>(wb + ha * S + d0) = make_float2(o[nt][c][0] * vmul, o[nt][c][2] * vmul);
+                *reinterpret_cast<float2 *>(wb + hb * S + d0) = make_float2(o[nt][c][1] * vmul, o[nt][c][3] * vmul);
             }
             if (r0 == 0) {
-                wb[G * D + ha] = m[nt][0] == -INFINITY ? -INFINITY : m[nt][0] - kPScale;
-                wb[G * D + hb] = m[nt][1] == -INFINITY ? -INFINITY : m[nt][1] - kPScale;
-                wb[G * D + G + ha] = l[nt][0];
-                wb[G * D + G + hb] = l[nt][1];
+                wb[G * S + ha] = m[nt][0] == -INFINITY ? -INFINITY : m[nt][0] - kPScale;
+                wb[G * S + hb] = m[nt][1] == -INFINITY ? -INFINITY : m[nt][1] - kPScale;
+                wb[G * S + G + ha] = l[nt][0];
+                wb[G * S + G + hb] = l[nt][1];
             }
         }
     }

@@ -123,6 +123,16 @@ __device__ __forceinline__ size_t seg_rows(const SplitParams &p) {
 
 constexpr int kPageWindow = 1024;                 // block-table entries staged in shared memory
 
+// One consumer warp's state in a merge buffer: o[G][D] with a row stride of
+// D + 4 floats, then m[G], l[G], padded to a multiple of 4 floats. The extra
+// 4 floats per head put the accumulator columns that lanes 4 apart hold
+// (heads 2c and 2c + 2) 8 banks apart, so a warp's stores of its
+// accumulators meet no bank conflict.
+template <int D>
+__host__ __device__ constexpr int merge_head_stride() { return D + 4; }
+template <int D, int G>
+__host__ __device__ constexpr int merge_warp_floats() { return (G * merge_head_stride<D>() + 2 * G + 3) / 4 * 4; }
+
 // Byte offset, inside a K or V tile, of 16-byte chunk j (0..7) of the
 // 64-element half `half` of token t. Default layout (one TMA box per half):
 // [half][64 tokens][128 B]. Interleaved layout (one box covers both halves
@@ -157,7 +167,7 @@ struct SplitConfig {
     static constexpr int kTileBytes = kTileTokens * kRowBytes;             // one K (or V) tile
     static constexpr int kQSlotBytes = (G * D * 2 + 1023) / 1024 * 1024;   // query heads of a row (bf16)
     static constexpr int kStageBytes = 2 * kTileBytes + kQSlotBytes;       // multiple of 1024 (swizzle)
-    static constexpr int kWarpFloats = G * D + 2 * G;                      // o, m, l of one warp
+    static constexpr int kWarpFloats = merge_warp_floats<D, G>();          // o, m, l of one warp
     static constexpr int kMergeFloats = kConsumerWarps * kWarpFloats;      // one merge buffer
     static constexpr int kCtrlBytes = 2048;                                // barriers, start info, queue, weights
     static constexpr int kPageBytes = kPageWindow * 4;                     // block-table window (paged)
@@ -444,12 +454,13 @@ template <int D, int G, class Bar>
 __device__ __forceinline__ void merge_warps_and_store(const float *merge, float *weights, const SplitParams &p,
                                                       const Cursor &c, bool whole, size_t slot, int tid,
                                                       int nthreads, Bar bar) {
-    constexpr int kWarpFloats = G * D + 2 * G;
+    constexpr int kWarpFloats = merge_warp_floats<D, G>();
+    constexpr int S = merge_head_stride<D>();
     float *lse_h = weights + G * kConsumerWarps;   // [G] natural-log lse per head
     for (int head = tid; head < p.cols; head += nthreads) {
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge[w * kWarpFloats + G * D + head]);
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge[w * kWarpFloats + G * S + head]);
         if (M == -INFINITY) {
 #pragma unroll
             for (int w = 0; w < kConsumerWarps; ++w) weights[head * kConsumerWarps + w] = 0.f;
@@ -458,8 +469,8 @@ __device__ __forceinline__ void merge_warps_and_store(const float *merge, float 
             float e[kConsumerWarps], lsum = 0.f;
 #pragma unroll
             for (int w = 0; w < kConsumerWarps; ++w) {
-                e[w] = ex2(merge[w * kWarpFloats + G * D + head] - M);
-                lsum = fmaf(e[w], merge[w * kWarpFloats + G * D + G + head], lsum);
+                e[w] = ex2(merge[w * kWarpFloats + G * S + head] - M);
+                lsum = fmaf(e[w], merge[w * kWarpFloats + G * S + G + head], lsum);
             }
             const float inv = 1.f / lsum;
 #pragma unroll
@@ -473,7 +484,7 @@ __device__ __forceinline__ void merge_warps_and_store(const float *merge, float 
         float o = 0.f;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w)
-            o = fmaf(weights[head * kConsumerWarps + w], merge[w * kWarpFloats + head * D + d], o);
+            o = fmaf(weights[head * kConsumerWarps + w], merge[w * kWarpFloats + head * S + d], o);
         if (whole) {
             const size_t row = out_row(p, c.b, c.h, head);
             if (!FD_DCHECK(row < out_rows(p))) continue;
@@ -643,6 +654,7 @@ struct GroupConsumer {
     }
 
     __device__ __forceinline__ void to_smem(float *wb) {
+        constexpr int S = merge_head_stride<D>();
         const int lane = threadIdx.x & 31;
         const int r0 = lane >> 2, cc = lane & 3;
 #pragma unroll
@@ -655,16 +667,16 @@ struct GroupConsumer {
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 const int d0 = 16 * mt + r0, d1 = d0 + 8;
-                wb[ha * D + d0] = o[nt][mt][0];
-                wb[hb * D + d0] = o[nt][mt][1];
-                wb[ha * D + d1] = o[nt][mt][2];
-                wb[hb * D + d1] = o[nt][mt][3];
+                wb[ha * S + d0] = o[nt][mt][0];
+                wb[hb * S + d0] = o[nt][mt][1];
+                wb[ha * S + d1] = o[nt][mt][2];
+                wb[hb * S + d1] = o[nt][mt][3];
             }
             if (r0 == 0) {
-                wb[G * D + ha] = m[nt][0];
-                wb[G * D + hb] = m[nt][1];
-                wb[G * D + G + ha] = l[nt][0];
-                wb[G * D + G + hb] = l[nt][1];
+                wb[G * S + ha] = m[nt][0];
+                wb[G * S + hb] = m[nt][1];
+                wb[G * S + G + ha] = l[nt][0];
+                wb[G * S + G + hb] = l[nt][1];
             }
         }
     }
@@ -832,13 +844,13 @@ struct HeadConsumer {
         float ls = l;
 #pragma unroll
         for (int s = 1; s < 32; s <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, s);
-        if (lane < LPT) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) wb[8 * lane + k] = acc[k];
+        if (lane < LPT) {   // two 16-byte stores per lane (the warp's slot is 16-byte aligned)
+            reinterpret_cast<float4 *>(wb)[2 * lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            reinterpret_cast<float4 *>(wb)[2 * lane + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
         }
         if (lane == 0) {
-            wb[D] = m;
-            wb[D + 1] = ls;
+            wb[merge_head_stride<D>()] = m;
+            wb[merge_head_stride<D>() + 1] = ls;
         }
     }
 };
