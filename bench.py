@@ -344,7 +344,7 @@ class Workspace:
     when a copy is larger than L2, so no call finds its predecessor's bytes
     in L2; one copy otherwise, with L2 flushed before every timed call)."""
 
-    def __init__(self, w, kv, seed, dev, stream, q_len=1, paged=0, layout="HND"):
+    def __init__(self, w, kv, seed, dev, stream, q_len=1, paged=0, layout="HND", page_order="shuffled"):
         self.w, self.kv, self.dev, self.stream = w, kv, dev, stream
         self.quant = kv != "bf16"
         self.S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.Lmax)
@@ -381,7 +381,7 @@ class Workspace:
         if paged:
             # the same logical caches, scattered into shuffled page pools
             from decode_attention_07_b200.inputs import make_paged
-            pgs = [make_paged(x, paged, layout, seed=7 + i) for i, x in enumerate(xs)]
+            pgs = [make_paged(x, paged, layout, seed=7 + i, order=page_order) for i, x in enumerate(xs)]
             for x in xs:   # the contiguous copies are not used by the paged calls
                 if self.quant:
                     x.k8 = x.v8 = None
@@ -516,7 +516,7 @@ def run_fd(args, w, rank, world):
     stream = torch.cuda.current_stream(dev)
     quant = args.kv != "bf16"
     Q = args.q_len
-    wk = Workspace(w, args.kv, rank_seed(args.seed, rank), dev, stream, Q, args.paged, args.layout)
+    wk = Workspace(w, args.kv, rank_seed(args.seed, rank), dev, stream, Q, args.paged, args.layout, args.page_order)
     S, n_copies, xs, out, lse, ws = wk.S, wk.n_copies, wk.xs, wk.out, wk.lse, wk.ws
     counts, kv_bytes, calls = wk.counts, wk.kv_bytes, wk.calls
 
@@ -645,7 +645,8 @@ def run_fd(args, w, rank, world):
         "warmup": max(3, args.warmup), "ms_per_step": ms_max / args.steps, "us_per_call": us_per_call,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": args.kv, "data": "synthetic",
         "config": dict(config_dict(w, S, wk.l2_note), **({"kv_cache": args.kv} if quant else {}),
-                       **({"paged": {"page_size": args.paged, "layout": args.layout}} if args.paged else {}),
+                       **({"paged": {"page_size": args.paged, "layout": args.layout, "page_order": args.page_order}}
+                          if args.paged else {}),
                        **({"q_len": Q} if Q > 1 else {})),
         "pct_of_nominal_hbm": 100.0 * gbs / world / NOMINAL_HBM_GBS,
         "pct_of_measured_copy": 100.0 * gbs / world / peak,
@@ -880,6 +881,8 @@ def main():
     ap.add_argument("--paged", type=int, default=0, metavar="PAGE_SIZE",
                     help="read the caches from a shuffled page pool with this page size (fd_decode_paged)")
     ap.add_argument("--layout", choices=["HND", "NHD"], default="HND", help="page layout for --paged")
+    ap.add_argument("--page-order", choices=["shuffled", "inorder"], default="shuffled",
+                    help="--paged: pool pages in a shuffled order, or in sequence order (consecutive pages)")
     ap.add_argument("--cp", action="store_true",
                     help="context parallelism: shard the cache's tokens over the ranks (strong scaling)")
     ap.add_argument("--kv", choices=["bf16", "e4m3", "int8"], default="bf16",

@@ -261,7 +261,8 @@ int encode_paged_map(CUtensorMap *map, const void *base, int D, int page_size, i
 // [token][half][128 B] with the 128-byte swizzle. Head-major pages:
 // {64, 2, page_size, Hkv, num_pages}, box {64, 2, page_size, 1, 1}; token-major:
 // {64, 2, Hkv, page_size, num_pages}, box {64, 2, 1, page_size, 1}.
-int encode_paged_map_rows(CUtensorMap *map, const void *base, int page_size, int Hkv, long long num_pages, bool nhd) {
+int encode_paged_map_rows(CUtensorMap *map, const void *base, int page_size, int Hkv, long long num_pages, bool nhd,
+                          int pages_per_box = 1) {
     const cuuint64_t row = 256;   // bytes of one token of one head (D = 128, bf16)
     cuuint64_t dims[5], strides[4];
     cuuint32_t box[5];
@@ -271,7 +272,7 @@ int encode_paged_map_rows(CUtensorMap *map, const void *base, int page_size, int
     strides[0] = 128;
     box[0] = 64;
     box[1] = 2;
-    box[4] = 1;
+    box[4] = static_cast<cuuint32_t>(pages_per_box);
     if (nhd) {
         dims[2] = static_cast<cuuint64_t>(Hkv);
         dims[3] = static_cast<cuuint64_t>(page_size);
@@ -289,6 +290,35 @@ int encode_paged_map_rows(CUtensorMap *map, const void *base, int page_size, int
     }
     strides[3] = static_cast<cuuint64_t>(page_size) * Hkv * row;
     return encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Small pages (page_size < 64): one box over a run of 64 / page_size
+// consecutive pages of one kv head, for tiles whose pages are consecutive in
+// the pool (the same bytes at the same places as one box per page). Head-major
+// pages: {D, page_size, Hkv, num_pages}, box {cols, page_size, 1, pages};
+// token-major: {D, Hkv, num_pages * page_size}, box {cols, 1, 64} (the pages'
+// tokens are one range of the third dimension). cols = 64 bf16 or all D codes.
+int encode_paged_run_map(CUtensorMap *map, const void *base, int D, int page_size, int Hkv, long long num_pages,
+                         bool nhd, bool one_byte) {
+    const cuuint64_t e = one_byte ? 1 : 2;
+    const cuuint64_t row = static_cast<cuuint64_t>(D) * e;
+    const cuuint32_t cols = one_byte ? static_cast<cuuint32_t>(D) : 64u;
+    const CUtensorMapSwizzle swz = one_byte && D == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    const CUtensorMapDataType dt = one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (nhd) {
+        cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv),
+                              static_cast<cuuint64_t>(num_pages) * page_size};
+        cuuint64_t strides[2] = {row, static_cast<cuuint64_t>(Hkv) * row};
+        cuuint32_t box[3] = {cols, 1, static_cast<cuuint32_t>(fd::kTileTokens)};
+        return encode_tiled(map, dt, 3, base, dims, strides, box, swz);
+    }
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(page_size), static_cast<cuuint64_t>(Hkv),
+                          static_cast<cuuint64_t>(num_pages)};
+    cuuint64_t strides[3] = {row, static_cast<cuuint64_t>(page_size) * row,
+                             static_cast<cuuint64_t>(page_size) * Hkv * row};
+    cuuint32_t box[4] = {cols, static_cast<cuuint32_t>(page_size), 1,
+                         static_cast<cuuint32_t>(fd::kTileTokens / page_size)};
+    return encode_tiled(map, dt, 4, base, dims, strides, box, swz);
 }
 
 // Host-side failure injection for tests: with FD_TEST_FAIL_LAUNCH set in the
@@ -328,7 +358,8 @@ int debug_spoil_guess() {
 
 // ---------------------------------------------------------------- launches --
 template <int D, class Consumer, bool kFused, bool kPaged>
-int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p, cudaStream_t st) {
+int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p, cudaStream_t st,
+                   const CUtensorMap *rk = nullptr, const CUtensorMap *rv = nullptr) {
     constexpr int smem = fd::SplitConfig<D, Consumer::G, Consumer::kElemBytes, kPaged>::kSmemBytes;
     auto kern = fd::fd_split_kernel<D, Consumer, kFused, kPaged>;
     // the attribute is per function and device; set it once per device
@@ -360,7 +391,8 @@ int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::Split
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (inject_launch_failure()) return FD_ERR_LAUNCH;
-    if (cudaLaunchKernelEx(&cfg, kern, tk, tv, p) != cudaSuccess) {
+    // the maps of consecutive page runs (small pages only; never read otherwise)
+    if (cudaLaunchKernelEx(&cfg, kern, tk, tv, rk ? *rk : tk, rv ? *rv : tv, p) != cudaSuccess) {
         cudaGetLastError();
         return FD_ERR_LAUNCH;
     }
@@ -369,29 +401,30 @@ int launch_split_t(const CUtensorMap &tk, const CUtensorMap &tv, const fd::Split
 
 template <bool kFused, bool kPaged = false>
 int launch_split(int D, int g, const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p,
-                 cudaStream_t st) {
+                 cudaStream_t st, const CUtensorMap *rk = nullptr, const CUtensorMap *rv = nullptr) {
     if (D == 128) {
-        if (g == 1) return launch_split_t<128, fd::HeadConsumer<128>, kFused, kPaged>(tk, tv, p, st);
-        if (g <= 8) return launch_split_t<128, fd::GroupConsumer<128, 1>, kFused, kPaged>(tk, tv, p, st);
-        return launch_split_t<128, fd::GroupConsumer<128, 2>, kFused, kPaged>(tk, tv, p, st);
+        if (g == 1) return launch_split_t<128, fd::HeadConsumer<128>, kFused, kPaged>(tk, tv, p, st, rk, rv);
+        if (g <= 8) return launch_split_t<128, fd::GroupConsumer<128, 1>, kFused, kPaged>(tk, tv, p, st, rk, rv);
+        return launch_split_t<128, fd::GroupConsumer<128, 2>, kFused, kPaged>(tk, tv, p, st, rk, rv);
     }
-    if (g == 1) return launch_split_t<64, fd::HeadConsumer<64>, kFused, kPaged>(tk, tv, p, st);
-    if (g <= 8) return launch_split_t<64, fd::GroupConsumer<64, 1>, kFused, kPaged>(tk, tv, p, st);
-    return launch_split_t<64, fd::GroupConsumer<64, 2>, kFused, kPaged>(tk, tv, p, st);
+    if (g == 1) return launch_split_t<64, fd::HeadConsumer<64>, kFused, kPaged>(tk, tv, p, st, rk, rv);
+    if (g <= 8) return launch_split_t<64, fd::GroupConsumer<64, 1>, kFused, kPaged>(tk, tv, p, st, rk, rv);
+    return launch_split_t<64, fd::GroupConsumer<64, 2>, kFused, kPaged>(tk, tv, p, st, rk, rv);
 }
 
 // 8-bit caches: the tensor-core consumer for every column count (fused form).
 template <bool kE4M3, bool kPaged = false>
 int launch_split_quant(int D, int cols, const CUtensorMap &tk, const CUtensorMap &tv, const fd::SplitParams &p,
-                       cudaStream_t st) {
+                       cudaStream_t st, const CUtensorMap *rk = nullptr, const CUtensorMap *rv = nullptr) {
     // up to 8 columns: four groups of two warps, 32 tokens per warp (more work
     // in flight per warp); 16 columns: the default two groups of four
     if (D == 128) {
-        if (cols <= 8) return launch_split_t<128, fd::QuantConsumer<128, 1, kE4M3, 32>, true, kPaged>(tk, tv, p, st);
-        return launch_split_t<128, fd::QuantConsumer<128, 2, kE4M3, 16>, true, kPaged>(tk, tv, p, st);
+        if (cols <= 8)
+            return launch_split_t<128, fd::QuantConsumer<128, 1, kE4M3, 32>, true, kPaged>(tk, tv, p, st, rk, rv);
+        return launch_split_t<128, fd::QuantConsumer<128, 2, kE4M3, 16>, true, kPaged>(tk, tv, p, st, rk, rv);
     }
-    if (cols <= 8) return launch_split_t<64, fd::QuantConsumer<64, 1, kE4M3, 32>, true, kPaged>(tk, tv, p, st);
-    return launch_split_t<64, fd::QuantConsumer<64, 2, kE4M3, 16>, true, kPaged>(tk, tv, p, st);
+    if (cols <= 8) return launch_split_t<64, fd::QuantConsumer<64, 1, kE4M3, 32>, true, kPaged>(tk, tv, p, st, rk, rv);
+    return launch_split_t<64, fd::QuantConsumer<64, 2, kE4M3, 16>, true, kPaged>(tk, tv, p, st, rk, rv);
 }
 
 int launch_combine(int D, const fd::CombineParams &p, cudaStream_t st, bool after_split) {
@@ -539,15 +572,32 @@ int run_split_paged(const Problem &pr, const PagedLayout &pl, int q_len = 1, int
     const bool quant = kv_type != 0;
     // bf16 at D = 128 with small pages: one box per page (both 128-byte halves of a row)
     const bool rows_map = !quant && pr.D == 128 && pl.page_size < fd::kTileTokens;
+    // small pages: maps of runs of 64 / page_size consecutive pages (one box per such tile)
+    CUtensorMap rk, rv;
+    const bool small = pl.page_size < fd::kTileTokens && pl.num_pages >= fd::kTileTokens / pl.page_size;
     if (rows_map) {
         if ((rc = encode_paged_map_rows(&tk, pr.k, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
         if ((rc = encode_paged_map_rows(&tv, pr.v, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd)) != FD_OK) return rc;
+        const int ppb = fd::kTileTokens / pl.page_size;
+        if (small) {
+            if ((rc = encode_paged_map_rows(&rk, pr.k, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd, ppb)) != FD_OK)
+                return rc;
+            if ((rc = encode_paged_map_rows(&rv, pr.v, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd, ppb)) != FD_OK)
+                return rc;
+        }
     } else {
         if ((rc = encode_paged_map(&tk, pr.k, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd, quant)) != FD_OK)
             return rc;
         if ((rc = encode_paged_map(&tv, pr.v, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd, quant)) != FD_OK)
             return rc;
+        if (small) {
+            if ((rc = encode_paged_run_map(&rk, pr.k, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd, quant)) != FD_OK)
+                return rc;
+            if ((rc = encode_paged_run_map(&rv, pr.v, pr.D, pl.page_size, pr.Hkv, pl.num_pages, pl.nhd, quant)) != FD_OK)
+                return rc;
+        }
     }
+    const CUtensorMap *rkp = small ? &rk : nullptr, *rvp = small ? &rv : nullptr;
     fd::SplitParams p;
     p.q = pr.q;
     p.seqlens = pr.seqlens;
@@ -576,15 +626,16 @@ int run_split_paged(const Problem &pr, const PagedLayout &pl, int q_len = 1, int
     p.debug_withhold = debug_withhold();
     p.debug_spoil_guess = debug_spoil_guess();
     if (quant)
-        return kv_type == FD_KV_E4M3 ? launch_split_quant<true, true>(pr.D, p.cols, tk, tv, p, pr.stream)
-                                     : launch_split_quant<false, true>(pr.D, p.cols, tk, tv, p, pr.stream);
+        return kv_type == FD_KV_E4M3 ? launch_split_quant<true, true>(pr.D, p.cols, tk, tv, p, pr.stream, rkp, rvp)
+                                     : launch_split_quant<false, true>(pr.D, p.cols, tk, tv, p, pr.stream, rkp, rvp);
     if (rows_map) {
-        if (p.cols == 1) return launch_split_t<128, fd::HeadConsumer<128, true>, true, true>(tk, tv, p, pr.stream);
+        if (p.cols == 1)
+            return launch_split_t<128, fd::HeadConsumer<128, true>, true, true>(tk, tv, p, pr.stream, rkp, rvp);
         if (p.cols <= 8)
-            return launch_split_t<128, fd::GroupConsumer<128, 1, true>, true, true>(tk, tv, p, pr.stream);
-        return launch_split_t<128, fd::GroupConsumer<128, 2, true>, true, true>(tk, tv, p, pr.stream);
+            return launch_split_t<128, fd::GroupConsumer<128, 1, true>, true, true>(tk, tv, p, pr.stream, rkp, rvp);
+        return launch_split_t<128, fd::GroupConsumer<128, 2, true>, true, true>(tk, tv, p, pr.stream, rkp, rvp);
     }
-    return launch_split<true, true>(pr.D, p.cols, tk, tv, p, pr.stream);
+    return launch_split<true, true>(pr.D, p.cols, tk, tv, p, pr.stream, rkp, rvp);
 }
 
 // Fused split kernel over an 8-bit cache (pr.k / pr.v point at the codes).

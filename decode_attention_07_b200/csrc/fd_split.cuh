@@ -859,6 +859,7 @@ struct HeadConsumer {
 template <int D, class Consumer, bool kFused, bool kPaged = false>
 __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
     fd_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_vr,
                     const SplitParams p) {
     constexpr int G = Consumer::G;
     using Cfg = SplitConfig<D, G, Consumer::kElemBytes, kPaged>;
@@ -921,6 +922,10 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
     if (warp == kProducerWarp && lane == 0) {   // kernel parameters, not inputs: safe before the wait
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
+        if (kPaged && p.page_shift < 6) {        // small pages: the maps of runs of consecutive pages
+            prefetch_tensormap(&tm_kr);
+            prefetch_tensormap(&tm_vr);
+        }
     }
     // While the previous grid drains (HBM mostly idle), guess this block's
     // first tiles from seqlens as read now and pull them into L2. L2 is the
@@ -1035,8 +1040,10 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
         int win_b = -1, win_lo = 0, win_hi = 0;
         uint32_t win_phase = 0;
         bool win_pending = false;   // a window copy issued and not yet seen complete
-        auto page_of = [&](int b, int lp, int *page) -> bool {
-            if (b != win_b || lp < win_lo || lp >= win_hi) {
+        // page of logical page lp; with need > 1 the window is also made to hold
+        // pages lp .. lp + need - 1 (need <= 8, all of them pages of the sequence)
+        auto page_of = [&](int b, int lp, int *page, int need = 1) -> bool {
+            if (b != win_b || lp < win_lo || lp + need > win_hi) {
                 win_b = b;
                 win_lo = lp & ~3;
                 win_hi = min(win_lo + kPageWindow, p.max_pages);
@@ -1108,12 +1115,39 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
                             return;
                         }
                     } else {
-                        for (int j = 0; j < nsub; ++j)
-                            if (!page_of(c.b, lp0 + j, &page[j])) {
-                                drain_copies<kStages>(full, seq, wbar, win_pending, win_phase);
-                                return;
-                            }
+                        // the tile's pages lp0 .. lp0 + nsub - 1 (lp0 a multiple of 64 / page_size):
+                        // one window check for all of them, then vector loads from the window
+                        // (the window starts at a multiple of 4 pages and is 16-byte aligned)
+                        if (!(c.b == win_b && lp0 >= win_lo && lp0 + nsub <= win_hi) &&
+                            !page_of(c.b, lp0, &page[0], nsub)) {
+                            drain_copies<kStages>(full, seq, wbar, win_pending, win_phase);
+                            return;
+                        }
+                        const int* wp = win + (lp0 - win_lo);
+                        const int full_tile = kTileTokens >> p.page_shift;
+                        if (nsub == full_tile && full_tile >= 4) {
+#pragma unroll
+                            for (int j4 = 0; j4 < kTileTokens / 8; j4 += 4)
+                                if (j4 < nsub) {
+                                    const int4 v4 = *reinterpret_cast<const int4 *>(wp + j4);
+                                    page[j4] = v4.x;
+                                    page[j4 + 1] = v4.y;
+                                    page[j4 + 2] = v4.z;
+                                    page[j4 + 3] = v4.w;
+                                }
+                        } else {
+                            for (int j = 0; j < nsub; ++j) page[j] = wp[j];
+                        }
                     }
+                    // small pages: when the tile's pages are consecutive pages of the pool
+                    // (an allocator that hands out pages in order), one box of the run maps
+                    // brings them all, with the same bytes at the same places
+                    bool run = psize < kTileTokens && nsub == (kTileTokens >> p.page_shift) && page[0] >= 0 &&
+                               page[0] <= p.num_pages - nsub;
+#pragma unroll
+                    for (int j = 1; j < kTileTokens / 8; ++j)
+                        if (j < nsub) run = run && page[j] == page[0] + j;
+                    const CUtensorMap *rmap = v_role ? &tm_vr : &tm_kr;
                     if constexpr (Consumer::kInterleaved) {
                         // one 5-D box per page, both halves of its tokens: [token][half][128 B].
                         // Coordinates {element, half, token, head, page} (head-major pages)
@@ -1123,14 +1157,32 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
                         const int cz = p.kv_nhd ? c.h : off, cw = p.kv_nhd ? off : c.h;
                         const CUtensorMap *map = v_role ? &tm_v : &tm_k;
                         uint8_t *dst = v_role ? vt : kt;
-                        for (int j = 0; j < nsub; ++j)
-                            tma_load_5d(dst + j * page_bytes, map, &full[stage], 0, 0, cz, cw, page[j], policy);
+                        if (run)   // box {64, 2, page_size, 1, nsub} (head-major) or {64, 2, 1, page_size, nsub}
+                            tma_load_5d(dst, rmap, &full[stage], 0, 0, cz, cw, page[0], policy);
+                        else
+                            for (int j = 0; j < nsub; ++j)
+                                tma_load_5d(dst + j * page_bytes, map, &full[stage], 0, 0, cz, cw, page[j], policy);
                     } else {
                         // a page's rows of one box column land at j * rows box rows
                         const uint32_t sub_bytes = static_cast<uint32_t>(rows) * Cfg::kBoxRowBytes;
                         mbar_arrive_expect_tx(&full[stage], nsub * sub_bytes * Cfg::kBoxes + qb);
                         const CUtensorMap *map = v_role ? &tm_v : &tm_k;
                         uint8_t *dstb = v_role ? vt : kt;
+                        if (run) {
+                            // run maps: {element, token, head, page} with box {cols, page_size, 1, nsub}
+                            // (head-major) or {element, head, page * page_size + token} with box
+                            // {cols, 1, 64} (token-major): page j's rows land at j * rows box rows
+#pragma unroll
+                            for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+                                const int x = Cfg::kBoxCols * bx;
+                                if (p.kv_nhd)
+                                    tma_load_3d(dstb + bx * Cfg::kBoxBytes, rmap, &full[stage], x, c.h,
+                                                page[0] << p.page_shift, policy);
+                                else
+                                    tma_load_4d(dstb + bx * Cfg::kBoxBytes, rmap, &full[stage], x, 0, c.h, page[0],
+                                                policy);
+                            }
+                        } else
                         for (int j = 0; j < nsub; ++j) {
                             const int pgj = psize >= kTileTokens ? page1 : page[j];
 #pragma unroll

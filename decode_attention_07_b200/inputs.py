@@ -102,12 +102,15 @@ class PagedInputs:
 
 
 def make_paged(x: DecodeInputs, page_size: int, layout: str = "HND", seed: int = 0, spare_pages: int = 3,
-               unused_entry: int = -1) -> PagedInputs:
-    """Scatter x's cache into a shuffled pool of pages (data movement only).
+               unused_entry: int = -1, order: str = "shuffled") -> PagedInputs:
+    """Scatter x's cache into a pool of pages (data movement only).
 
     Sequence b needs ceil(seqlens[b] / page_size) pages; the pool holds those
     plus `spare_pages` more, in an order drawn from a CPU generator seeded
-    `seed`. Block-table entries past a sequence's pages are `unused_entry`;
+    `seed` (order "shuffled"), or in sequence order, sequence after sequence
+    (order "inorder": consecutive logical pages are consecutive pool pages,
+    as an allocator that hands out pages in order produces). Block-table
+    entries past a sequence's pages are `unused_entry`;
     pool slots that no sequence position maps to are NaN (for an 8-bit cache,
     QuantInputs: its padding code, and the pools hold codes)."""
     w = x.workload
@@ -120,8 +123,13 @@ def make_paged(x: DecodeInputs, page_size: int, layout: str = "HND", seed: int =
     max_pages = max(1, -(-w.Lmax // page_size))
     max_pages = (max_pages + 3) // 4 * 4
     total = sum(need) + spare_pages
-    g = torch.Generator(device="cpu").manual_seed(int(seed))
-    order = torch.randperm(total, generator=g).numpy()
+    if order not in ("shuffled", "inorder"):
+        raise ValueError("order must be 'shuffled' or 'inorder'")
+    if order == "inorder":
+        order = np.arange(total)
+    else:
+        g = torch.Generator(device="cpu").manual_seed(int(seed))
+        order = torch.randperm(total, generator=g).numpy()
     table = np.full((w.B, max_pages), unused_entry, dtype=np.int32)
     shape = (total, w.Hkv, page_size, w.D) if layout == "HND" else (total, page_size, w.Hkv, w.D)
     k_pages = torch.full(shape, fill, dtype=src_k.dtype, device=dev)

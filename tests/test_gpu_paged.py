@@ -106,3 +106,52 @@ def test_page_outside_the_pool_reads_zeros(layout, page_size, g):
         x.v[b, :, lp * page_size:(lp + 1) * page_size] = 0
     ref_o, ref_l = oracle_rows(x)
     compare(out, lse, ref_o, ref_l, f"out-of-pool pages, {page_size} {layout}")
+
+
+@pytest.mark.parametrize("layout", ["HND", "NHD"])
+@pytest.mark.parametrize("page_size", [8, 16, 32])
+@pytest.mark.parametrize("g,D", [(1, 128), (4, 128), (1, 64), (16, 128)])
+def test_consecutive_pages_one_box(layout, page_size, g, D):
+    """Small pages that are consecutive in the pool are brought by one box per
+    tile (a map over runs of pages): an in-order pool, and one where some
+    tiles' pages are consecutive and others are not (two logical pages
+    swapped, a run ending at the pool's last page), give bitwise the same
+    out/lse as the contiguous path."""
+    w = Workload("paged", B=3, Hq=2 * g, Hkv=2, D=D, Lmax=2000, ragged=False, sigma_k=3.0, nan_pad=True)
+    x = make_inputs(w, 13, device="cuda", seqlens=[2000, 700, 1])
+    S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.Lmax)
+    out_c, lse_c = fd.decode(x.q, x.k, x.v, x.seqlens, x.scale, num_splits=S)
+    pg = make_paged(x, page_size, layout, order="inorder", spare_pages=0)
+    out_p, lse_p = fd.decode_paged(x.q, pg.k_pages, pg.v_pages, pg.block_table, x.seqlens, x.scale, layout=layout,
+                                   num_splits=S)
+    torch.cuda.synchronize()
+    assert torch.equal(out_p, out_c) and torch.equal(lse_p, lse_c), f"in-order pool, page {page_size} {layout}"
+    # swap two logical pages of sequence 0 (their tiles are no longer runs), keep the rest in order
+    a, b = 3, 17
+    bt = pg.block_table
+    pa, pb = int(bt[0, a]), int(bt[0, b])
+    for pool in (pg.k_pages, pg.v_pages):
+        tmp = pool[pa].clone()
+        pool[pa] = pool[pb]
+        pool[pb] = tmp
+    bt[0, a], bt[0, b] = pb, pa
+    out_m, lse_m = fd.decode_paged(x.q, pg.k_pages, pg.v_pages, bt, x.seqlens, x.scale, layout=layout, num_splits=S)
+    torch.cuda.synchronize()
+    assert torch.equal(out_m, out_c) and torch.equal(lse_m, lse_c), f"mixed pool, page {page_size} {layout}"
+
+
+@pytest.mark.parametrize("kv_type", ["e4m3", "int8"])
+@pytest.mark.parametrize("layout", ["HND", "NHD"])
+def test_consecutive_pages_one_box_8bit(kv_type, layout):
+    """The same for 8-bit page pools (16-token pages): an in-order pool gives
+    bitwise the contiguous 8-bit result."""
+    from decode_attention_07_b200.inputs import make_quant
+    w = Workload("paged", B=2, Hq=8, Hkv=2, D=128, Lmax=1500, ragged=False, nan_pad=True)
+    x = make_quant(w, kv_type, 21, device="cuda", seqlens=[1500, 333])
+    S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.Lmax)
+    out_c, lse_c = fd.decode_quant(x.q, x.k8, x.v8, x.k_scale, x.v_scale, kv_type, x.seqlens, x.scale, num_splits=S)
+    pg = make_paged(x, 16, layout, order="inorder")
+    out_p, lse_p = fd.decode_quant_paged(x.q, pg.k_pages, pg.v_pages, x.k_scale, x.v_scale, kv_type, pg.block_table,
+                                         x.seqlens, x.scale, layout=layout, num_splits=S)
+    torch.cuda.synchronize()
+    assert torch.equal(out_p, out_c) and torch.equal(lse_p, lse_c)
