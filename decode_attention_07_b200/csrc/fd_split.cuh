@@ -1136,7 +1136,9 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
                                     page[j4 + 3] = v4.w;
                                 }
                         } else {
-                            for (int j = 0; j < nsub; ++j) page[j] = wp[j];
+#pragma unroll
+                            for (int j = 0; j < kTileTokens / 8; ++j)
+                                if (j < nsub) page[j] = wp[j];
                         }
                     }
                     // small pages: when the tile's pages are consecutive pages of the pool
@@ -1159,7 +1161,7 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
                         uint8_t *dst = v_role ? vt : kt;
                         if (run)   // box {64, 2, page_size, 1, nsub} (head-major) or {64, 2, 1, page_size, nsub}
                             tma_load_5d(dst, rmap, &full[stage], 0, 0, cz, cw, page[0], policy);
-                        else
+                        else   // (a loop with constant indices measured slower here, unlike the 3-D boxes below)
                             for (int j = 0; j < nsub; ++j)
                                 tma_load_5d(dst + j * page_bytes, map, &full[stage], 0, 0, cz, cw, page[j], policy);
                     } else {
@@ -1183,7 +1185,9 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
                                                 policy);
                             }
                         } else
-                        for (int j = 0; j < nsub; ++j) {
+#pragma unroll
+                        for (int j = 0; j < kTileTokens / 8; ++j) {   // constant indices: page[] stays in registers
+                            if (j >= nsub) break;
                             const int pgj = psize >= kTileTokens ? page1 : page[j];
 #pragma unroll
                             for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
