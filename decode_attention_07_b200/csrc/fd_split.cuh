@@ -1123,7 +1123,7 @@ __global__ void __launch_bounds__(split_threads<kPaged>(), 1)
                             drain_copies<kStages>(full, seq, wbar, win_pending, win_phase);
                             return;
                         }
-                        const int *wp = win + (lp0 - win_lo);
+                        const int* wp = win + (lp0 - win_lo);
                         const int full_tile = kTileTokens >> p.page_shift;
                         if (nsub == full_tile && full_tile >= 4) {
 #pragma unroll
