@@ -4,6 +4,7 @@ computation runs in the library's CUDA kernels. There is no fallback: if the
 library is missing or a call fails, an exception is raised."""
 import ctypes
 import os
+import warnings
 
 import numpy as np
 import torch
@@ -36,6 +37,14 @@ _lib = None
 _i, _p, _sz, _f = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
 
 
+def _newer_sources(path: str) -> list:
+    """Sources of the library (decode_attention_07_b200.build.DEPS) modified
+    after the library at `path` was built; those not shipped are skipped."""
+    from .build import DEPS
+    t = os.path.getmtime(path)
+    return sorted(os.path.basename(d) for d in DEPS if os.path.exists(d) and os.path.getmtime(d) > t)
+
+
 def lib() -> ctypes.CDLL:
     """Load libfdecode.so (built in-tree by decode_attention_07_b200.build);
     with FD_DEBUG=1 in the environment, the debug build libfdecode_debug.so."""
@@ -44,6 +53,11 @@ def lib() -> ctypes.CDLL:
         path = DEBUG_LIBRARY if os.environ.get("FD_DEBUG", "0") not in ("", "0") else LIBRARY
         if not os.path.exists(path):
             raise RuntimeError(f"{path} is not built: run `python -c 'import __graft_entry__ as g; g.build()'`")
+        stale = _newer_sources(path)
+        if stale:
+            warnings.warn(f"{os.path.basename(path)} is older than {', '.join(stale)}: the loaded kernels may not be "
+                          "the sources' (rebuild with `python -c 'import __graft_entry__ as g; g.build()'`)",
+                          RuntimeWarning, stacklevel=2)
         L = ctypes.CDLL(path)
         L.fd_plan.argtypes = [_i] * 5
         L.fd_plan_for_sms.argtypes = [_i] * 6
