@@ -300,3 +300,14 @@ def test_segments_errors():
     assert L.fd_segments(2, 2, 10, lens.ctypes.data, 4, ptr, ptr, ptr, ptr, 4) == -11
     assert L.fd_segments(2, 2, 10, lens.ctypes.data, 0, ptr, ptr, ptr, ptr, 8) == -7
     assert L.fd_segments(2, 2, 10, None, 4, ptr, ptr, ptr, ptr, 8) == -1
+
+
+def test_stale_library_is_reported(tmp_path):
+    """A library file older than its sources is named by _newer_sources (the
+    binding then warns at load time); the in-tree build is not stale."""
+    old = tmp_path / "libold.so"
+    old.write_bytes(b"")
+    os.utime(old, (1, 1))
+    from decode_attention_07_b200.build import DEPS
+    assert _lib._newer_sources(str(old)) == sorted(os.path.basename(d) for d in DEPS if os.path.exists(d))
+    assert _lib._newer_sources(_lib.LIBRARY) == []
