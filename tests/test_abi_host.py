@@ -304,10 +304,13 @@ def test_segments_errors():
 
 def test_stale_library_is_reported(tmp_path):
     """A library file older than its sources is named by _newer_sources (the
-    binding then warns at load time); the in-tree build is not stale."""
-    old = tmp_path / "libold.so"
-    old.write_bytes(b"")
-    os.utime(old, (1, 1))
+    binding then warns at load time); one newer than all of them is not."""
     from decode_attention_07_b200.build import DEPS
-    assert _lib._newer_sources(str(old)) == sorted(os.path.basename(d) for d in DEPS if os.path.exists(d))
-    assert _lib._newer_sources(_lib.LIBRARY) == []
+    shipped = sorted(os.path.basename(d) for d in DEPS if os.path.exists(d))
+    lib = tmp_path / "libx.so"
+    lib.write_bytes(b"")
+    os.utime(lib, (1, 1))
+    assert _lib._newer_sources(str(lib)) == shipped
+    newest = max(os.path.getmtime(d) for d in DEPS if os.path.exists(d))
+    os.utime(lib, (newest + 10, newest + 10))
+    assert _lib._newer_sources(str(lib)) == []
