@@ -50,8 +50,11 @@
  *
  * OWNERSHIP AND ERRORS
  * Every pointer is owned by the caller; the library allocates nothing and
- * keeps no state between calls except a per-device cache of the SM count
- * and a per-device error word (see fd_device_status). Calls are
+ * keeps no state between calls except, per device, a cache of the SM count,
+ * an error word (see fd_device_status), a cache of the last 32 encoded TMA
+ * tensor maps (keyed by address, shape and box, so reusing a buffer skips the
+ * encode; a map describes memory, it owns none) and the fixed scratch buffer
+ * of fd_decode_static (a file-scope device array, not an allocation). Calls are
  * asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream)
  * and never synchronise, except fd_device_status. Every entry point returns
  * FD_OK (0) or a negative FD_ERR_* code; argument checks run before any CUDA
